@@ -1,0 +1,419 @@
+"""Oracle for UltraGen's hierarchical local attention (HLA). TEST INFRASTRUCTURE ONLY.
+
+A plain, slow, obviously-correct fp64 NumPy restatement of what the hot path computes.
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py`` (its cpu_baseline leg and its
+reference arm) may import or run this module.  It shares no code, table or helper with the
+CUDA library, and it imports nothing from the product package.
+
+Sources (page title, then the section on the page):
+  [UG-note]  "UltraGen: Efficient Ultra-High-Resolution Image Generation with Hierarchical
+             Local Attention" -- papernotes.org note (ECCV 2026), section 方法详解 / 关键设计 1-3
+             and the MMA equation under 关键设计 3.
+  [UG-gist]  same title -- gist.science English summary of arXiv 2510.16325, section
+             "2. Methodology", parts A (window-first permutation) and B (low-resolution
+             global guidance, "Attention Masking").
+
+What each function follows:
+  * geometry / window partition ............ [UG-note] 关键设计 1; [UG-gist] 2.A
+  * window-first permutation ............... [UG-note] 关键设计 1 (window-first token order)
+  * LR position scaling (m,n)->(rho m,rho n) [UG-note] 关键设计 2, the scaling equation
+  * sequence order [C_T; X; X_lr] .......... [UG-note] 关键设计 3
+  * visibility (mask M) .................... [UG-note] 关键设计 2 (last paragraph);
+                                             [UG-gist] 2.B "Attention Masking"
+  * masked softmax attention ............... [UG-note] 关键设计 3, the MMA equation
+  * 2D RoPE on Q/K ......................... implied by [UG-note] 关键设计 1 and 3 ("RoPE"),
+                                             convention fixed by the readings below
+
+Readings taken where the pages are silent or garbled (each is listed in the design doc):
+  R1  l counts latent tokens (l=16 <-> 256x256 pixels at a 16x VAE).
+  R2  Halo: the query's own window box grown by b tokens on every side, clipped to the
+      image; every query of a window sees the same set.  0 <= b <= l.
+  R3  HR queries see ALL low-resolution tokens.
+  R4  LR queries see LR and text.  R5 text queries see text and HR, not LR.
+  R6  The "* M" inside the softmax is read as an additive -inf on masked pairs; the
+      scale is 1/sqrt(head_dim).
+  R7  RoPE: interleaved pairs (2k, 2k+1); dims split into axes (a0, a1, a2) laid out
+      consecutively; pair k of an axis of width d rotates by pos * theta**(-2k/d);
+      theta = 1e4; axis 0 position is always 0; text tokens sit at (0, 0, 0).
+  R8  Sequence layout [text | pad | HR window-first | pad | LR | pad], every segment
+      starting on a multiple of 128; partial edge windows keep l*l slots (pad slots).
+  R9  H counts rows (axis 1 <- row i), W counts columns (axis 2 <- column j).
+  R13 Windows in row-major order; raster order inside a window.
+  R15 Pad slots are not tokens: never visible as keys; pad query rows output 0; tile lists
+      are derived from the mask rows of real tokens only.
+
+Parity status: every function here is pinned by ``tests/test_oracle_pins.py`` (brute force
+on tiny grids, closed forms, textbook special cases, invariants).  The pages print no
+numeric worked example for this method, so no value is pinned to a printed number except
+the closed forms the pages state (the 256x window reduction at 4K, rho = H/h).
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+import numpy as np
+
+TEXT, HR, LR, PAD = 0, 1, 2, -1
+TILE = 128
+
+
+def pad128(n: int) -> int:
+    return TILE * ((n + TILE - 1) // TILE)
+
+
+def cdiv(a: int, b: int) -> int:
+    return -(-a // b)
+
+
+@dataclass(frozen=True)
+class Geometry:
+    """Token geometry of one joint sequence [C_T; X; X_lr] ([UG-note] 关键设计 1-3)."""
+
+    H: int          # HR latent rows
+    W: int          # HR latent columns
+    l: int          # window side in latent tokens (R1)
+    b: int          # halo width in tokens (R2)
+    rho: int        # LR down-scale factor, rho = H / h ([UG-note] 关键设计 2); 0 = no LR
+    T: int          # text tokens
+
+    @property
+    def nWh(self) -> int:
+        return cdiv(self.H, self.l)
+
+    @property
+    def nWw(self) -> int:
+        return cdiv(self.W, self.l)
+
+    @property
+    def h(self) -> int:
+        return cdiv(self.H, self.rho) if self.rho > 0 else 0
+
+    @property
+    def w(self) -> int:
+        return cdiv(self.W, self.rho) if self.rho > 0 else 0
+
+    @property
+    def N_hr(self) -> int:
+        return self.H * self.W
+
+    @property
+    def N_lr(self) -> int:
+        return self.h * self.w
+
+    @property
+    def N_hrp(self) -> int:
+        return self.nWh * self.nWw * self.l * self.l
+
+    @property
+    def off_hr(self) -> int:
+        return pad128(self.T)
+
+    @property
+    def off_lr(self) -> int:
+        return self.off_hr + pad128(self.N_hrp)
+
+    @property
+    def N_tot(self) -> int:
+        return self.off_lr + pad128(self.N_lr)
+
+    @property
+    def N_raster(self) -> int:
+        return self.T + self.N_hr + self.N_lr
+
+
+# --------------------------------------------------------------------------------------
+# Tokens, raster order and the window-first permutation
+# --------------------------------------------------------------------------------------
+
+def raster_tokens(g: Geometry):
+    """Every token of [C_T; X; X_lr] in raster order: (segment, a, b) per token.
+
+    text t -> (TEXT, t, 0); HR (i, j) -> (HR, i, j); LR (m, n) -> (LR, m, n).
+    """
+    seg = np.empty(g.N_raster, np.int64)
+    ca = np.empty(g.N_raster, np.int64)
+    cb = np.empty(g.N_raster, np.int64)
+    r = 0
+    seg[r:r + g.T] = TEXT
+    ca[r:r + g.T] = np.arange(g.T)
+    cb[r:r + g.T] = 0
+    r += g.T
+    ii, jj = np.meshgrid(np.arange(g.H), np.arange(g.W), indexing="ij")
+    seg[r:r + g.N_hr] = HR
+    ca[r:r + g.N_hr] = ii.ravel()
+    cb[r:r + g.N_hr] = jj.ravel()
+    r += g.N_hr
+    mm, nn = np.meshgrid(np.arange(g.h), np.arange(g.w), indexing="ij")
+    seg[r:r + g.N_lr] = LR
+    ca[r:r + g.N_lr] = mm.ravel()
+    cb[r:r + g.N_lr] = nn.ravel()
+    return seg, ca, cb
+
+
+def slot_of_tokens(g: Geometry) -> np.ndarray:
+    """Permuted slot of every raster token (window-first order, [UG-note] 关键设计 1; R8, R13).
+
+    HR token (i, j) lies in window (i // l, j // l); windows are numbered row-major and
+    tokens inside a window are numbered in raster order.
+    """
+    seg, ca, cb = raster_tokens(g)
+    slot = np.empty(g.N_raster, np.int64)
+    t = seg == TEXT
+    slot[t] = ca[t]
+    hr = seg == HR
+    i, j = ca[hr], cb[hr]
+    window = (i // g.l) * g.nWw + (j // g.l)
+    slot[hr] = g.off_hr + window * g.l * g.l + (i % g.l) * g.l + (j % g.l)
+    lr = seg == LR
+    slot[lr] = g.off_lr + ca[lr] * g.w + cb[lr]
+    return slot
+
+
+def perm_map(g: Geometry) -> np.ndarray:
+    """pi: permuted slot -> raster index, -1 for pad slots."""
+    perm = np.full(g.N_tot, -1, np.int64)
+    perm[slot_of_tokens(g)] = np.arange(g.N_raster)
+    return perm
+
+
+def slot_info(g: Geometry):
+    """Per permuted slot: segment (PAD for pad slots) and the token's two coordinates."""
+    seg_r, ca_r, cb_r = raster_tokens(g)
+    perm = perm_map(g)
+    real = perm >= 0
+    seg = np.full(g.N_tot, PAD, np.int64)
+    ca = np.zeros(g.N_tot, np.int64)
+    cb = np.zeros(g.N_tot, np.int64)
+    seg[real] = seg_r[perm[real]]
+    ca[real] = ca_r[perm[real]]
+    cb[real] = cb_r[perm[real]]
+    return seg, ca, cb
+
+
+def permute(x: np.ndarray, g: Geometry) -> np.ndarray:
+    """Raster [B, N_raster, Hh, D] -> window-first [B, Hh, N_tot, D]; pad slots are zero."""
+    B, N, Hh, D = x.shape
+    assert N == g.N_raster
+    perm = perm_map(g)
+    out = np.zeros((B, Hh, g.N_tot, D), x.dtype)
+    real = perm >= 0
+    out[:, :, real, :] = np.transpose(x, (0, 2, 1, 3))[:, :, perm[real], :]
+    return out
+
+
+def unpermute(xp: np.ndarray, g: Geometry) -> np.ndarray:
+    """Window-first [B, Hh, N_tot, D] -> raster [B, N_raster, Hh, D]; pad slots dropped."""
+    B, Hh, N, D = xp.shape
+    assert N == g.N_tot
+    slot = slot_of_tokens(g)
+    return np.transpose(xp[:, :, slot, :], (0, 2, 1, 3)).copy()
+
+
+# --------------------------------------------------------------------------------------
+# Positions and 2D RoPE
+# --------------------------------------------------------------------------------------
+
+def positions(g: Geometry) -> np.ndarray:
+    """(p0, p1, p2) per raster token: text (0,0,0); HR (0,i,j); LR (0, rho*m, rho*n).
+
+    The LR scaling is the equation of [UG-note] 关键设计 2; the rest is R7/R9.
+    """
+    seg, ca, cb = raster_tokens(g)
+    pos = np.zeros((g.N_raster, 3), np.int64)
+    hr = seg == HR
+    pos[hr, 1] = ca[hr]
+    pos[hr, 2] = cb[hr]
+    lr = seg == LR
+    pos[lr, 1] = g.rho * ca[lr]
+    pos[lr, 2] = g.rho * cb[lr]
+    return pos
+
+
+def rope(x: np.ndarray, pos: np.ndarray, axes, theta: float = 1.0e4) -> np.ndarray:
+    """Axial RoPE in fp64 on x [B, N, Hh, D] with per-token positions pos [N, 3] (R7).
+
+    For axis a of width d_a starting at dim o_a, pair k = (o_a + 2k, o_a + 2k + 1) rotates
+    by phi = pos_a * theta**(-2k / d_a):  (x0, x1) -> (x0 cos phi - x1 sin phi,
+    x0 sin phi + x1 cos phi).
+    """
+    x = np.asarray(x, np.float64)
+    assert sum(axes) == x.shape[-1] and all(d % 2 == 0 for d in axes)
+    out = x.copy()
+    o = 0
+    for a, d in enumerate(axes):
+        k = np.arange(d // 2, dtype=np.float64)
+        omega = theta ** (-2.0 * k / d)
+        phi = pos[:, a].astype(np.float64)[:, None] * omega[None, :]      # [N, d/2]
+        c = np.cos(phi)[None, :, None, :]
+        s = np.sin(phi)[None, :, None, :]
+        x0 = x[..., o + 0:o + d:2]
+        x1 = x[..., o + 1:o + d:2]
+        out[..., o + 0:o + d:2] = x0 * c - x1 * s
+        out[..., o + 1:o + d:2] = x0 * s + x1 * c
+        o += d
+    return out
+
+
+# --------------------------------------------------------------------------------------
+# The mask M
+# --------------------------------------------------------------------------------------
+
+def window_box(g: Geometry, i: np.ndarray, j: np.ndarray):
+    """Halo box of the window holding HR token (i, j): [r0, r1) x [c0, c1) (R2)."""
+    wr, wc = i // g.l, j // g.l
+    r0 = np.maximum(0, wr * g.l - g.b)
+    r1 = np.minimum(g.H, (wr + 1) * g.l + g.b)
+    c0 = np.maximum(0, wc * g.l - g.b)
+    c1 = np.minimum(g.W, (wc + 1) * g.l + g.b)
+    return r0, r1, c0, c1
+
+
+def visible_rows(g: Geometry, q_slots: np.ndarray) -> np.ndarray:
+    """Explicit boolean mask rows M[q, :] over all N_tot key slots (R2-R5, R15).
+
+    text q -> text and HR keys;  HR q -> text, LR, and HR keys in its window's halo box;
+    LR q -> LR and text keys;  pad q -> nothing.  Pad keys are never visible.
+    """
+    seg, ca, cb = slot_info(g)
+    q_slots = np.asarray(q_slots, np.int64)
+    qs = seg[q_slots]
+    kseg = seg[None, :]
+    vis = np.zeros((len(q_slots), g.N_tot), bool)
+
+    t = qs == TEXT
+    vis[t] = ((kseg == TEXT) | (kseg == HR))[0]
+
+    lr = qs == LR
+    vis[lr] = ((kseg == LR) | (kseg == TEXT))[0]
+
+    hr = np.nonzero(qs == HR)[0]
+    if len(hr):
+        r0, r1, c0, c1 = window_box(g, ca[q_slots[hr]], cb[q_slots[hr]])
+        ki, kj = ca[None, :], cb[None, :]
+        in_box = ((kseg == HR) & (ki >= r0[:, None]) & (ki < r1[:, None])
+                  & (kj >= c0[:, None]) & (kj < c1[:, None]))
+        vis[hr] = in_box | (kseg == TEXT) | (kseg == LR)
+    return vis
+
+
+# --------------------------------------------------------------------------------------
+# Masked softmax attention ([UG-note] 关键设计 3, MMA equation; R6)
+# --------------------------------------------------------------------------------------
+
+def attention_rows(qp: np.ndarray, kp: np.ndarray, vp: np.ndarray, g: Geometry,
+                   rows: np.ndarray, heads=None, chunk: int = 256) -> np.ndarray:
+    """Dense fp64 masked softmax attention for selected permuted query rows.
+
+    qp, kp, vp: [B, Hh, N_tot, D] (already RoPE'd and permuted).  Returns [B, Hh', len(rows), D]
+    with heads' = ``heads`` (all by default).  Pad rows give 0.
+    """
+    B, Hh, N, D = qp.shape
+    heads = range(Hh) if heads is None else heads
+    rows = np.asarray(rows, np.int64)
+    out = np.zeros((B, len(list(heads)), len(rows), D), np.float64)
+    scale = 1.0 / math.sqrt(D)
+    for c0 in range(0, len(rows), chunk):
+        rr = rows[c0:c0 + chunk]
+        vis = visible_rows(g, rr)
+        any_vis = vis.any(axis=1)
+        for bi in range(B):
+            for hi, h in enumerate(heads):
+                K = np.asarray(kp[bi, h], np.float64)
+                V = np.asarray(vp[bi, h], np.float64)
+                q = np.asarray(qp[bi, h, rr], np.float64)
+                s = (q @ K.T) * scale
+                s = np.where(vis, s, -np.inf)
+                m = np.max(np.where(any_vis[:, None], s, 0.0), axis=1, keepdims=True)
+                p = np.exp(s - m)
+                p[~any_vis] = 0.0
+                den = p.sum(axis=1, keepdims=True)
+                den[~any_vis] = 1.0
+                p = p / den
+                ok = np.abs(p[any_vis].sum(axis=1) - 1.0) < 1e-12
+                assert ok.all(), "softmax rows must sum to 1"
+                out[bi, hi, c0:c0 + len(rr)] = p @ V
+    return out
+
+
+def forward(q: np.ndarray, k: np.ndarray, v: np.ndarray, g: Geometry, axes,
+            theta: float = 1.0e4, rows=None, heads=None):
+    """Whole path on raster inputs [B, N_raster, Hh, D]: RoPE -> permute -> attention.
+
+    Returns (O_rows [B, Hh', n, D] for the permuted ``rows`` (all slots by default),
+    rows).  Unpermute the full result with ``unpermute``.
+    """
+    pos = positions(g)
+    qr = rope(q, pos, axes, theta)
+    kr = rope(k, pos, axes, theta)
+    qp, kp, vp = permute(qr, g), permute(kr, g), permute(np.asarray(v, np.float64), g)
+    rows = np.arange(g.N_tot) if rows is None else np.asarray(rows, np.int64)
+    return attention_rows(qp, kp, vp, g, rows, heads=heads), rows
+
+
+# --------------------------------------------------------------------------------------
+# Tile lists derived from the explicit mask (R15)
+# --------------------------------------------------------------------------------------
+
+def qtile_entries(g: Geometry, t: int):
+    """Entries of query tile t: ascending key tiles with any visible (real row, col) cell;
+    bit 31 marks a partial tile (some real-row cell not visible).  Also returns the
+    per-entry row masks [n_entries, 128, 4] uint32 (bit c%32 of word c//32 = column c
+    visible for that row; rows of pad slots are 0)."""
+    perm = perm_map(g)
+    slots = np.arange(t * TILE, (t + 1) * TILE)
+    real = perm[slots] >= 0
+    nk = g.N_tot // TILE
+    vis = np.zeros((TILE, g.N_tot), bool)
+    if real.any():
+        vis[real] = visible_rows(g, slots[real])
+    blocks = vis.reshape(TILE, nk, TILE)
+    anyv = blocks[real].any(axis=(0, 2)) if real.any() else np.zeros(nk, bool)
+    allv = blocks[real].all(axis=(0, 2)) if real.any() else np.zeros(nk, bool)
+    ks = np.nonzero(anyv)[0]
+    entries = (ks.astype(np.uint64) | ((~allv[ks]).astype(np.uint64) << np.uint64(31)))
+    bits = blocks[:, ks, :].transpose(1, 0, 2).reshape(len(ks), TILE, 4, 32)
+    weights = (np.uint64(1) << np.arange(32, dtype=np.uint64))
+    words = (bits.astype(np.uint64) * weights).sum(axis=-1).astype(np.uint32)
+    return entries.astype(np.uint32), words
+
+
+def tile_lists(g: Geometry, qtiles=None):
+    """CSR over query tiles: (row_ptr, entries) as uint32, for the given q-tiles (all)."""
+    qtiles = range(g.N_tot // TILE) if qtiles is None else qtiles
+    row_ptr = [0]
+    ents = []
+    for t in qtiles:
+        e, _ = qtile_entries(g, t)
+        ents.append(e)
+        row_ptr.append(row_ptr[-1] + len(e))
+    entries = np.concatenate(ents) if ents else np.zeros(0, np.uint32)
+    return np.asarray(row_ptr, np.int64), entries
+
+
+def visible_pair_count(g: Geometry, chunk: int = 1024) -> int:
+    """Number of visible (query, key) pairs of one head, from the explicit mask."""
+    total = 0
+    for c0 in range(0, g.N_tot, chunk):
+        total += int(visible_rows(g, np.arange(c0, min(g.N_tot, c0 + chunk))).sum())
+    return total
+
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """Round fp64 values to the nearest bfloat16 (ties to even); returns fp64.
+
+    Works on the fp64 bit pattern so there is no double rounding through fp32.
+    Finite inputs only.
+    """
+    x = np.asarray(x, np.float64)
+    out = np.zeros_like(x)
+    nz = x != 0
+    xv = x[nz]
+    e = np.floor(np.log2(np.abs(xv)))
+    # guard against log2 rounding at exact powers of two
+    e = np.where(np.abs(xv) < 2.0 ** e, e - 1, e)
+    e = np.where(np.abs(xv) >= 2.0 ** (e + 1), e + 1, e)
+    e = np.maximum(e, -126.0)                 # below 2**-126 the ulp stays 2**-133
+    ulp = 2.0 ** (e - 7)
+    out[nz] = np.round(xv / ulp) * ulp        # np.round: ties to even
+    return out

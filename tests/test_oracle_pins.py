@@ -1,0 +1,419 @@
+"""Pins of the fp64 oracle against things other than itself.
+
+Brute force on tiny grids (pure-Python loops written from the rules, not from the
+oracle's vectorised formulas), textbook special cases (dense softmax attention from torch),
+closed forms, and invariants.  Every test here runs on the CPU.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import hla_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "page_claims.json")
+
+
+def claims():
+    with open(GOLDEN) as f:
+        return json.load(f)
+
+
+# ----------------------------------------------------------------------------------------
+# brute force, written from the rules with loops
+# ----------------------------------------------------------------------------------------
+
+def bf_tokens(H, W, rho, T):
+    toks = [("text", t, 0) for t in range(T)]
+    toks += [("hr", i, j) for i in range(H) for j in range(W)]
+    if rho:
+        h, w = math.ceil(H / rho), math.ceil(W / rho)
+        toks += [("lr", m, n) for m in range(h) for n in range(w)]
+    return toks
+
+
+def bf_slots(H, W, l, rho, T):
+    """Walk the permuted sequence slot by slot: text, pad to 128, windows row-major with
+    raster order inside, pad to 128, LR raster, pad to 128.  Returns list of token keys
+    (None for pad)."""
+    seq = [("text", t, 0) for t in range(T)]
+    while len(seq) % 128:
+        seq.append(None)
+    for wr in range(math.ceil(H / l)):
+        for wc in range(math.ceil(W / l)):
+            for di in range(l):
+                for dj in range(l):
+                    i, j = wr * l + di, wc * l + dj
+                    seq.append(("hr", i, j) if (i < H and j < W) else None)
+    while len(seq) % 128:
+        seq.append(None)
+    if rho:
+        h, w = math.ceil(H / rho), math.ceil(W / rho)
+        for m in range(h):
+            for n in range(w):
+                seq.append(("lr", m, n))
+    while len(seq) % 128:
+        seq.append(None)
+    return seq
+
+
+def bf_visible(qt, kt, l, b):
+    """Visibility of key token kt to query token qt (None = pad)."""
+    if qt is None or kt is None:
+        return False
+    qk, kk = qt[0], kt[0]
+    if qk == "text":
+        return kk in ("text", "hr")
+    if qk == "lr":
+        return kk in ("lr", "text")
+    # HR query: text, all LR, and HR keys within b of its window rectangle
+    if kk in ("text", "lr"):
+        return True
+    wr, wc = qt[1] // l, qt[2] // l
+    top, bottom = wr * l, (wr + 1) * l - 1
+    left, right = wc * l, (wc + 1) * l - 1
+    dr = max(0, top - kt[1], kt[1] - bottom)
+    dc = max(0, left - kt[2], kt[2] - right)
+    return dr <= b and dc <= b
+
+
+def bf_position(tok, rho):
+    kind, a, c = tok
+    if kind == "text":
+        return (0, 0, 0)
+    if kind == "hr":
+        return (0, a, c)
+    return (0, rho * a, rho * c)
+
+
+def bf_rope_vec(x, pos, axes, theta=1e4):
+    """Rotate one D-vector (list of floats) element pair by element pair."""
+    y = list(x)
+    base = 0
+    for a, d in enumerate(axes):
+        for k in range(d // 2):
+            ang = pos[a] / (theta ** (2.0 * k / d))
+            c, s = math.cos(ang), math.sin(ang)
+            x0, x1 = x[base + 2 * k], x[base + 2 * k + 1]
+            y[base + 2 * k] = x0 * c - x1 * s
+            y[base + 2 * k + 1] = x0 * s + x1 * c
+        base += d
+    return y
+
+
+def bf_forward(q, k, v, H, W, l, b, rho, T, axes):
+    """Pure-Python HLA on raster inputs [B, N, Hh, D]; returns raster output."""
+    toks = bf_tokens(H, W, rho, T)
+    B, N, Hh, D = q.shape
+    out = np.zeros((B, N, Hh, D))
+    for bi, hh in itertools.product(range(B), range(Hh)):
+        qr = [bf_rope_vec(q[bi, t, hh].tolist(), bf_position(tok, rho), axes) for t, tok in enumerate(toks)]
+        kr = [bf_rope_vec(k[bi, t, hh].tolist(), bf_position(tok, rho), axes) for t, tok in enumerate(toks)]
+        for t, tok in enumerate(toks):
+            logits = []
+            for u, utok in enumerate(toks):
+                if bf_visible(tok, utok, l, b):
+                    logits.append((u, sum(a * c for a, c in zip(qr[t], kr[u])) / math.sqrt(D)))
+            mx = max(s for _, s in logits)
+            wts = [(u, math.exp(s - mx)) for u, s in logits]
+            z = sum(wv for _, wv in wts)
+            for u, wv in wts:
+                out[bi, t, hh] += (wv / z) * v[bi, u, hh]
+    return out
+
+
+TINY_GEOMS = [
+    # H, W, l, b, rho, T, axes (D = sum(axes))
+    (8, 8, 4, 1, 4, 3, (4, 6, 6)),
+    (7, 10, 4, 2, 3, 5, (2, 4, 4)),
+    (5, 6, 3, 0, 2, 0, (2, 2, 4)),
+    (6, 9, 4, 4, 0, 2, (2, 2, 2)),
+]
+
+
+@pytest.mark.parametrize("geom", TINY_GEOMS)
+def test_perm_matches_slot_walk(geom):
+    H, W, l, b, rho, T, _ = geom
+    g = O.Geometry(H, W, l, b, rho, T)
+    seq = bf_slots(H, W, l, rho, T)
+    toks = bf_tokens(H, W, rho, T)
+    index = {tok: r for r, tok in enumerate(toks)}
+    expect = np.array([-1 if s is None else index[s] for s in seq])
+    assert len(seq) == g.N_tot
+    np.testing.assert_array_equal(O.perm_map(g), expect)
+
+
+@pytest.mark.parametrize("geom", TINY_GEOMS)
+def test_mask_matches_brute_force(geom):
+    H, W, l, b, rho, T, _ = geom
+    g = O.Geometry(H, W, l, b, rho, T)
+    seq = bf_slots(H, W, l, rho, T)
+    expect = np.array([[bf_visible(qt, kt, l, b) for kt in seq] for qt in seq])
+    got = O.visible_rows(g, np.arange(g.N_tot))
+    np.testing.assert_array_equal(got, expect)
+
+
+@pytest.mark.parametrize("geom", TINY_GEOMS)
+def test_forward_matches_brute_force(geom):
+    H, W, l, b, rho, T, axes = geom
+    g = O.Geometry(H, W, l, b, rho, T)
+    D = sum(axes)
+    rng = np.random.default_rng(7)
+    B, Hh = 2, 2
+    q, k, v = (rng.standard_normal((B, g.N_raster, Hh, D)) for _ in range(3))
+    expect = bf_forward(q, k, v, H, W, l, b, rho, T, axes)
+    o_perm, _ = O.forward(q, k, v, g, axes)
+    got = O.unpermute(o_perm, g)
+    np.testing.assert_allclose(got, expect, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("geom", TINY_GEOMS[:2])
+def test_tile_lists_match_brute_force(geom):
+    H, W, l, b, rho, T, _ = geom
+    g = O.Geometry(H, W, l, b, rho, T)
+    seq = bf_slots(H, W, l, rho, T)
+    nt = len(seq) // 128
+    row_ptr, entries = O.tile_lists(g)
+    ents = []
+    for qt in range(nt):
+        rows = [seq[qt * 128 + r] for r in range(128)]
+        real_rows = [r for r in rows if r is not None]
+        for kt in range(nt):
+            cols = [seq[kt * 128 + c] for c in range(128)]
+            cells = [bf_visible(r, c, l, b) for r in real_rows for c in cols]
+            if any(cells):
+                ents.append(kt | ((0 if all(cells) else 1) << 31))
+    np.testing.assert_array_equal(entries.astype(np.int64), np.array(ents, np.int64))
+
+
+# ----------------------------------------------------------------------------------------
+# textbook special cases
+# ----------------------------------------------------------------------------------------
+
+def sdpa(q, k, v):
+    """Plain softmax attention from torch for [N, Hh, D] fp64 tensors."""
+    qt, kt, vt = (torch.from_numpy(np.ascontiguousarray(np.transpose(x, (1, 0, 2)))) for x in (q, k, v))
+    o = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt)
+    return np.transpose(o.numpy(), (1, 0, 2))
+
+
+@pytest.mark.parametrize("H,W,l", [(12, 12, 12), (10, 7, 16), (9, 9, 64)])
+def test_one_window_is_dense_attention(H, W, l):
+    g = O.Geometry(H, W, l, 0, 0, 0)
+    axes = (4, 6, 6)
+    rng = np.random.default_rng(1)
+    q, k, v = (rng.standard_normal((1, g.N_raster, 3, 16)) for _ in range(3))
+    o_perm, _ = O.forward(q, k, v, g, axes)
+    got = O.unpermute(o_perm, g)[0]
+    pos = O.positions(g)
+    qr, kr = O.rope(q, pos, axes)[0], O.rope(k, pos, axes)[0]
+    np.testing.assert_allclose(got, sdpa(qr, kr, v[0]), atol=1e-12)
+
+
+def test_b0_windows_are_independent():
+    H, W, l = 12, 8, 4
+    g = O.Geometry(H, W, l, 0, 0, 0)
+    axes = (2, 4, 4)
+    rng = np.random.default_rng(2)
+    q, k, v = (rng.standard_normal((1, g.N_raster, 2, 10)) for _ in range(3))
+    got = O.unpermute(O.forward(q, k, v, g, axes)[0], g)[0]
+    pos = O.positions(g)
+    qr, kr = O.rope(q, pos, axes)[0], O.rope(k, pos, axes)[0]
+    for wr in range(H // l):
+        for wc in range(W // l):
+            idx = [i * W + j for i in range(wr * l, wr * l + l) for j in range(wc * l, wc * l + l)]
+            np.testing.assert_allclose(got[idx], sdpa(qr[idx], kr[idx], v[0][idx]), atol=1e-12)
+
+
+def test_single_visible_key_returns_its_value():
+    g = O.Geometry(6, 5, 1, 0, 0, 0)           # every token is its own window
+    rng = np.random.default_rng(3)
+    q, k, v = (rng.standard_normal((1, g.N_raster, 2, 8)) for _ in range(3))
+    got = O.unpermute(O.forward(q, k, v, g, (2, 2, 4))[0], g)
+    np.testing.assert_allclose(got, v, atol=1e-14)
+
+
+def test_constant_value_gives_constant_output():
+    g = O.Geometry(16, 12, 8, 2, 4, 5)
+    rng = np.random.default_rng(4)
+    q, k = (rng.standard_normal((1, g.N_raster, 2, 16)) for _ in range(2))
+    v = np.full((1, g.N_raster, 2, 16), 0.375)
+    got = O.unpermute(O.forward(q, k, v, g, (4, 6, 6))[0], g)
+    np.testing.assert_allclose(got, 0.375, atol=1e-14)
+
+
+def test_pad_rows_are_zero():
+    g = O.Geometry(9, 7, 4, 1, 3, 5)
+    rng = np.random.default_rng(5)
+    q, k, v = (rng.standard_normal((1, g.N_raster, 1, 8)) for _ in range(3))
+    o_perm, _ = O.forward(q, k, v, g, (2, 2, 4))
+    pad = O.perm_map(g) < 0
+    assert pad.any()
+    assert np.all(o_perm[:, :, pad, :] == 0)
+
+
+# ----------------------------------------------------------------------------------------
+# permutation and positions
+# ----------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("geom", TINY_GEOMS + [(256, 135, 16, 16, 4, 256, (2, 2, 2))])
+def test_permute_roundtrip_and_bijection(geom):
+    H, W, l, b, rho, T, _ = geom
+    g = O.Geometry(H, W, l, b, rho, T)
+    perm = O.perm_map(g)
+    real = perm[perm >= 0]
+    assert sorted(real.tolist()) == list(range(g.N_raster))
+    x = np.random.default_rng(0).standard_normal((2, g.N_raster, 3, 4)).astype(np.float32)
+    assert np.array_equal(O.unpermute(O.permute(x, g), g), x)
+
+
+def test_lr_positions_are_scaled_by_rho():
+    c = claims()
+    rho = c["rho_default"]["value"]
+    g = O.Geometry(33, 18, 16, 4, rho, 7)
+    pos = O.positions(g)
+    r = g.T + g.H * g.W
+    for m in range(g.h):
+        for n in range(g.w):
+            assert tuple(pos[r]) == (0, rho * m, rho * n)
+            r += 1
+    assert g.h == math.ceil(33 / rho) and g.w == math.ceil(18 / rho)
+
+
+# ----------------------------------------------------------------------------------------
+# RoPE
+# ----------------------------------------------------------------------------------------
+
+AXES = (16, 56, 56)
+
+
+def test_rope_matches_per_element_closed_form():
+    rng = np.random.default_rng(8)
+    x = rng.standard_normal((1, 5, 1, 128))
+    pos = np.array([[0, 0, 0], [0, 3, 7], [0, 255, 1], [0, 12, 300], [0, 64, 64]])
+    got = O.rope(x, pos, AXES)
+    for t in range(5):
+        np.testing.assert_allclose(got[0, t, 0], bf_rope_vec(x[0, t, 0].tolist(), pos[t], AXES), atol=1e-13)
+
+
+def test_rope_unit_vector_angle():
+    # pair k of axis 1 applied to e0 = (1, 0) gives (cos phi, sin phi), phi = p / 1e4^(2k/56)
+    x = np.zeros((1, 1, 1, 128))
+    k, p = 5, 11
+    x[0, 0, 0, 16 + 2 * k] = 1.0
+    got = O.rope(x, np.array([[0, p, 0]]), AXES)[0, 0, 0]
+    phi = p * 10000.0 ** (-2 * k / 56)
+    assert got[16 + 2 * k] == pytest.approx(math.cos(phi), abs=1e-15)
+    assert got[16 + 2 * k + 1] == pytest.approx(math.sin(phi), abs=1e-15)
+
+
+def test_rope_invariants():
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal((1, 64, 2, 128))
+    y = rng.standard_normal((1, 64, 2, 128))
+    pos = rng.integers(0, 400, size=(64, 3))
+    pos[:, 0] = 0
+    xr = O.rope(x, pos, AXES)
+    # norm of each pair is preserved
+    np.testing.assert_allclose(np.hypot(xr[..., 0::2], xr[..., 1::2]), np.hypot(x[..., 0::2], x[..., 1::2]), rtol=1e-12)
+    # position 0 is the identity
+    np.testing.assert_array_equal(O.rope(x, np.zeros_like(pos), AXES), x)
+    # logits depend only on relative position: shift every position by the same offset
+    shift = np.array([0, 17, 23])
+    a = np.einsum("bnhd,bmhd->bhnm", O.rope(x, pos, AXES), O.rope(y, pos, AXES))
+    c = np.einsum("bnhd,bmhd->bhnm", O.rope(x, pos + shift, AXES), O.rope(y, pos + shift, AXES))
+    np.testing.assert_allclose(a, c, atol=1e-9)
+    # rotations compose
+    p2 = rng.integers(0, 50, size=(64, 3))
+    p2[:, 0] = 0
+    np.testing.assert_allclose(O.rope(O.rope(x, pos, AXES), p2, AXES), O.rope(x, pos + p2, AXES), atol=1e-11)
+
+
+# ----------------------------------------------------------------------------------------
+# pair counts: closed forms and the pages' numbers
+# ----------------------------------------------------------------------------------------
+
+def closed_form_pairs(H, W, l, b, rho, T):
+    """Visible pairs of one head, segment by segment, from closed forms."""
+    h = math.ceil(H / rho) if rho else 0
+    w = math.ceil(W / rho) if rho else 0
+    Nhr, Nlr = H * W, h * w
+
+    def axis_sum(n):
+        s = 0
+        for wi in range(math.ceil(n / l)):
+            rows_in = min(n, (wi + 1) * l) - wi * l
+            box = min(n, (wi + 1) * l + b) - max(0, wi * l - b)
+            s += rows_in * box
+        return s
+
+    return {
+        "hr_hr": axis_sum(H) * axis_sum(W),
+        "hr_text": Nhr * T, "hr_lr": Nhr * Nlr,
+        "text_text": T * T, "text_hr": T * Nhr,
+        "lr_lr": Nlr * Nlr, "lr_text": Nlr * T,
+    }
+
+
+@pytest.mark.parametrize("geom", [(32, 32, 8, 2, 4, 16), (64, 64, 16, 4, 4, 512), (40, 27, 16, 16, 4, 64), (19, 23, 8, 3, 3, 9)])
+def test_pair_count_equals_closed_form(geom):
+    g = O.Geometry(*geom)
+    assert O.visible_pair_count(g) == sum(closed_form_pairs(*geom).values())
+
+
+def test_window_reduction_at_4k_is_256():
+    c = claims()
+    l = c["window_side_tokens"]["value"]
+    n4k = c["tokens_4k"]["value"]
+    side = int(math.isqrt(n4k))
+    # b = 0, HR only: the oracle's mask count equals N*l^2 on a grid the mask can hold,
+    g_small = O.Geometry(64, 64, l, 0, 0, 0)
+    assert O.visible_pair_count(g_small) == 64 * 64 * l * l
+    # so at 4K the local-window cut against dense attention is N^2 / (N l^2)
+    pairs = sum(closed_form_pairs(side, side, l, 0, 0, 0).values())
+    assert pairs == n4k * l * l
+    assert n4k * n4k // pairs == c["window_reduction_4k"]["value"]
+    # and dense attention grows 256x from 1K to 4K
+    assert (n4k / c["tokens_1k"]["value"]) ** 2 == c["full_attention_growth_1k_to_4k"]["value"]
+
+
+def test_halo_overhead_against_the_pages_bound():
+    """The pages bound the halo's extra compute by 2%.  Under these readings (all LR visible,
+    b = 4) the bound holds at 8K and not at 4K; both values are pinned here."""
+    bound = claims()["halo_overhead_bound"]["value"]
+
+    def overhead(side):
+        with_halo = closed_form_pairs(side, side, 16, 4, 4, 512)
+        no_halo = closed_form_pairs(side, side, 16, 0, 4, 512)
+        # extra pairs the halo adds, relative to the layer's pairs without it
+        return (with_halo["hr_hr"] - no_halo["hr_hr"]) / sum(no_halo.values())
+
+    assert overhead(512) < bound
+    assert overhead(512) == pytest.approx(80_756_736 / 4_907_597_824, rel=1e-12)
+    assert overhead(256) == pytest.approx(19_415_040 / 371_458_048, rel=1e-12)
+    assert overhead(256) > bound
+
+
+# ----------------------------------------------------------------------------------------
+# bf16 rounding helper
+# ----------------------------------------------------------------------------------------
+
+def test_round_bf16_matches_torch_on_fp32_values():
+    rng = np.random.default_rng(10)
+    x = np.concatenate([rng.standard_normal(20000) * 10.0 ** rng.integers(-30, 30, 20000),
+                        [0.0, 1.0, -1.0, 1.00390625, 1.01171875, 3e-39]]).astype(np.float32)
+    expect = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(O.round_bf16(x.astype(np.float64)), expect)
+
+
+def test_round_bf16_ties_and_no_double_rounding():
+    # 1 + 2^-8 is a tie between 1 and 1 + 2^-7: even mantissa (1) wins
+    assert O.round_bf16(np.array([1.0 + 2.0 ** -8]))[0] == 1.0
+    # 1 + 2^-8 + 2^-30 is just above the tie: rounds up (an fp32 detour would not see it
+    # if the extra bit were below fp32 precision; here 2^-30 is kept by fp64)
+    assert O.round_bf16(np.array([1.0 + 2.0 ** -8 + 2.0 ** -30]))[0] == 1.0 + 2.0 ** -7
+    assert O.round_bf16(np.array([1.0 + 2.0 ** -8 + 2.0 ** -40]))[0] == 1.0 + 2.0 ** -7
