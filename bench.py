@@ -1,0 +1,343 @@
+"""Benchmark of the HLA hot path: permute_rope -> hla_forward (+ split combine) -> unpermute.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 4k|8k|1k|ragged]
+                    [--impl ultragen|reference]
+
+One step is one pass of the whole path over one layer of synthetic Q/K/V (resident in HBM).
+The metric is useful TFLOP/s: 4 * head_dim FLOPs per visible (query, key) pair per head
+(masked pairs and padding count for nothing), whole job over all ranks; ms per step and per
+kernel are reported beside it.  Multi-GPU runs are weak scaling: every rank runs its own
+independent layer (no collective on the data path); timing is the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the plain restatement the tests check against) on
+a bounded row sample of the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ms/layer and useful TFLOP/s of masked HLA at 4K/8K; % of B200 BF16 tensor peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "hla_fwd_traffic.json")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="4k")
+    ap.add_argument("--impl", default="ultragen", choices=["ultragen", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() in ("active", "1", "0x1"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("hla_fwd.cu", "ptx.cuh", "kernels.h"):
+        with open(os.path.join(ROOT, "diffusion_transformer_ultra_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per hla_forward launch from the committed ncu summary, only while the kernel
+    source still matches the one the counters were taken on."""
+    if not os.path.exists(PROFILE_TRAFFIC):
+        return None
+    with open(PROFILE_TRAFFIC) as f:
+        d = json.load(f)
+    ent = d.get(workload)
+    if not ent or ent.get("kernel_sha") != kernel_source_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+def cpu_baseline(wl, q, k, v, budget_s: float = 12.0):
+    """The oracle as it stands, timed on this host on a bounded sample: one head, rows of one
+    interior window plus text and LR rows, growing until about `budget_s` of CPU work."""
+    import numpy as np
+
+    from oracle import hla_oracle as O
+    g = O.Geometry(wl.H, wl.W, wl.l, wl.b, wl.rho, wl.T)
+    l2 = g.l * g.l
+    win = (g.nWh // 2) * g.nWw + g.nWw // 2
+    rows = list(range(g.off_hr + win * l2, g.off_hr + (win + 1) * l2))
+    rows += list(range(0, min(g.T, 8)))
+    if g.N_lr:
+        rows += list(np.linspace(g.off_lr, g.off_lr + g.N_lr - 1, 32).astype(int))
+    rows = np.array(sorted(set(rows)), np.int64)
+    vis_pairs = int(O.visible_rows(g, rows).sum())
+    qh, kh, vh = (x[:1, :, :1, :].to(dtype=__import__("torch").float64).numpy() for x in (q, k, v))
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        O.forward(qh, kh, vh, g, wl.axes, rows=rows)
+        reps += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = (time.perf_counter() - t0) / reps
+    flops = 4.0 * wl.D * vis_pairs
+    return {"value": flops / dt / 1e12, "unit": "useful TFLOP/s", "cores": os.cpu_count(),
+            "kind": "oracle",
+            "sample": f"1 head, {len(rows)} query rows ({vis_pairs} visible pairs), full RoPE + "
+                      f"explicit mask, fp64 NumPy; {reps} rep(s), {dt:.2f} s each"}
+
+
+def run_reference(args, rank, world):
+    import torch
+    if rank != 0:
+        return
+    import diffusion_transformer_ultra_b200 as ug
+    wl = ug.WORKLOADS[args.workload]
+    q, k, v = ug.make_qkv(wl)
+    per_step = []
+    base = None
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        r = cpu_baseline(wl, q, k, v, budget_s=0.0)
+        if i >= args.warmup:
+            per_step.append(time.perf_counter() - t0)
+            base = r
+    value = base["value"]
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "useful TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * statistics.mean(per_step), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "H": wl.H, "W": wl.W, "l": wl.l, "b": wl.b, "rho": wl.rho,
+                   "text_len": wl.T, "heads": wl.heads, "head_dim": wl.D, "batch": wl.batch},
+        "cpu_baseline": {"kind": "oracle", "cores": base["cores"], "sample": base["sample"],
+                         "value": value, "unit": "useful TFLOP/s"},
+        "e2e": {"value": value, "unit": "useful TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import diffusion_transformer_ultra_b200 as ug
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    wl = ug.WORKLOADS[args.workload]
+    plan = ug.plan_for(wl)
+    info = plan.info
+    q, k, v = ug.make_qkv(wl)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    lay = ug.Layer(plan, wl.batch)
+    o = torch.empty((wl.batch, info["N_raster"], wl.heads, wl.D), dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        ug.permute_rope(qd, kd, vd, lay.qp, lay.kp, lay.vp, plan)
+        n = 1
+        if evs:
+            evs[1].record(stream)
+        ug.hla_forward(lay.qp, lay.kp, lay.vp, lay.op, plan)
+        n += plan.last_launch_count()
+        if evs:
+            evs[2].record(stream)
+        ug.unpermute(lay.op, o, plan)
+        n += 1
+        if evs:
+            evs[3].record(stream)
+        return n
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if plan.sync_status() != 0:
+        raise RuntimeError("device error during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    launches = 0
+    start.record(stream)
+    for i in range(args.steps):
+        launches += step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    if plan.sync_status() != 0:
+        raise RuntimeError("device error during the timed steps")
+    ms_total = start.elapsed_time(end)
+    ms_perm = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    ms_attn = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    ms_unperm = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    t = torch.tensor([ms_total], device="cuda")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_step = float(t.item()) / args.steps
+
+    flops = 4.0 * wl.D * info["useful_pairs"] * wl.heads * wl.batch
+    value = flops * world / (ms_step * 1e-3) / 1e12
+    pk, src = peaks()
+    attn_tflops = flops / (ms_attn * 1e-3) / 1e12
+    peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    elem = wl.batch * wl.heads * info["N_tot"] * wl.D
+    perm_bytes = 3 * (wl.batch * info["N_raster"] * wl.heads * wl.D * (2 if wl.dtype == "bf16" else 4)) + 3 * elem * 2
+    unperm_bytes = elem * 2 + wl.batch * info["N_raster"] * wl.heads * wl.D * 2
+    traffic = profiled_traffic(wl.name)
+
+    e2e = None
+    if not args.no_e2e:
+        qh, kh, vh = (x.pin_memory() for x in (q, k, v))
+        oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        for _ in range(2):
+            qd.copy_(qh, non_blocking=True); kd.copy_(kh, non_blocking=True); vd.copy_(vh, non_blocking=True)
+            step()
+            oh.copy_(o, non_blocking=True)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(3, args.steps // 4)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            qd.copy_(qh, non_blocking=True); kd.copy_(kh, non_blocking=True); vd.copy_(vh, non_blocking=True)
+            step()
+            oh.copy_(o, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        t2 = torch.tensor([e0.elapsed_time(e1) / n_e2e], device="cuda")
+        if world > 1:
+            dist.all_reduce(t2, op=dist.ReduceOp.MAX)
+        ms_e2e = float(t2.item())
+        e2e = {"value": flops * world / (ms_e2e * 1e-3) / 1e12, "unit": "useful TFLOP/s",
+               "ms_per_step": ms_e2e,
+               "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
+               "d2h_bytes_per_step": o.numel() * o.element_size()}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, q, k, v)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "useful TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) + smooth 2D sinusoid Q/K/V; no weights needed)",
+            "config": {"workload": wl.name, "H": wl.H, "W": wl.W, "l": wl.l, "b": wl.b,
+                       "rho": wl.rho, "text_len": wl.T, "heads": wl.heads, "head_dim": wl.D,
+                       "batch": wl.batch, "N_tot": info["N_tot"], "useful_pairs_per_head": info["useful_pairs"],
+                       "l2": "inputs larger than L2 (Q, K, V permuted: 3 x %.0f MB); no flush" % (elem * 2 / 1e6),
+                       "parallelism": f"independent layer per rank x{world}"},
+            "ms_per_kernel": {"permute_rope": ms_perm, "hla_forward": ms_attn, "unpermute": ms_unperm},
+            "hla_forward_tflops": attn_tflops,
+            "permute_rope_gbs": perm_bytes / (ms_perm * 1e-3) / 1e9,
+            "unpermute_gbs": unperm_bytes / (ms_unperm * 1e-3) / 1e9,
+            "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
+                         "frac": attn_tflops / peak, "traffic": traffic,
+                         "peak_source": f"{src} bf16 dense, sustained (kernel timed inside a repeated step)",
+                         "algorithmic_flops_per_launch": flops},
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

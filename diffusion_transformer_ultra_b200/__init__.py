@@ -1,0 +1,16 @@
+"""UltraGen hierarchical local attention (HLA) hot path for NVIDIA B200 (sm_100a).
+
+The compute lives in ``libultragen.so`` (hand-written CUDA behind a C ABI, see
+``include/ultragen.h``); this package holds its ctypes binding, the in-tree build script and
+the seeded synthetic-input generator.
+"""
+from ._ffi import (BF16, F32, Layer, Plan, UltragenError, hla_forward, lib,  # noqa: F401
+                   permute_rope, unpermute)
+from .inputs import WORKLOADS, Workload, make_qkv  # noqa: F401
+
+
+def plan_for(wl: "Workload") -> "Plan":
+    """Plan for one of the named workloads (geometry, heads, head_dim and RoPE axes)."""
+    p = Plan(wl.H, wl.W, wl.l, wl.b, wl.rho, wl.T, wl.heads, wl.D)
+    p.set_rope(wl.axes)
+    return p

@@ -1,0 +1,237 @@
+"""ctypes binding of libultragen.so: argument marshalling only.
+
+Every step of the hot path runs in the library's CUDA kernels; this module checks shapes,
+dtypes and devices of torch tensors and passes raw pointers.  There is no fallback: if the
+library is missing the import of any entry point raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libultragen.so")
+
+OK = 0
+STATUS = {
+    0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "CUDA error",
+    4: "out of memory", 5: "device wait timed out", 6: "plan does not match the call",
+    7: "no sm_100 device",
+}
+BF16, F32 = 0, 1
+
+# exported names of include/ultragen.h
+SYMBOLS = (
+    "ultragen_status_string", "ultragen_plan", "ultragen_plan_set_rope", "ultragen_plan_set_split",
+    "ultragen_plan_info", "ultragen_plan_export", "ultragen_plan_export_rowmasks",
+    "ultragen_plan_destroy", "ultragen_permute_rope", "ultragen_hla_forward",
+    "ultragen_unpermute", "ultragen_sync_status", "ultragen_last_launch_count",
+)
+
+
+class PlanInfo(ctypes.Structure):
+    _fields_ = [
+        ("H", ctypes.c_int32), ("W", ctypes.c_int32), ("l", ctypes.c_int32), ("b", ctypes.c_int32),
+        ("rho", ctypes.c_int32), ("text_len", ctypes.c_int32), ("heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32), ("nWh", ctypes.c_int32), ("nWw", ctypes.c_int32),
+        ("h", ctypes.c_int32), ("w", ctypes.c_int32), ("N_raster", ctypes.c_int64),
+        ("N_tot", ctypes.c_int64), ("off_hr", ctypes.c_int64), ("off_lr", ctypes.c_int64),
+        ("n_qtiles", ctypes.c_int32), ("n_items", ctypes.c_int32), ("n_entries", ctypes.c_int64),
+        ("n_partial", ctypes.c_int64), ("useful_pairs", ctypes.c_int64),
+        ("rope_axes", ctypes.c_int32 * 3), ("rope_theta", ctypes.c_double),
+        ("split_chunk", ctypes.c_int32), ("n_split_groups", ctypes.c_int32),
+        ("n_split_items", ctypes.c_int32), ("workspace_bytes_per_head", ctypes.c_int64),
+    ]
+
+    def as_dict(self):
+        d = {f: getattr(self, f) for f, _ in self._fields_}
+        d["rope_axes"] = tuple(self.rope_axes)
+        return d
+
+
+class UltragenError(RuntimeError):
+    def __init__(self, what: str, status: int):
+        super().__init__(f"{what} failed: {STATUS.get(status, status)} (status {status})")
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load the in-tree library (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m diffusion_transformer_ultra_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, cint = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int
+    L.ultragen_status_string.restype = ctypes.c_char_p
+    L.ultragen_status_string.argtypes = [cint]
+    L.ultragen_plan.argtypes = [cint] * 8 + [ctypes.POINTER(vp)]
+    L.ultragen_plan_set_rope.argtypes = [vp, cint, cint, cint, ctypes.c_double]
+    L.ultragen_plan_set_split.argtypes = [vp, cint]
+    L.ultragen_plan_info.argtypes = [vp, ctypes.POINTER(PlanInfo)]
+    L.ultragen_plan_export.argtypes = [vp, vp, vp, vp]
+    L.ultragen_plan_export_rowmasks.argtypes = [vp, cint, vp]
+    L.ultragen_plan_destroy.argtypes = [vp]
+    L.ultragen_permute_rope.argtypes = [vp, vp, vp, cint, vp, vp, vp, cint, vp, vp]
+    L.ultragen_hla_forward.argtypes = [vp, vp, vp, vp, vp, cint, vp]
+    L.ultragen_unpermute.argtypes = [vp, vp, cint, cint, vp, vp]
+    L.ultragen_sync_status.argtypes = [vp, vp]
+    L.ultragen_last_launch_count.argtypes = [vp]
+    for name in SYMBOLS:
+        if name != "ultragen_status_string":
+            getattr(L, name).restype = cint
+    _lib = L
+    return L
+
+
+def _check(what: str, st: int):
+    if st != OK:
+        raise UltragenError(what, st)
+
+
+class Plan:
+    """Owner of one ultragen_plan_t."""
+
+    def __init__(self, H, W, l, b, rho, text_len, heads, head_dim):
+        self._h = ctypes.c_void_p()
+        _check("ultragen_plan", lib().ultragen_plan(H, W, l, b, rho, text_len, heads, head_dim,
+                                                    ctypes.byref(self._h)))
+        self._refresh()
+
+    def _refresh(self):
+        info = PlanInfo()
+        _check("ultragen_plan_info", lib().ultragen_plan_info(self._h, ctypes.byref(info)))
+        self.info = info.as_dict()
+
+    @property
+    def handle(self):
+        return self._h
+
+    def set_rope(self, axes, theta=1.0e4):
+        _check("ultragen_plan_set_rope", lib().ultragen_plan_set_rope(self._h, *axes, float(theta)))
+        self._refresh()
+
+    def set_split(self, chunk: int):
+        _check("ultragen_plan_set_split", lib().ultragen_plan_set_split(self._h, int(chunk)))
+        self._refresh()
+
+    def export(self):
+        i = self.info
+        perm = np.empty(i["N_tot"], np.int32)
+        row_ptr = np.empty(i["n_qtiles"] + 1, np.int32)
+        entries = np.empty(max(1, i["n_entries"]), np.int32)
+        _check("ultragen_plan_export", lib().ultragen_plan_export(
+            self._h, perm.ctypes.data, row_ptr.ctypes.data, entries.ctypes.data))
+        return perm, row_ptr, entries[:i["n_entries"]]
+
+    def rowmasks(self, qtile: int, n_entries: int):
+        out = np.empty((max(1, n_entries), 128, 4), np.uint32)
+        _check("ultragen_plan_export_rowmasks",
+               lib().ultragen_plan_export_rowmasks(self._h, int(qtile), out.ctypes.data))
+        return out[:n_entries]
+
+    def sync_status(self, stream=None) -> int:
+        return lib().ultragen_sync_status(self._h, _stream_ptr(stream))
+
+    def last_launch_count(self) -> int:
+        return lib().ultragen_last_launch_count(self._h)
+
+    def close(self):
+        if self._h:
+            lib().ultragen_plan_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def _stream_ptr(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t, shape, dtypes, name):
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name} has dtype {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def permute_rope(q, k, v, qp, kp, vp, plan: Plan, stream=None):
+    """Raster Q/K/V [B, N_raster, H, D] -> window-first [B, H, N_tot, D] bf16 with RoPE on Q, K."""
+    import torch
+    i = plan.info
+    B = q.shape[0]
+    raster = (B, i["N_raster"], i["heads"], i["head_dim"])
+    perm_shape = (B, i["heads"], i["N_tot"], i["head_dim"])
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, raster, (torch.bfloat16, torch.float32), n)
+    if not (q.dtype == k.dtype == v.dtype):
+        raise ValueError("q, k, v must share a dtype")
+    for t, n in ((qp, "qp"), (kp, "kp"), (vp, "vp")):
+        _need(t, perm_shape, (torch.bfloat16,), n)
+    dt = BF16 if q.dtype == torch.bfloat16 else F32
+    _check("ultragen_permute_rope", lib().ultragen_permute_rope(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), dt, qp.data_ptr(), kp.data_ptr(), vp.data_ptr(),
+        B, plan.handle, _stream_ptr(stream)))
+
+
+def hla_forward(qp, kp, vp, op, plan: Plan, stream=None):
+    """Block-sparse masked attention over the window-first layout."""
+    import torch
+    i = plan.info
+    B = qp.shape[0]
+    shape = (B, i["heads"], i["N_tot"], i["head_dim"])
+    for t, n in ((qp, "qp"), (kp, "kp"), (vp, "vp"), (op, "op")):
+        _need(t, shape, (torch.bfloat16,), n)
+    _check("ultragen_hla_forward", lib().ultragen_hla_forward(
+        qp.data_ptr(), kp.data_ptr(), vp.data_ptr(), op.data_ptr(), plan.handle, B,
+        _stream_ptr(stream)))
+
+
+def unpermute(op, o, plan: Plan, stream=None):
+    """Window-first [B, H, N_tot, D] bf16 -> raster [B, N_raster, H, D] (bf16 or fp32)."""
+    import torch
+    i = plan.info
+    B = op.shape[0]
+    _need(op, (B, i["heads"], i["N_tot"], i["head_dim"]), (torch.bfloat16,), "op")
+    _need(o, (B, i["N_raster"], i["heads"], i["head_dim"]), (torch.bfloat16, torch.float32), "o")
+    dt = BF16 if o.dtype == torch.bfloat16 else F32
+    _check("ultragen_unpermute", lib().ultragen_unpermute(
+        op.data_ptr(), o.data_ptr(), dt, B, plan.handle, _stream_ptr(stream)))
+
+
+class Layer:
+    """The whole path for one shape: permute_rope -> hla_forward -> unpermute, with the
+    permuted buffers kept resident between calls."""
+
+    def __init__(self, plan: Plan, batch: int, device="cuda"):
+        import torch
+        i = plan.info
+        self.plan = plan
+        shape = (batch, i["heads"], i["N_tot"], i["head_dim"])
+        self.qp, self.kp, self.vp, self.op = (torch.empty(shape, dtype=torch.bfloat16, device=device)
+                                              for _ in range(4))
+
+    def __call__(self, q, k, v, o, stream=None):
+        permute_rope(q, k, v, self.qp, self.kp, self.vp, self.plan, stream)
+        hla_forward(self.qp, self.kp, self.vp, self.op, self.plan, stream)
+        unpermute(self.op, o, self.plan, stream)
+        return o

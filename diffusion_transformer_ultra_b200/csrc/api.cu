@@ -1,0 +1,309 @@
+// C entry points that touch the device: plan table upload, tensor-map creation, launches,
+// error read-back.  Host-only entry points live in plan.cpp.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "kernels.h"
+#include "plan_internal.h"
+
+namespace ug {
+namespace {
+
+constexpr unsigned long long kDefaultTimeoutNs = 2000ull * 1000 * 1000;   // 2 s per wait
+
+template <typename T>
+int upload(T** dst, const std::vector<T>& src) {
+  const size_t bytes = std::max<size_t>(src.size(), 1) * sizeof(T);
+  if (cudaMalloc(reinterpret_cast<void**>(dst), bytes) != cudaSuccess) {
+    cudaGetLastError();
+    *dst = nullptr;
+    return ULTRAGEN_ERR_OOM;
+  }
+  if (!src.empty() && cudaMemcpy(*dst, src.data(), src.size() * sizeof(T), cudaMemcpyHostToDevice) != cudaSuccess)
+    return ULTRAGEN_ERR_CUDA;
+  return ULTRAGEN_OK;
+}
+
+void free_device(ultragen_plan_t* p) {
+  DeviceTables& d = p->dev;
+  void* ptrs[] = {d.items, d.entries, d.mask_off, d.mask_pool, d.perm, d.inv_perm,
+                  d.slot_pos, d.rope, d.combine, d.error, d.ws};
+  for (void* q : ptrs)
+    if (q) cudaFree(q);
+  d = DeviceTables();
+}
+
+int check_device(int* dev_out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return ULTRAGEN_ERR_NO_DEVICE;
+  }
+  int major = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return ULTRAGEN_ERR_NO_DEVICE;
+  }
+  if (major != 10) return ULTRAGEN_ERR_NO_DEVICE;
+  *dev_out = dev;
+  return ULTRAGEN_OK;
+}
+
+// Uploads (or re-uploads after a change) the plan's tables to the current device.
+int ensure_device(ultragen_plan_t* p) {
+  int dev;
+  int st = check_device(&dev);
+  if (st != ULTRAGEN_OK) return st;
+  if (p->dev.valid && p->dev.device == dev && !p->dirty) return ULTRAGEN_OK;
+  free_device(p);
+  DeviceTables& d = p->dev;
+  std::vector<int32_t> items;
+  items.reserve(p->items.size() * kItemInts);
+  for (const Item& it : p->items) items.insert(items.end(), it.v, it.v + kItemInts);
+  std::vector<int32_t> comb;
+  for (const CombineGroup& g : p->combine) {
+    comb.push_back(g.qtile0);
+    comb.push_back(g.qtile1);
+    comb.push_back(g.ws_first);
+    comb.push_back(g.nsplit);
+  }
+  const std::vector<float> rope = rope_table(p);
+  if ((st = upload(&d.items, items)) || (st = upload(&d.entries, p->entries)) ||
+      (st = upload(&d.mask_off, p->mask_off)) || (st = upload(&d.mask_pool, p->mask_pool)) ||
+      (st = upload(&d.perm, p->perm)) || (st = upload(&d.inv_perm, p->inv_perm)) ||
+      (st = upload(&d.slot_pos, p->slot_pos)) || (st = upload(&d.rope, rope)) ||
+      (st = upload(&d.combine, comb)) || (st = upload(&d.error, std::vector<int>(1, 0)))) {
+    free_device(p);
+    return st;
+  }
+  d.device = dev;
+  d.valid = true;
+  p->dirty = false;
+  return ULTRAGEN_OK;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+    cudaGetLastError();
+  });
+  return fn;
+}
+
+// 2D view [rows, D] bf16 with [128 x 64] boxes and the 128-byte swizzle.
+int make_tmap(CUtensorMap* m, const void* base, uint64_t rows, int D) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return ULTRAGEN_ERR_CUDA;
+  const cuuint64_t dims[2] = {(cuuint64_t)D, rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ULTRAGEN_OK : ULTRAGEN_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  cudaGetLastError();
+  return n > 0 ? n : 148;
+}
+
+int grid_for(int64_t rows, int rows_per_block) {
+  const int64_t need = (rows + rows_per_block - 1) / rows_per_block;
+  const int64_t cap = (int64_t)sm_count() * 8;
+  return (int)std::max<int64_t>(1, std::min(need, cap));
+}
+
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return ULTRAGEN_OK;
+  cudaGetLastError();
+  return e == cudaErrorMemoryAllocation ? ULTRAGEN_ERR_OOM : ULTRAGEN_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace ug
+
+using namespace ug;
+
+extern "C" {
+
+int ultragen_plan_destroy(ultragen_plan_t* p) {
+  if (!p) return ULTRAGEN_ERR_INVALID_ARG;
+  if (p->dev.valid) free_device(p);
+  delete p;
+  return ULTRAGEN_OK;
+}
+
+int ultragen_permute_rope(const void* q, const void* k, const void* v, int in_dtype, void* qp,
+                          void* kp, void* vp, int batch, const ultragen_plan_t* cplan,
+                          ultragen_stream_t stream) {
+  ultragen_plan_t* p = const_cast<ultragen_plan_t*>(cplan);
+  if (!p || !q || !k || !v || !qp || !kp || !vp || batch < 1) return ULTRAGEN_ERR_INVALID_ARG;
+  if (in_dtype != ULTRAGEN_BF16 && in_dtype != ULTRAGEN_F32) return ULTRAGEN_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, qp, kp, vp};
+  for (const void* x : ptrs)
+    if (!aligned16(x)) return ULTRAGEN_ERR_INVALID_ARG;
+  if ((int64_t)batch * p->heads * p->N_tot >= ((int64_t)1 << 31) ||
+      (int64_t)batch * p->heads * p->N_raster >= ((int64_t)1 << 31))
+    return ULTRAGEN_ERR_UNSUPPORTED;
+  int st = ensure_device(p);
+  if (st) return st;
+  PermuteArgs a;
+  a.in[0] = q; a.in[1] = k; a.in[2] = v;
+  a.out[0] = static_cast<__nv_bfloat16*>(qp);
+  a.out[1] = static_cast<__nv_bfloat16*>(kp);
+  a.out[2] = static_cast<__nv_bfloat16*>(vp);
+  a.perm = p->dev.perm;
+  a.slot_pos = p->dev.slot_pos;
+  a.rope = p->dev.rope;
+  a.rows_total = (int64_t)batch * p->heads * p->N_tot;
+  a.N_tot = (int)p->N_tot;
+  a.N_raster = (int)p->N_raster;
+  a.heads = p->heads;
+  a.pair_a0 = p->axes[0] / 2;
+  a.pair_a01 = (p->axes[0] + p->axes[1]) / 2;
+  const int rows_per_block = (256 / (p->D / 8)) * 4;
+  p->last_launches = 1;
+  return cuda_status(launch_permute_rope(a, in_dtype, p->D, grid_for(a.rows_total, rows_per_block),
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int ultragen_hla_forward(const void* qp, const void* kp, const void* vp, void* op,
+                         const ultragen_plan_t* cplan, int batch, ultragen_stream_t stream) {
+  ultragen_plan_t* p = const_cast<ultragen_plan_t*>(cplan);
+  if (!p || !qp || !kp || !vp || !op || batch < 1) return ULTRAGEN_ERR_INVALID_ARG;
+  const void* ptrs[] = {qp, kp, vp, op};
+  for (const void* x : ptrs)
+    if (!aligned16(x)) return ULTRAGEN_ERR_INVALID_ARG;
+  const int64_t rows = (int64_t)batch * p->heads * p->N_tot;
+  const int64_t items = (int64_t)batch * p->heads * (int64_t)p->items.size();
+  if (rows >= ((int64_t)1 << 31) || items >= ((int64_t)1 << 31)) return ULTRAGEN_ERR_UNSUPPORTED;
+  int st = ensure_device(p);
+  if (st) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  // split workspace, owned by the plan and grown on demand
+  const size_t ws_need = (size_t)batch * p->heads * p->n_split_items * 2 * kTile * (p->D + 1) * sizeof(float);
+  if (ws_need > p->dev.ws_bytes) {
+    if (p->dev.ws) {
+      cudaStreamSynchronize(s);
+      cudaFree(p->dev.ws);
+      p->dev.ws = nullptr;
+      p->dev.ws_bytes = 0;
+    }
+    if (cudaMalloc(reinterpret_cast<void**>(&p->dev.ws), ws_need) != cudaSuccess) {
+      cudaGetLastError();
+      p->dev.ws = nullptr;
+      return ULTRAGEN_ERR_OOM;
+    }
+    p->dev.ws_bytes = ws_need;
+  }
+
+  alignas(64) CUtensorMap tq, tk, tv;
+  if ((st = make_tmap(&tq, qp, rows, p->D)) || (st = make_tmap(&tk, kp, rows, p->D)) ||
+      (st = make_tmap(&tv, vp, rows, p->D)))
+    return st;
+
+  FwdParams f;
+  f.items = p->dev.items;
+  f.entries = p->dev.entries;
+  f.mask_off = p->dev.mask_off;
+  f.mask_pool = p->dev.mask_pool;
+  f.perm = p->dev.perm;
+  f.out = static_cast<__nv_bfloat16*>(op);
+  f.ws = p->dev.ws;
+  f.err = p->dev.error;
+  f.n_items_head = (int)p->items.size();
+  f.total_items = (int)items;
+  f.N_tot = (int)p->N_tot;
+  f.off_hr = (int)p->off_hr;
+  f.l2 = p->l * p->l;
+  f.n_ws_head = p->n_split_items;
+  f.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)p->D));
+  f.timeout_ns = kDefaultTimeoutNs;
+  const int grid = (int)std::min<int64_t>(items, sm_count());
+  p->last_launches = 0;
+  if (grid > 0) {
+    st = cuda_status(launch_hla_fwd(&tq, &tk, &tv, f, p->D, grid, s));
+    if (st) return st;
+    p->last_launches++;
+  }
+  if (!p->combine.empty()) {
+    CombineArgs c;
+    c.ws = p->dev.ws;
+    c.out = f.out;
+    c.groups = p->dev.combine;
+    c.perm = p->dev.perm;
+    c.n_groups = (int)p->combine.size();
+    c.n_ws_head = p->n_split_items;
+    c.N_tot = (int)p->N_tot;
+    c.BH = batch * p->heads;
+    st = cuda_status(launch_combine(c, p->D, s));
+    if (st) return st;
+    p->last_launches++;
+  }
+  return ULTRAGEN_OK;
+}
+
+int ultragen_unpermute(const void* op, void* o, int out_dtype, int batch,
+                       const ultragen_plan_t* cplan, ultragen_stream_t stream) {
+  ultragen_plan_t* p = const_cast<ultragen_plan_t*>(cplan);
+  if (!p || !op || !o || batch < 1) return ULTRAGEN_ERR_INVALID_ARG;
+  if (out_dtype != ULTRAGEN_BF16 && out_dtype != ULTRAGEN_F32) return ULTRAGEN_ERR_INVALID_ARG;
+  if (!aligned16(op) || !aligned16(o)) return ULTRAGEN_ERR_INVALID_ARG;
+  if ((int64_t)batch * p->heads * p->N_tot >= ((int64_t)1 << 31)) return ULTRAGEN_ERR_UNSUPPORTED;
+  int st = ensure_device(p);
+  if (st) return st;
+  UnpermuteArgs a;
+  a.in = static_cast<const __nv_bfloat16*>(op);
+  a.out = o;
+  a.inv_perm = p->dev.inv_perm;
+  a.rows_total = (int64_t)batch * p->N_raster * p->heads;
+  a.N_tot = (int)p->N_tot;
+  a.N_raster = (int)p->N_raster;
+  a.heads = p->heads;
+  const int rows_per_block = (256 / (p->D / 8)) * 4;
+  p->last_launches = 1;
+  return cuda_status(launch_unpermute(a, out_dtype, p->D, grid_for(a.rows_total, rows_per_block),
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int ultragen_sync_status(const ultragen_plan_t* cplan, ultragen_stream_t stream) {
+  ultragen_plan_t* p = const_cast<ultragen_plan_t*>(cplan);
+  if (!p) return ULTRAGEN_ERR_INVALID_ARG;
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_status(e);
+  if (!p->dev.valid || !p->dev.error) return ULTRAGEN_OK;
+  int h = 0;
+  if (cudaMemcpy(&h, p->dev.error, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return cuda_status(cudaGetLastError());
+  if (h != 0) {
+    cudaMemset(p->dev.error, 0, sizeof(int));
+    return ULTRAGEN_ERR_TIMEOUT;
+  }
+  return ULTRAGEN_OK;
+}
+
+int ultragen_last_launch_count(const ultragen_plan_t* p) { return p ? p->last_launches : -1; }
+
+}  // extern "C"

@@ -1,0 +1,454 @@
+// Block-sparse masked attention forward for sm_100a (tcgen05 + TMEM + TMA).
+//
+// Computes softmax(Q K^T / sqrt(d) + M) V over the window-first layout ("UltraGen ..."
+// papernotes note, 关键设计 3, the MMA equation, with M read as an additive -inf on masked
+// pairs), visiting for each query tile only the key tiles its plan list names; masks are
+// applied per element on partial tiles only.
+//
+// CTA organisation (one persistent CTA per SM, 320 threads):
+//   warps 0-3   softmax group 0: owns query tile slot 0 (thread = row, TMEM lane = row)
+//   warps 4-7   softmax group 1: owns query tile slot 1
+//   warp  8     producer: TMA loads of Q (per item) and of K, V tiles into a ring
+//   warp  9     MMA issuer: tcgen05.mma for S = Q K^T (both operands in shared memory) and
+//               O += P V (P read from TMEM, V from shared memory); owns TMEM allocation
+// A work item is one or two query tiles with the same key list (the two 128-row halves of
+// a 16x16 window, two text tiles, two LR tiles), so each K/V tile is loaded once per two
+// query tiles.  The issue order S0(j) / S1(j) / [P0 V(j)] / S0(j+1) ... lets one softmax
+// group work on its tile while the tensor core runs the other group's products.
+//
+// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D, 256+2D).
+// P (bf16, packed in pairs) overwrites the first 64 columns of its S block.
+// Shared memory: Q0, Q1, and NS K/V slots, each [128 rows x D] bf16 stored as D/64 boxes of
+// [128 x 64] with the 128-byte swizzle (TMA writes it, the MMA descriptors read it).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace ug {
+
+template <int D>
+struct FwdCfg {
+  static constexpr int BOXES = D / 64;
+  static constexpr int BOX_BYTES = 128 * 64 * 2;
+  static constexpr int TILE_BYTES = 128 * D * 2;
+  static constexpr int NS = D == 128 ? 4 : 8;
+  static constexpr int Q_OFF = 0;
+  static constexpr int KV_OFF = 2 * TILE_BYTES;
+  static constexpr int BAR_OFF = KV_OFF + NS * TILE_BYTES;
+  // barrier indices
+  static constexpr int B_QF = 0, B_QE = 1, B_KVF = 2, B_KVE = 2 + NS, B_SF = 2 + 2 * NS,
+                       B_PF = 4 + 2 * NS, B_OF = 6 + 2 * NS, B_DRAIN = 8 + 2 * NS;
+  static constexpr int NBAR = 9 + 2 * NS;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+  static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;   // + slack for 1024-B alignment
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t O_COL = 256;
+};
+
+constexpr int kThreads = 320;
+constexpr int kWarpProducer = 8;
+constexpr int kWarpMma = 9;
+constexpr uint64_t kDrainNs = 50ull * 1000 * 1000;   // bounded drain on the abort path
+
+__device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// ------------------------------------------------------------------------ producer warp
+template <int D>
+__device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
+                              const CUtensorMap* tmV, const FwdParams& p, uint32_t sbase,
+                              volatile int* abort_flag) {
+  using C = FwdCfg<D>;
+  const uint32_t sQ = sbase + C::Q_OFF, sKV = sbase + C::KV_OFF, bar = sbase + C::BAR_OFF;
+  uint32_t ld = 0, qi = 0;
+  bool ok = true;
+  for (int it = blockIdx.x; it < p.total_items && ok; it += gridDim.x) {
+    const int32_t* I = p.items + (it % p.n_items_head) * 8;
+    const int bh = it / p.n_items_head;
+    const int qt0 = I[0], qt1 = I[1], e0 = I[2], e1 = I[3];
+    if (e1 == e0) continue;
+    if (!mbar_wait(bar + 8 * C::B_QE, (qi & 1) ^ 1, abort_flag, p.err, DEV_TIMEOUT_PRODUCER,
+                   p.timeout_ns)) {
+      ok = false;
+      break;
+    }
+    const int ntile = qt1 >= 0 ? 2 : 1;
+    mbar_expect_tx(bar + 8 * C::B_QF, ntile * C::TILE_BYTES);
+    for (int t = 0; t < ntile; ++t) {
+      const int y = bh * p.N_tot + (t ? qt1 : qt0) * 128;
+#pragma unroll
+      for (int bx = 0; bx < C::BOXES; ++bx)
+        tma_load_2d(sQ + t * C::TILE_BYTES + bx * C::BOX_BYTES, tmQ, bx * 64, y,
+                    bar + 8 * C::B_QF);
+    }
+    ++qi;
+    for (int e = e0; e < e1 && ok; ++e) {
+      const int y = bh * p.N_tot + (__ldg(p.entries + e) & 0x7fffffff) * 128;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t s = ld % C::NS, ph = (ld / C::NS) & 1;
+        if (!mbar_wait(bar + 8 * (C::B_KVE + s), ph ^ 1, abort_flag, p.err, DEV_TIMEOUT_PRODUCER,
+                       p.timeout_ns)) {
+          ok = false;
+          break;
+        }
+        mbar_expect_tx(bar + 8 * (C::B_KVF + s), C::TILE_BYTES);
+#pragma unroll
+        for (int bx = 0; bx < C::BOXES; ++bx)
+          tma_load_2d(sKV + s * C::TILE_BYTES + bx * C::BOX_BYTES, which ? tmV : tmK, bx * 64, y,
+                      bar + 8 * (C::B_KVF + s));
+        ++ld;
+      }
+    }
+  }
+  if (!ok) {
+    // Abort: wait (bounded) until the copies this thread issued have landed, so that no TMA
+    // write targets this CTA's shared memory after it exits.
+    for (uint32_t s = 0; s < (uint32_t)C::NS; ++s) {
+      if (ld <= s) break;
+      const uint32_t last = ld - 1 - ((ld - 1 - s) % C::NS);
+      mbar_wait(bar + 8 * (C::B_KVF + s), (last / C::NS) & 1, nullptr, p.err, DEV_TIMEOUT_DRAIN,
+                kDrainNs);
+    }
+    if (qi > 0) mbar_wait(bar + 8 * C::B_QF, (qi - 1) & 1, nullptr, p.err, DEV_TIMEOUT_DRAIN, kDrainNs);
+  }
+}
+
+// ------------------------------------------------------------------------ MMA warp
+template <int D>
+__device__ __forceinline__ void issue_s(uint32_t tmem_d, uint32_t sQt, uint32_t sK) {
+  using C = FwdCfg<D>;
+  constexpr uint32_t idS = idesc_bf16(128, 128, 0);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (kk / 4) * C::BOX_BYTES + (kk % 4) * 32;
+    mma_ss(tmem_d, smem_desc_sw128(sQt + off, 16, 1024), smem_desc_sw128(sK + off, 16, 1024), idS,
+           kk > 0 ? 1u : 0u);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void issue_pv(uint32_t tmem_d, uint32_t tmem_p, uint32_t sV,
+                                         bool accumulate) {
+  using C = FwdCfg<D>;
+  constexpr uint32_t idO = idesc_bf16(128, D, 1);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    mma_ts(tmem_d, tmem_p + kk * 8, smem_desc_sw128(sV + kk * 2048, C::BOX_BYTES, 1024), idO,
+           (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+template <int D>
+__device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t tbase,
+                         volatile int* abort_flag) {
+  using C = FwdCfg<D>;
+  const uint32_t sQ = sbase + C::Q_OFF, sKV = sbase + C::KV_OFF, bar = sbase + C::BAR_OFF;
+  uint32_t ld = 0, qi = 0, pc0 = 0, pc1 = 0;
+  auto wait = [&](int b, uint32_t par) {
+    return mbar_wait(bar + 8 * b, par, abort_flag, p.err, DEV_TIMEOUT_MMA, p.timeout_ns);
+  };
+  bool ok = true;
+  for (int it = blockIdx.x; it < p.total_items && ok; it += gridDim.x) {
+    const int32_t* I = p.items + (it % p.n_items_head) * 8;
+    const int qt1 = I[1], n = I[3] - I[2];
+    if (n == 0) continue;
+    const int ntile = qt1 >= 0 ? 2 : 1;
+    if (!wait(C::B_QF, qi & 1)) { ok = false; break; }
+    ++qi;
+    tc_fence_after();
+    {  // j = 0: S_t = Q_t K_0^T
+      const uint32_t s = ld % C::NS;
+      if (!wait(C::B_KVF + s, (ld / C::NS) & 1)) { ok = false; break; }
+      tc_fence_after();
+      for (int t = 0; t < ntile; ++t) {
+        issue_s<D>(tbase + 128 * t, sQ + t * C::TILE_BYTES, sKV + s * C::TILE_BYTES);
+        mma_commit(bar + 8 * (C::B_SF + t));
+      }
+      mma_commit(bar + 8 * (C::B_KVE + s));
+    }
+    for (int j = 1; j < n && ok; ++j) {
+      const uint32_t nv = ld + 2 * j - 1, nk = ld + 2 * j;
+      const uint32_t sv = nv % C::NS, sk = nk % C::NS;
+      if (!wait(C::B_KVF + sv, (nv / C::NS) & 1) || !wait(C::B_KVF + sk, (nk / C::NS) & 1)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      for (int t = 0; t < ntile; ++t) {
+        uint32_t& pc = t ? pc1 : pc0;
+        if (!wait(C::B_PF + t, pc & 1)) { ok = false; break; }
+        ++pc;
+        tc_fence_after();
+        issue_pv<D>(tbase + C::O_COL + D * t, tbase + 128 * t, sKV + sv * C::TILE_BYTES, j > 1);
+        issue_s<D>(tbase + 128 * t, sQ + t * C::TILE_BYTES, sKV + sk * C::TILE_BYTES);
+        mma_commit(bar + 8 * (C::B_SF + t));
+      }
+      if (!ok) break;
+      mma_commit(bar + 8 * (C::B_KVE + sv));
+      mma_commit(bar + 8 * (C::B_KVE + sk));
+    }
+    if (!ok) break;
+    mma_commit(bar + 8 * C::B_QE);   // all products that read Q of this item are issued
+    {
+      const uint32_t nv = ld + 2 * n - 1, sv = nv % C::NS;
+      if (!wait(C::B_KVF + sv, (nv / C::NS) & 1)) { ok = false; break; }
+      tc_fence_after();
+      for (int t = 0; t < ntile; ++t) {
+        uint32_t& pc = t ? pc1 : pc0;
+        if (!wait(C::B_PF + t, pc & 1)) { ok = false; break; }
+        ++pc;
+        tc_fence_after();
+        issue_pv<D>(tbase + C::O_COL + D * t, tbase + 128 * t, sKV + sv * C::TILE_BYTES, n > 1);
+        mma_commit(bar + 8 * (C::B_OF + t));
+      }
+      if (!ok) break;
+      mma_commit(bar + 8 * (C::B_KVE + sv));
+    }
+    ld += 2 * n;
+  }
+  if (!ok) {
+    // Abort: let the products already issued finish before TMEM is released.
+    mma_commit(bar + 8 * C::B_DRAIN);
+    mbar_wait(bar + 8 * C::B_DRAIN, 0, nullptr, p.err, DEV_TIMEOUT_DRAIN, kDrainNs);
+  }
+}
+
+// ------------------------------------------------------------------------ softmax groups
+template <int D>
+__device__ void softmax_role(const FwdParams& p, uint32_t sbase, uint32_t tbase,
+                             volatile int* abort_flag) {
+  using C = FwdCfg<D>;
+  const uint32_t bar = sbase + C::BAR_OFF;
+  const int t = threadIdx.x >> 7;                 // query tile slot 0 / 1
+  const int r = threadIdx.x & 127;                // row inside the tile = TMEM lane
+  const uint32_t lane_off = (uint32_t)((threadIdx.x >> 5) & 3) * 32u << 16;
+  const uint32_t tS = tbase + lane_off + (uint32_t)(t * 128);
+  const uint32_t tO = tbase + lane_off + C::O_COL + (uint32_t)(t * D);
+  const float scale = p.scale_log2;
+  uint32_t sc = 0, oc = 0;
+
+  for (int it = blockIdx.x; it < p.total_items; it += gridDim.x) {
+    const int32_t* I = p.items + (it % p.n_items_head) * 8;
+    const int bh = it / p.n_items_head;
+    const int qt = t ? I[1] : I[0];
+    if (qt < 0) continue;
+    const int e0 = I[2], n = I[3] - I[2], ws_slot = I[4], ncls = I[5], wfirst = I[6];
+    const int slot = qt * 128 + r;
+    const bool real = __ldg(p.perm + slot) >= 0;
+    int cls = 0;
+    if (ncls > 1 && wfirst >= 0) {
+      cls = (slot - p.off_hr) / p.l2 - wfirst;
+      cls = cls < 0 ? 0 : (cls > ncls - 1 ? ncls - 1 : cls);
+    }
+    __nv_bfloat16* orow = p.out + ((size_t)bh * p.N_tot + slot) * D;
+    if (n == 0) {
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(orow)[c] = make_uint4(0, 0, 0, 0);
+      continue;
+    }
+    float m = neg_inf(), lsum = 0.f;
+    for (int j = 0; j < n; ++j) {
+      const int ent = __ldg(p.entries + e0 + j);
+      uint32_t mw[4] = {~0u, ~0u, ~0u, ~0u};
+      if (ent < 0) {
+        const uint32_t* mp = p.mask_pool + __ldg(p.mask_off + e0 + j) + cls * 4;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) mw[w] = __ldg(mp + w);
+      }
+      bool ok = mbar_wait(bar + 8 * (C::B_SF + t), sc & 1, abort_flag, p.err, DEV_TIMEOUT_SOFTMAX,
+                          p.timeout_ns);
+      if (!__all_sync(0xffffffffu, ok)) return;
+      ++sc;
+      tc_fence_after();
+      uint32_t s[128];
+      tmem_ld128_sync(tS, s);
+      float mx = neg_inf();
+      if (ent < 0) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          const float v = ((mw[c >> 5] >> (c & 31)) & 1u) ? __uint_as_float(s[c]) : neg_inf();
+          s[c] = __float_as_uint(v);
+          mx = fmaxf(mx, v);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
+      }
+      const float mnew = fmaxf(m, mx * scale);
+      if (j == 0) {
+        m = mnew;
+      } else {
+        // Lazy rescale: keep the running max unless it grew by more than 2^8; the final
+        // division by the matching row sum makes the result exact either way.
+        const bool need = mnew > m + 8.0f;
+        if (__any_sync(0xffffffffu, need)) {
+          const float f = need ? ex2(m - mnew) : 1.0f;
+          if (need) {
+            lsum *= f;
+            m = mnew;
+          }
+          __syncwarp();
+#pragma unroll
+          for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t o[32];
+            tmem_ld32_sync(tO + ch * 32, o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+            tmem_st32(tO + ch * 32, o);
+          }
+        }
+      }
+      const float mu = (m == neg_inf()) ? 0.f : m;
+#pragma unroll
+      for (int c2 = 0; c2 < 64; ++c2) {
+        const float p0 = ex2(fmaf(__uint_as_float(s[2 * c2]), scale, -mu));
+        const float p1 = ex2(fmaf(__uint_as_float(s[2 * c2 + 1]), scale, -mu));
+        lsum += p0 + p1;
+        s[c2] = pack_bf16x2(p0, p1);
+      }
+      __syncwarp();
+      tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(&s[0]));
+      tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(&s[32]));
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar + 8 * (C::B_PF + t));
+    }
+    bool ok = mbar_wait(bar + 8 * (C::B_OF + t), oc & 1, abort_flag, p.err, DEV_TIMEOUT_SOFTMAX,
+                        p.timeout_ns);
+    if (!__all_sync(0xffffffffu, ok)) return;
+    ++oc;
+    tc_fence_after();
+    __syncwarp();
+    const float inv = (lsum > 0.f) ? 1.0f / lsum : 0.f;
+    if (ws_slot < 0) {
+      const float f = real ? inv : 0.f;
+#pragma unroll
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t o[32];
+        tmem_ld32_sync(tO + ch * 32, o);
+        uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint4 v;
+          v.x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * f, __uint_as_float(o[8 * q + 1]) * f);
+          v.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * f, __uint_as_float(o[8 * q + 3]) * f);
+          v.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * f, __uint_as_float(o[8 * q + 5]) * f);
+          v.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * f, __uint_as_float(o[8 * q + 7]) * f);
+          dst[q] = v;
+        }
+      }
+    } else {
+      float* wsb = p.ws + ((size_t)bh * p.n_ws_head + ws_slot) * ((size_t)2 * 128 * (D + 1));
+      float* wo = wsb + (size_t)(t * 128 + r) * D;
+#pragma unroll
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t o[32];
+        tmem_ld32_sync(tO + ch * 32, o);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          float4 v = make_float4(__uint_as_float(o[4 * q + 0]) * inv, __uint_as_float(o[4 * q + 1]) * inv,
+                                 __uint_as_float(o[4 * q + 2]) * inv, __uint_as_float(o[4 * q + 3]) * inv);
+          reinterpret_cast<float4*>(wo + ch * 32)[q] = v;
+        }
+      }
+      wsb[2 * 128 * D + t * 128 + r] = (lsum > 0.f) ? m + log2f(lsum) : neg_inf();
+    }
+    tc_fence_before();
+  }
+}
+
+// ------------------------------------------------------------------------ kernel
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    hla_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  using C = FwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar = sbase + C::BAR_OFF;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar + 8 * C::B_QF, 1);
+    mbar_init(bar + 8 * C::B_QE, 1);
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(bar + 8 * (C::B_KVF + s), 1);
+      mbar_init(bar + 8 * (C::B_KVE + s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar + 8 * (C::B_SF + t), 1);
+      mbar_init(bar + 8 * (C::B_PF + t), 128);
+      mbar_init(bar + 8 * (C::B_OF + t), 1);
+    }
+    mbar_init(bar + 8 * C::B_DRAIN, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kWarpProducer && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(smem_u32(misc), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = misc[0];
+
+  if (warp == kWarpProducer) {
+    if (lane == 0) producer_role<D>(&tmQ, &tmK, &tmV, p, sbase, abort_flag);
+  } else if (warp == kWarpMma) {
+    if (lane == 0) mma_role<D>(p, sbase, tbase, abort_flag);
+  } else {
+    softmax_role<D>(p, sbase, tbase, abort_flag);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kWarpMma) {
+    __syncwarp();
+    tmem_dealloc(tbase, C::TMEM_COLS);
+  }
+}
+
+template <int D>
+static cudaError_t launch_d(const void* tmQ, const void* tmK, const void* tmV, const FwdParams& p,
+                            int grid, cudaStream_t st) {
+  static bool attr_set = false;
+  const int smem = FwdCfg<D>::SMEM_BYTES;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(hla_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  hla_fwd_kernel<D><<<grid, kThreads, smem, st>>>(*static_cast<const CUtensorMap*>(tmQ),
+                                                   *static_cast<const CUtensorMap*>(tmK),
+                                                   *static_cast<const CUtensorMap*>(tmV), p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_hla_fwd(const void* tmQ, const void* tmK, const void* tmV, const FwdParams& p,
+                           int D, int grid, cudaStream_t st) {
+  return D == 128 ? launch_d<128>(tmQ, tmK, tmV, p, grid, st)
+                  : launch_d<64>(tmQ, tmK, tmV, p, grid, st);
+}
+
+}  // namespace ug

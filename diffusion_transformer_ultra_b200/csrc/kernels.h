@@ -1,0 +1,66 @@
+// Argument blocks and launchers of the device kernels (host side includes this).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace ug {
+
+struct PermuteArgs {
+  const void* in[3];               // q, k, v raster [B, N_raster, heads, D]
+  __nv_bfloat16* out[3];           // qp, kp, vp window-first [B, heads, N_tot, D]
+  const int32_t* perm;             // slot -> raster, -1 pad
+  const uint32_t* slot_pos;        // (row_pos << 16) | col_pos
+  const float* rope;               // [max(H,W)][D/2][2] (cos, sin)
+  int64_t rows_total;              // B * heads * N_tot
+  int N_tot, N_raster, heads;
+  int pair_a0, pair_a01;           // pairs [0,a0) axis 0, [a0,a01) axis 1, rest axis 2
+};
+
+struct UnpermuteArgs {
+  const __nv_bfloat16* in;         // [B, heads, N_tot, D]
+  void* out;                       // [B, N_raster, heads, D]
+  const int32_t* inv_perm;         // raster -> slot
+  int64_t rows_total;              // B * N_raster * heads
+  int N_tot, N_raster, heads;
+};
+
+struct CombineArgs {
+  const float* ws;                 // split partials
+  __nv_bfloat16* out;              // [B*heads, N_tot, D]
+  const int32_t* groups;           // 4 ints per split group: qt0, qt1, ws_first, nsplit
+  const int32_t* perm;
+  int n_groups, n_ws_head, N_tot, BH;
+};
+
+struct FwdParams {
+  const int32_t* items;            // 8 ints per item (per batch-head)
+  const int32_t* entries;          // key tile | partial << 31
+  const int32_t* mask_off;         // per entry, -1 full
+  const uint32_t* mask_pool;       // per partial entry: classes x 4 words
+  const int32_t* perm;             // slot -> raster, -1 pad
+  __nv_bfloat16* out;              // [B*heads, N_tot, D]
+  float* ws;                       // split partials [B*heads][n_ws_head][2][128][D+1]
+  int* err;                        // device error word
+  int n_items_head;
+  int total_items;
+  int N_tot;
+  int off_hr;
+  int l2;                          // l * l
+  int n_ws_head;
+  float scale_log2;                // log2(e) / sqrt(D)
+  unsigned long long timeout_ns;   // limit of every device-side wait
+};
+
+cudaError_t launch_permute_rope(const PermuteArgs& a, int in_dtype, int D, int grid_x,
+                                cudaStream_t st);
+cudaError_t launch_unpermute(const UnpermuteArgs& a, int out_dtype, int D, int grid_x,
+                             cudaStream_t st);
+cudaError_t launch_combine(const CombineArgs& a, int D, cudaStream_t st);
+// Launches the block-sparse attention kernel; tensor maps are built by the caller.
+cudaError_t launch_hla_fwd(const void* tmQ, const void* tmK, const void* tmV,
+                           const FwdParams& p, int D, int grid, cudaStream_t st);
+
+}  // namespace ug

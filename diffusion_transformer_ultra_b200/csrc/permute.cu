@@ -1,0 +1,238 @@
+// HBM-bound passes around the attention:
+//   permute_rope   raster [B, N_raster, H, D] -> window-first [B, H, N_tot, D] bf16, with axial
+//                  2D RoPE on Q and K ("UltraGen ..." papernotes note, 关键设计 1 window-first
+//                  order; 关键设计 2 LR positions (rho m, rho n)).
+//   unpermute      window-first [B, H, N_tot, D] bf16 -> raster [B, N_raster, H, D].
+//   split combine  log-sum-exp merge of the partial outputs of split query groups.
+// Every thread moves 16-byte chunks (8 bf16) so loads and stores are full-sector.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "kernels.h"
+
+namespace ug {
+
+namespace {
+
+__device__ __forceinline__ void load8(const __nv_bfloat16* src, float (&x)[8]) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4*>(src));
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    x[2 * i] = __uint_as_float(w[i] << 16);
+    x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+__device__ __forceinline__ void load8(const float* src, float (&x)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(src));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(src) + 1);
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+  x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+}  // namespace
+
+// One thread = one 16-byte output chunk of one output row; a block covers ROWS rows per
+// pass and each thread handles U rows per pass so that U loads are in flight together.
+template <typename Tin, int D>
+__global__ void __launch_bounds__(256) permute_rope_kernel(PermuteArgs a) {
+  constexpr int CH = D / 8;
+  constexpr int ROWS = 256 / CH;
+  constexpr int U = 4;
+  constexpr int HALF = D / 2;
+  const int which = blockIdx.y;
+  const bool do_rope = which < 2;
+  const Tin* __restrict__ in = static_cast<const Tin*>(a.in[which]);
+  __nv_bfloat16* __restrict__ out = a.out[which];
+  const int c = threadIdx.x % CH;
+  const int rsub = threadIdx.x / CH;
+  const int64_t step = (int64_t)gridDim.x * ROWS * U;
+
+  for (int64_t row0 = (int64_t)blockIdx.x * ROWS * U; row0 < a.rows_total; row0 += step) {
+    float x[U][8];
+    int pos_r[U], pos_c[U];
+    bool live[U], real[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t row = row0 + u * ROWS + rsub;
+      live[u] = row < a.rows_total;
+      real[u] = false;
+      if (!live[u]) continue;
+      const int slot = (int)(row % a.N_tot);
+      const int64_t bh = row / a.N_tot;
+      const int h = (int)(bh % a.heads);
+      const int b = (int)(bh / a.heads);
+      const int r = __ldg(a.perm + slot);
+      if (r < 0) continue;
+      real[u] = true;
+      const uint32_t sp = __ldg(a.slot_pos + slot);
+      pos_r[u] = (int)(sp >> 16);
+      pos_c[u] = (int)(sp & 0xffffu);
+      load8(in + (((int64_t)b * a.N_raster + r) * a.heads + h) * D + c * 8, x[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (!live[u]) continue;
+      const int64_t row = row0 + u * ROWS + rsub;
+      uint4 o = make_uint4(0u, 0u, 0u, 0u);
+      if (real[u]) {
+        if (do_rope) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int q = c * 4 + k;                       // rotation pair index
+            const int pos = q < a.pair_a0 ? 0 : (q < a.pair_a01 ? pos_r[u] : pos_c[u]);
+            if (pos != 0) {
+              const float2 cs = __ldg(reinterpret_cast<const float2*>(a.rope) + (int64_t)pos * HALF + q);
+              const float x0 = x[u][2 * k], x1 = x[u][2 * k + 1];
+              x[u][2 * k] = x0 * cs.x - x1 * cs.y;
+              x[u][2 * k + 1] = x0 * cs.y + x1 * cs.x;
+            }
+          }
+        }
+        o.x = pack_bf16(x[u][0], x[u][1]);
+        o.y = pack_bf16(x[u][2], x[u][3]);
+        o.z = pack_bf16(x[u][4], x[u][5]);
+        o.w = pack_bf16(x[u][6], x[u][7]);
+      }
+      *reinterpret_cast<uint4*>(out + row * D + c * 8) = o;
+    }
+  }
+}
+
+template <typename Tout, int D>
+__global__ void __launch_bounds__(256) unpermute_kernel(UnpermuteArgs a) {
+  constexpr int CH = D / 8;
+  constexpr int ROWS = 256 / CH;
+  constexpr int U = 4;
+  const int c = threadIdx.x % CH;
+  const int rsub = threadIdx.x / CH;
+  const int64_t step = (int64_t)gridDim.x * ROWS * U;
+  Tout* __restrict__ out = static_cast<Tout*>(a.out);
+  for (int64_t row0 = (int64_t)blockIdx.x * ROWS * U; row0 < a.rows_total; row0 += step) {
+    uint4 v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t row = row0 + u * ROWS + rsub;      // (b, t, h) raster row
+      if (row >= a.rows_total) continue;
+      const int h = (int)(row % a.heads);
+      const int64_t bt = row / a.heads;
+      const int t = (int)(bt % a.N_raster);
+      const int b = (int)(bt / a.N_raster);
+      const int slot = __ldg(a.inv_perm + t);
+      v[u] = __ldg(reinterpret_cast<const uint4*>(a.in + (((int64_t)b * a.heads + h) * a.N_tot + slot) * D + c * 8));
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t row = row0 + u * ROWS + rsub;
+      if (row >= a.rows_total) continue;
+      if constexpr (sizeof(Tout) == 2) {
+        *reinterpret_cast<uint4*>(out + row * D + c * 8) = v[u];
+      } else {
+        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+        float4 f0, f1;
+        f0.x = __uint_as_float(w[0] << 16); f0.y = __uint_as_float(w[0] & 0xffff0000u);
+        f0.z = __uint_as_float(w[1] << 16); f0.w = __uint_as_float(w[1] & 0xffff0000u);
+        f1.x = __uint_as_float(w[2] << 16); f1.y = __uint_as_float(w[2] & 0xffff0000u);
+        f1.z = __uint_as_float(w[3] << 16); f1.w = __uint_as_float(w[3] & 0xffff0000u);
+        reinterpret_cast<float4*>(out + row * D + c * 8)[0] = f0;
+        reinterpret_cast<float4*>(out + row * D + c * 8)[1] = f1;
+      }
+    }
+  }
+}
+
+// One warp per output row of a split group: merges nsplit partial rows (O_s normalised,
+// lse_s in log2 units) as O = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M), M = max_s lse_s.
+template <int D>
+__global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
+  constexpr int PER = D / 32;
+  const int64_t warp_id = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t total = (int64_t)a.BH * a.n_groups * 2 * 128;
+  if (warp_id >= total) return;
+  const int row = (int)(warp_id % 128);
+  const int t = (int)((warp_id / 128) % 2);
+  const int g = (int)((warp_id / 256) % a.n_groups);
+  const int64_t bh = warp_id / (256 * (int64_t)a.n_groups);
+  const int32_t* G = a.groups + 4 * g;
+  const int qt = t ? G[1] : G[0];
+  if (qt < 0) return;
+  const int slot = qt * 128 + row;
+  __nv_bfloat16* dst = a.out + (bh * a.N_tot + slot) * D + lane * PER;
+  const size_t item_floats = (size_t)2 * 128 * (D + 1);
+  const float* base = a.ws + (size_t)(bh * a.n_ws_head) * item_floats;
+  float acc[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) acc[i] = 0.f;
+  float M = -INFINITY;
+  if (__ldg(a.perm + slot) >= 0) {
+    for (int s = 0; s < G[3]; ++s) {
+      const float* it = base + (size_t)(G[2] + s) * item_floats;
+      M = fmaxf(M, __ldg(it + 2 * 128 * D + t * 128 + row));
+    }
+  }
+  float den = 0.f;
+  if (M != -INFINITY) {
+    for (int s = 0; s < G[3]; ++s) {
+      const float* it = base + (size_t)(G[2] + s) * item_floats;
+      const float wgt = exp2f(__ldg(it + 2 * 128 * D + t * 128 + row) - M);
+      den += wgt;
+      const float* o = it + (size_t)(t * 128 + row) * D + lane * PER;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) acc[i] += wgt * __ldg(o + i);
+    }
+  }
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  uint32_t pk[PER / 2];
+#pragma unroll
+  for (int i = 0; i < PER / 2; ++i) pk[i] = pack_bf16(acc[2 * i] * inv, acc[2 * i + 1] * inv);
+  if constexpr (PER == 4) {
+    *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[1]);
+  } else {
+    *reinterpret_cast<uint32_t*>(dst) = pk[0];
+  }
+}
+
+// ------------------------------------------------------------------------------ launchers
+cudaError_t launch_permute_rope(const PermuteArgs& a, int in_dtype, int D, int grid_x,
+                                cudaStream_t st) {
+  dim3 grid(grid_x, 3);
+  if (D == 128) {
+    if (in_dtype == 0) permute_rope_kernel<__nv_bfloat16, 128><<<grid, 256, 0, st>>>(a);
+    else permute_rope_kernel<float, 128><<<grid, 256, 0, st>>>(a);
+  } else {
+    if (in_dtype == 0) permute_rope_kernel<__nv_bfloat16, 64><<<grid, 256, 0, st>>>(a);
+    else permute_rope_kernel<float, 64><<<grid, 256, 0, st>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unpermute(const UnpermuteArgs& a, int out_dtype, int D, int grid_x,
+                             cudaStream_t st) {
+  if (D == 128) {
+    if (out_dtype == 0) unpermute_kernel<__nv_bfloat16, 128><<<grid_x, 256, 0, st>>>(a);
+    else unpermute_kernel<float, 128><<<grid_x, 256, 0, st>>>(a);
+  } else {
+    if (out_dtype == 0) unpermute_kernel<__nv_bfloat16, 64><<<grid_x, 256, 0, st>>>(a);
+    else unpermute_kernel<float, 64><<<grid_x, 256, 0, st>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const CombineArgs& a, int D, cudaStream_t st) {
+  const int64_t warps = (int64_t)a.BH * a.n_groups * 2 * 128;
+  const int64_t blocks = (warps * 32 + 255) / 256;
+  if (D == 128) combine_kernel<128><<<(unsigned)blocks, 256, 0, st>>>(a);
+  else combine_kernel<64><<<(unsigned)blocks, 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace ug

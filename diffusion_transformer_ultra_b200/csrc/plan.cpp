@@ -1,0 +1,470 @@
+// Host plan builder: window geometry, window-first permutation, block-sparse tile lists with
+// per-class column masks, RoPE tables and the kernel schedule.
+//
+// Method (page title, section):
+//   "UltraGen: Efficient Ultra-High-Resolution Image Generation with Hierarchical Local
+//   Attention" -- papernotes.org note, 关键设计 1 (l x l windows, window-first token order,
+//   dense local blocks), 关键设计 2 (LR positions (m,n) -> (rho m, rho n); the mask M:
+//   text <-> text + HR, HR -> own window + neighbouring boundary tokens + text + LR,
+//   LR -> LR), 关键设计 3 (sequence [C_T; X; X_lr]); gist.science summary, 2.B.
+//
+// Visibility classes.  Every query row of a query tile belongs to one class: "text", "LR",
+// or "HR window w" (all rows of a window share the window's halo box).  A key column is
+// visible to a class by the rules above; pad slots are never visible.  For a (query tile,
+// key tile) pair the plan stores, per class of the tile, a 128-bit column mask; the kernel
+// only applies masks on partial entries.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <new>
+
+#include "plan_internal.h"
+
+namespace ug {
+namespace {
+
+int64_t pad128(int64_t n) { return (n + kTile - 1) / kTile * kTile; }
+int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+struct ClassDesc {
+  int kind;              // SEG_TEXT, SEG_HR, SEG_LR
+  int r0, r1, c0, c1;    // HR halo box [r0, r1) x [c0, c1)
+};
+
+inline bool visible(const ultragen_plan_t* p, const ClassDesc& c, int64_t s) {
+  const int sg = p->seg[s];
+  switch (c.kind) {
+    case SEG_TEXT:
+      return sg == SEG_TEXT || sg == SEG_HR;
+    case SEG_LR:
+      return sg == SEG_LR || sg == SEG_TEXT;
+    default:
+      if (sg == SEG_TEXT || sg == SEG_LR) return true;
+      if (sg != SEG_HR) return false;
+      return p->ci[s] >= c.r0 && p->ci[s] < c.r1 && p->cj[s] >= c.c0 && p->cj[s] < c.c1;
+  }
+}
+
+ClassDesc window_class(const ultragen_plan_t* p, int wid) {
+  const int wr = wid / p->nWw, wc = wid % p->nWw;
+  ClassDesc c;
+  c.kind = SEG_HR;
+  c.r0 = std::max(0, wr * p->l - p->b);
+  c.r1 = std::min(p->H, (wr + 1) * p->l + p->b);
+  c.c0 = std::max(0, wc * p->l - p->b);
+  c.c1 = std::min(p->W, (wc + 1) * p->l + p->b);
+  return c;
+}
+
+void add_range(std::vector<int>& v, int64_t s_begin, int64_t s_end) {
+  if (s_end <= s_begin) return;
+  for (int64_t t = s_begin / kTile; t <= (s_end - 1) / kTile; ++t) v.push_back((int)t);
+}
+
+}  // namespace
+
+int build_tables(ultragen_plan_t* p) {
+  p->nWh = cdiv(p->H, p->l);
+  p->nWw = cdiv(p->W, p->l);
+  p->h = p->rho > 0 ? cdiv(p->H, p->rho) : 0;
+  p->w = p->rho > 0 ? cdiv(p->W, p->rho) : 0;
+  p->N_hr = (int64_t)p->H * p->W;
+  p->N_lr = (int64_t)p->h * p->w;
+  p->N_hrp = (int64_t)p->nWh * p->nWw * p->l * p->l;
+  p->off_hr = pad128(p->T);
+  p->off_lr = p->off_hr + pad128(p->N_hrp);
+  p->N_tot = p->off_lr + pad128(p->N_lr);
+  p->N_raster = p->T + p->N_hr + p->N_lr;
+  if (p->N_tot > (int64_t)1 << 30) return ULTRAGEN_ERR_UNSUPPORTED;
+  p->n_qtiles = (int)(p->N_tot / kTile);
+
+  const int64_t N = p->N_tot;
+  p->perm.assign(N, -1);
+  p->inv_perm.assign(p->N_raster, -1);
+  p->seg.assign(N, SEG_PAD);
+  p->ci.assign(N, 0);
+  p->cj.assign(N, 0);
+  p->slot_pos.assign(N, 0u);
+
+  // window-first permutation ([UG-note] 关键设计 1)
+  for (int t = 0; t < p->T; ++t) {
+    p->perm[t] = t;
+    p->inv_perm[t] = t;
+    p->seg[t] = SEG_TEXT;
+    p->ci[t] = t;
+  }
+  const int64_t l2 = (int64_t)p->l * p->l;
+  for (int i = 0; i < p->H; ++i) {
+    for (int j = 0; j < p->W; ++j) {
+      const int64_t win = (int64_t)(i / p->l) * p->nWw + (j / p->l);
+      const int64_t s = p->off_hr + win * l2 + (int64_t)(i % p->l) * p->l + (j % p->l);
+      const int64_t r = p->T + (int64_t)i * p->W + j;
+      p->perm[s] = (int32_t)r;
+      p->inv_perm[r] = (int32_t)s;
+      p->seg[s] = SEG_HR;
+      p->ci[s] = i;
+      p->cj[s] = j;
+      p->slot_pos[s] = ((uint32_t)i << 16) | (uint32_t)j;
+    }
+  }
+  // LR tokens at positions (rho m, rho n) ([UG-note] 关键设计 2)
+  for (int m = 0; m < p->h; ++m) {
+    for (int n = 0; n < p->w; ++n) {
+      const int64_t s = p->off_lr + (int64_t)m * p->w + n;
+      const int64_t r = p->T + p->N_hr + (int64_t)m * p->w + n;
+      p->perm[s] = (int32_t)r;
+      p->inv_perm[r] = (int32_t)s;
+      p->seg[s] = SEG_LR;
+      p->ci[s] = m;
+      p->cj[s] = n;
+      p->slot_pos[s] = ((uint32_t)(p->rho * m) << 16) | (uint32_t)(p->rho * n);
+    }
+  }
+
+  // tile lists
+  const int nq = p->n_qtiles;
+  p->row_ptr.assign(nq + 1, 0);
+  p->entries.clear();
+  p->mask_off.clear();
+  p->mask_pool.clear();
+  p->qt_classes.assign(nq, 1);
+  p->qt_wfirst.assign(nq, -1);
+  p->qt_real.assign(nq, 0);
+  p->useful_pairs = 0;
+  p->n_partial = 0;
+
+  const int64_t hr_end = p->off_hr + p->N_hrp;
+  std::vector<ClassDesc> classes;
+  std::vector<int> class_real;
+  std::vector<int> cand;
+  std::vector<uint32_t> masks;
+
+  for (int t = 0; t < nq; ++t) {
+    const int64_t s0 = (int64_t)t * kTile;
+    int kind = s0 < p->off_hr ? SEG_TEXT : (s0 < p->off_lr ? SEG_HR : SEG_LR);
+    classes.clear();
+    int wfirst = -1;
+    if (kind == SEG_HR && s0 < hr_end) {
+      wfirst = (int)((s0 - p->off_hr) / l2);
+      const int wlast = (int)((std::min<int64_t>(s0 + kTile, hr_end) - 1 - p->off_hr) / l2);
+      for (int wid = wfirst; wid <= wlast; ++wid) classes.push_back(window_class(p, wid));
+    } else {
+      ClassDesc c{kind, 0, 0, 0, 0};
+      classes.push_back(c);
+      if (kind == SEG_HR) wfirst = -1;   // pad-only tile between HR and LR segments
+    }
+    const int C = (int)classes.size();
+    p->qt_classes[t] = C;
+    p->qt_wfirst[t] = wfirst;
+
+    class_real.assign(C, 0);
+    int real = 0;
+    for (int r = 0; r < kTile; ++r) {
+      const int64_t s = s0 + r;
+      if (p->perm[s] < 0) continue;
+      int c = 0;
+      if (wfirst >= 0) c = std::min(C - 1, (int)((s - p->off_hr) / l2) - wfirst);
+      class_real[c]++;
+      real++;
+    }
+    p->qt_real[t] = real;
+    p->row_ptr[t + 1] = p->row_ptr[t];
+    if (real == 0) continue;
+
+    // candidate key tiles
+    cand.clear();
+    add_range(cand, 0, p->T);
+    if (kind == SEG_TEXT) add_range(cand, p->off_hr, hr_end);
+    if (kind == SEG_HR || kind == SEG_LR) add_range(cand, p->off_lr, p->off_lr + p->N_lr);
+    if (kind == SEG_HR) {
+      for (int c = 0; c < C; ++c) {
+        if (class_real[c] == 0) continue;
+        const ClassDesc& cd = classes[c];
+        if (cd.r1 <= cd.r0 || cd.c1 <= cd.c0) continue;
+        for (int wr = cd.r0 / p->l; wr <= (cd.r1 - 1) / p->l; ++wr)
+          for (int wc = cd.c0 / p->l; wc <= (cd.c1 - 1) / p->l; ++wc) {
+            const int64_t ws = p->off_hr + ((int64_t)wr * p->nWw + wc) * l2;
+            add_range(cand, ws, ws + l2);
+          }
+      }
+    }
+    std::sort(cand.begin(), cand.end());
+    cand.erase(std::unique(cand.begin(), cand.end()), cand.end());
+
+    masks.assign((size_t)C * 4, 0u);
+    for (int kt : cand) {
+      std::fill(masks.begin(), masks.end(), 0u);
+      const int64_t k0 = (int64_t)kt * kTile;
+      for (int c = 0; c < C; ++c)
+        for (int col = 0; col < kTile; ++col)
+          if (visible(p, classes[c], k0 + col)) masks[c * 4 + col / 32] |= 1u << (col % 32);
+      bool any = false, all = true;
+      int64_t pairs = 0;
+      for (int c = 0; c < C; ++c) {
+        if (class_real[c] == 0) continue;
+        int pc = 0;
+        for (int wd = 0; wd < 4; ++wd) {
+          pc += __builtin_popcount(masks[c * 4 + wd]);
+          if (masks[c * 4 + wd] != 0xffffffffu) all = false;
+        }
+        if (pc) any = true;
+        pairs += (int64_t)pc * class_real[c];
+      }
+      if (!any) continue;
+      p->useful_pairs += pairs;
+      if (all) {
+        p->entries.push_back(kt);
+        p->mask_off.push_back(-1);
+      } else {
+        p->entries.push_back((int32_t)((uint32_t)kt | 0x80000000u));
+        p->mask_off.push_back((int32_t)p->mask_pool.size());
+        p->mask_pool.insert(p->mask_pool.end(), masks.begin(), masks.end());
+        p->n_partial++;
+      }
+      p->row_ptr[t + 1]++;
+    }
+  }
+  build_schedule(p);
+  return ULTRAGEN_OK;
+}
+
+static bool same_list(const ultragen_plan_t* p, int a, int b) {
+  const int na = p->row_ptr[a + 1] - p->row_ptr[a];
+  const int nb = p->row_ptr[b + 1] - p->row_ptr[b];
+  if (na != nb || p->qt_classes[a] != 1 || p->qt_classes[b] != 1) return false;
+  if (p->qt_real[a] == 0 || p->qt_real[b] == 0) return false;
+  for (int e = 0; e < na; ++e) {
+    const int ea = p->row_ptr[a] + e, eb = p->row_ptr[b] + e;
+    if (p->entries[ea] != p->entries[eb]) return false;
+    if (p->mask_off[ea] >= 0) {
+      for (int wd = 0; wd < 4; ++wd)
+        if (p->mask_pool[p->mask_off[ea] + wd] != p->mask_pool[p->mask_off[eb] + wd]) return false;
+    }
+  }
+  return true;
+}
+
+void build_schedule(ultragen_plan_t* p) {
+  struct Group { int qt0, qt1, e0, n; };
+  std::vector<Group> groups;
+  for (int t = 0; t < p->n_qtiles;) {
+    if (t + 1 < p->n_qtiles && same_list(p, t, t + 1)) {
+      groups.push_back({t, t + 1, p->row_ptr[t], p->row_ptr[t + 1] - p->row_ptr[t]});
+      t += 2;
+    } else {
+      groups.push_back({t, -1, p->row_ptr[t], p->row_ptr[t + 1] - p->row_ptr[t]});
+      t += 1;
+    }
+  }
+
+  // split policy
+  int chunk = 0;
+  double threshold = 0;
+  if (p->split_req > 0) {
+    chunk = p->split_req;
+    threshold = chunk;
+  } else if (p->split_req < 0) {
+    int longest = 0;
+    for (const Group& g : groups) {
+      const int64_t s0 = (int64_t)g.qt0 * kTile;
+      if (s0 >= p->off_hr && g.n > longest) longest = g.n;   // HR and LR groups
+    }
+    if (longest > 0) {
+      chunk = std::max(longest, 8);
+      threshold = 1.5 * chunk;
+    }
+  }
+  p->split_chunk = chunk;
+
+  p->items.clear();
+  p->combine.clear();
+  p->n_split_items = 0;
+  std::vector<ug::Item> rest;
+  auto make = [&](const Group& g, int e0, int e1, int ws) {
+    ug::Item it;
+    it.v[0] = g.qt0;
+    it.v[1] = g.qt1;
+    it.v[2] = e0;
+    it.v[3] = e1;
+    it.v[4] = ws;
+    it.v[5] = p->qt_classes[g.qt0];
+    it.v[6] = p->qt_wfirst[g.qt0];
+    it.v[7] = 0;
+    return it;
+  };
+  for (const Group& g : groups) {
+    if (chunk > 0 && g.n > threshold && g.n > chunk) {
+      const int nsplit = cdiv(g.n, chunk);
+      const int cs = cdiv(g.n, nsplit);
+      ug::CombineGroup cg{g.qt0, g.qt1, p->n_split_items, nsplit};
+      p->combine.push_back(cg);
+      for (int s = 0; s < nsplit; ++s) {
+        const int e0 = g.e0 + s * cs;
+        const int e1 = g.e0 + std::min(g.n, (s + 1) * cs);
+        p->items.push_back(make(g, e0, e1, p->n_split_items++));
+      }
+    } else {
+      rest.push_back(make(g, g.e0, g.e0 + g.n, -1));
+    }
+  }
+  p->items.insert(p->items.end(), rest.begin(), rest.end());
+  p->dirty = true;
+}
+
+std::vector<float> rope_table(const ultragen_plan_t* p) {
+  const int P = std::max(p->H, p->W);
+  const int half = p->D / 2;
+  std::vector<float> tab((size_t)P * half * 2);
+  for (int q = 0; q < half; ++q) {
+    int axis, k, d;
+    if (q < p->axes[0] / 2) {
+      axis = 0; k = q; d = p->axes[0];
+    } else if (q < (p->axes[0] + p->axes[1]) / 2) {
+      axis = 1; k = q - p->axes[0] / 2; d = p->axes[1];
+    } else {
+      axis = 2; k = q - (p->axes[0] + p->axes[1]) / 2; d = p->axes[2];
+    }
+    (void)axis;
+    const double omega = std::pow(p->theta, -2.0 * k / d);
+    for (int pos = 0; pos < P; ++pos) {
+      const double phi = pos * omega;
+      tab[((size_t)pos * half + q) * 2 + 0] = (float)std::cos(phi);
+      tab[((size_t)pos * half + q) * 2 + 1] = (float)std::sin(phi);
+    }
+  }
+  return tab;
+}
+
+}  // namespace ug
+
+// ------------------------------------------------------------------------------------
+// host-only C entry points
+// ------------------------------------------------------------------------------------
+extern "C" {
+
+const char* ultragen_status_string(int s) {
+  switch (s) {
+    case ULTRAGEN_OK: return "ok";
+    case ULTRAGEN_ERR_INVALID_ARG: return "invalid argument";
+    case ULTRAGEN_ERR_UNSUPPORTED: return "unsupported configuration";
+    case ULTRAGEN_ERR_CUDA: return "CUDA error";
+    case ULTRAGEN_ERR_OOM: return "out of memory";
+    case ULTRAGEN_ERR_TIMEOUT: return "device wait timed out";
+    case ULTRAGEN_ERR_PLAN_MISMATCH: return "plan does not match the call";
+    case ULTRAGEN_ERR_NO_DEVICE: return "no sm_100 device";
+    default: return "unknown status";
+  }
+}
+
+int ultragen_plan(int H, int W, int l, int b, int rho, int text_len, int heads, int head_dim,
+                  ultragen_plan_t** out) {
+  if (!out) return ULTRAGEN_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (H < 1 || W < 1 || l < 1 || b < 0 || rho < 0 || text_len < 0 || heads < 1)
+    return ULTRAGEN_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return ULTRAGEN_ERR_UNSUPPORTED;
+  if (b > l || H > 32767 || W > 32767 || l > 4096 || text_len > (1 << 24) || heads > 4096)
+    return ULTRAGEN_ERR_UNSUPPORTED;
+  ultragen_plan_t* p = new (std::nothrow) ultragen_plan_t();
+  if (!p) return ULTRAGEN_ERR_OOM;
+  p->H = H; p->W = W; p->l = l; p->b = b; p->rho = rho; p->T = text_len;
+  p->heads = heads; p->D = head_dim;
+  if (head_dim == 64) { p->axes[0] = 16; p->axes[1] = 24; p->axes[2] = 24; }
+  else { p->axes[0] = 16; p->axes[1] = 56; p->axes[2] = 56; }
+  p->theta = 1.0e4;
+  int st;
+  try {
+    st = ug::build_tables(p);
+  } catch (const std::bad_alloc&) {
+    st = ULTRAGEN_ERR_OOM;
+  } catch (...) {
+    st = ULTRAGEN_ERR_INVALID_ARG;
+  }
+  if (st != ULTRAGEN_OK) {
+    delete p;
+    return st;
+  }
+  *out = p;
+  return ULTRAGEN_OK;
+}
+
+int ultragen_plan_set_rope(ultragen_plan_t* p, int a0, int a1, int a2, double theta) {
+  if (!p) return ULTRAGEN_ERR_INVALID_ARG;
+  if (a0 < 0 || a1 < 0 || a2 < 0 || (a0 | a1 | a2) & 1 || a0 + a1 + a2 != p->D ||
+      !(theta > 0.0) || !std::isfinite(theta))
+    return ULTRAGEN_ERR_INVALID_ARG;
+  p->axes[0] = a0; p->axes[1] = a1; p->axes[2] = a2;
+  p->theta = theta;
+  p->dirty = true;
+  return ULTRAGEN_OK;
+}
+
+int ultragen_plan_set_split(ultragen_plan_t* p, int chunk) {
+  if (!p || chunk < -1) return ULTRAGEN_ERR_INVALID_ARG;
+  p->split_req = chunk;
+  try {
+    ug::build_schedule(p);
+  } catch (...) {
+    return ULTRAGEN_ERR_OOM;
+  }
+  return ULTRAGEN_OK;
+}
+
+int ultragen_plan_info(const ultragen_plan_t* p, ultragen_plan_info_t* o) {
+  if (!p || !o) return ULTRAGEN_ERR_INVALID_ARG;
+  std::memset(o, 0, sizeof(*o));
+  o->H = p->H; o->W = p->W; o->l = p->l; o->b = p->b; o->rho = p->rho;
+  o->text_len = p->T; o->heads = p->heads; o->head_dim = p->D;
+  o->nWh = p->nWh; o->nWw = p->nWw; o->h = p->h; o->w = p->w;
+  o->N_raster = p->N_raster; o->N_tot = p->N_tot;
+  o->off_hr = p->off_hr; o->off_lr = p->off_lr;
+  o->n_qtiles = p->n_qtiles;
+  o->n_items = (int32_t)p->items.size();
+  o->n_entries = (int64_t)p->entries.size();
+  o->n_partial = p->n_partial;
+  o->useful_pairs = p->useful_pairs;
+  for (int i = 0; i < 3; ++i) o->rope_axes[i] = p->axes[i];
+  o->rope_theta = p->theta;
+  o->split_chunk = p->split_chunk;
+  o->n_split_groups = (int32_t)p->combine.size();
+  o->n_split_items = p->n_split_items;
+  o->workspace_bytes_per_head = (int64_t)p->n_split_items * 2 * ug::kTile * (p->D + 1) * 4;
+  return ULTRAGEN_OK;
+}
+
+int ultragen_plan_export(const ultragen_plan_t* p, int32_t* perm, int32_t* row_ptr,
+                         int32_t* entries) {
+  if (!p) return ULTRAGEN_ERR_INVALID_ARG;
+  if (perm) std::memcpy(perm, p->perm.data(), p->perm.size() * sizeof(int32_t));
+  if (row_ptr) std::memcpy(row_ptr, p->row_ptr.data(), p->row_ptr.size() * sizeof(int32_t));
+  if (entries) std::memcpy(entries, p->entries.data(), p->entries.size() * sizeof(int32_t));
+  return ULTRAGEN_OK;
+}
+
+int ultragen_plan_export_rowmasks(const ultragen_plan_t* p, int qtile, uint32_t* out) {
+  if (!p || !out || qtile < 0 || qtile >= p->n_qtiles) return ULTRAGEN_ERR_INVALID_ARG;
+  const int e0 = p->row_ptr[qtile], e1 = p->row_ptr[qtile + 1];
+  const int64_t s0 = (int64_t)qtile * ug::kTile;
+  const int64_t l2 = (int64_t)p->l * p->l;
+  const int C = p->qt_classes[qtile], wfirst = p->qt_wfirst[qtile];
+  for (int e = e0; e < e1; ++e) {
+    for (int r = 0; r < ug::kTile; ++r) {
+      uint32_t* dst = out + ((size_t)(e - e0) * ug::kTile + r) * 4;
+      const int64_t s = s0 + r;
+      if (p->perm[s] < 0) {
+        dst[0] = dst[1] = dst[2] = dst[3] = 0u;
+        continue;
+      }
+      if (p->mask_off[e] < 0) {
+        dst[0] = dst[1] = dst[2] = dst[3] = 0xffffffffu;
+        continue;
+      }
+      int c = 0;
+      if (wfirst >= 0) c = std::min(C - 1, (int)((s - p->off_hr) / l2) - wfirst);
+      for (int wd = 0; wd < 4; ++wd) dst[wd] = p->mask_pool[p->mask_off[e] + c * 4 + wd];
+    }
+  }
+  return ULTRAGEN_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,97 @@
+// Internal plan representation shared by the host plan builder and the device entry points.
+#pragma once
+
+#include <cstdint>
+#include <vector>
+
+#include "ultragen.h"
+
+namespace ug {
+
+constexpr int kTile = 128;          // query and key tile edge (rows / columns)
+constexpr int kItemInts = 8;        // int32 fields per work item
+
+enum Seg : int8_t { SEG_PAD = -1, SEG_TEXT = 0, SEG_HR = 1, SEG_LR = 2 };
+
+// One unit of kernel work for one (batch, head): one or two query tiles that share the same
+// key-tile list and masks, over a contiguous range of that list.
+//   [0] qtile0   [1] qtile1 (-1: single tile)   [2] entry begin   [3] entry end
+//   [4] workspace slot (-1: write the output directly)   [5] row classes C of qtile0
+//   [6] first window of qtile0 (HR tiles) or -1   [7] unused
+struct Item {
+  int32_t v[kItemInts];
+};
+
+// A query group whose key list is split: partials of its nsplit items are merged.
+struct CombineGroup {
+  int32_t qtile0, qtile1, ws_first, nsplit;
+};
+
+struct DeviceTables {
+  int device = -1;
+  bool valid = false;
+  int32_t* items = nullptr;
+  int32_t* entries = nullptr;
+  int32_t* mask_off = nullptr;
+  uint32_t* mask_pool = nullptr;
+  int32_t* perm = nullptr;
+  int32_t* inv_perm = nullptr;
+  uint32_t* slot_pos = nullptr;    // (pos_row << 16) | pos_col per slot; 0 for text/pad
+  float* rope = nullptr;           // [max(H,W)][head_dim/2][2] (cos, sin)
+  int32_t* combine = nullptr;      // CombineGroup[]
+  int* error = nullptr;            // device error word
+  float* ws = nullptr;             // split partials
+  size_t ws_bytes = 0;
+};
+
+}  // namespace ug
+
+struct ultragen_plan {
+  // arguments
+  int H, W, l, b, rho, T, heads, D;
+  // geometry
+  int nWh, nWw, h, w;
+  int64_t N_hr, N_lr, N_hrp, off_hr, off_lr, N_tot, N_raster;
+  int n_qtiles;
+  // rope
+  int axes[3];
+  double theta;
+  // split policy (-1 auto, 0 off, >0 chunk) and the chunk in effect
+  int split_req = -1;
+  int split_chunk = 0;
+
+  // host tables
+  std::vector<int32_t> perm;       // slot -> raster (-1 pad)
+  std::vector<int32_t> inv_perm;   // raster -> slot
+  std::vector<int8_t> seg;         // per slot
+  std::vector<int32_t> ci, cj;     // per slot coordinates (HR: i,j; LR: m,n; text: t,0)
+  std::vector<uint32_t> slot_pos;  // per slot packed RoPE positions
+  std::vector<int32_t> row_ptr;    // CSR over query tiles
+  std::vector<int32_t> entries;    // key tile | partial << 31
+  std::vector<int32_t> mask_off;   // per entry: offset into mask_pool, -1 when full
+  std::vector<uint32_t> mask_pool; // per partial entry: C classes x 4 words
+  std::vector<int32_t> qt_classes; // per query tile: C
+  std::vector<int32_t> qt_wfirst;  // per query tile: first window (HR) or -1
+  std::vector<int32_t> qt_real;    // per query tile: real rows
+  int64_t useful_pairs = 0;
+  int64_t n_partial = 0;
+
+  // schedule
+  std::vector<ug::Item> items;               // per (batch, head)
+  std::vector<ug::CombineGroup> combine;     // split groups
+  int n_split_items = 0;
+
+  // device
+  ug::DeviceTables dev;
+  bool dirty = true;
+  int last_launches = 0;
+};
+
+namespace ug {
+// Builds every host table of `p` from its arguments (plan.cpp).
+int build_tables(ultragen_plan_t* p);
+// Rebuilds the schedule (pairing, splitting) from the tile lists (plan.cpp).
+void build_schedule(ultragen_plan_t* p);
+// Fills the RoPE table on the host: [max(H,W)][D/2][2] (cos, sin) floats (plan.cpp).
+std::vector<float> rope_table(const ultragen_plan_t* p);
+}  // namespace ug

@@ -1,0 +1,172 @@
+/*
+ * ultragen.h -- C ABI of the B200 (sm_100a) hot path of UltraGen's hierarchical local
+ * attention (HLA): window-first permuted, block-masked multi-head attention of one MMDiT
+ * layer over the joint sequence [C_T; X; X_lr].
+ *
+ * Sources (page title, then section):
+ *   [UG-note] "UltraGen: Efficient Ultra-High-Resolution Image Generation with Hierarchical
+ *             Local Attention", papernotes.org note (ECCV 2026), 方法详解 / 关键设计 1-3.
+ *   [UG-gist] same title, gist.science summary of arXiv 2510.16325, "2. Methodology" A-B.
+ *
+ * Conventions shared by every call
+ *   - Every function returns an int status (ULTRAGEN_OK or an ULTRAGEN_ERR_* code); no C++
+ *     exception crosses this boundary.  Argument errors are reported before any work.
+ *   - Device pointers are CUDA global-memory pointers of the current device, contiguous,
+ *     16-byte aligned.  The caller owns every tensor; the plan owns its own tables.
+ *   - "stream" is a cudaStream_t (0 = legacy default stream).  Device calls are
+ *     asynchronous on that stream; errors raised by a kernel while it runs (a wait that
+ *     timed out) are read back by ultragen_sync_status().
+ *   - A plan is not thread-safe: do not use one plan from two host threads or on two
+ *     streams at once.  The first device call on a plan uploads its tables with a
+ *     synchronous copy; make that call before any stream capture.
+ *
+ * Sequence layout (the "permuted" layout, readings of the pages listed in the design doc):
+ *   slots [0, T) text | pad to a multiple of 128 | HR tokens window-first (windows row-major,
+ *   l*l slots each, raster order inside; partial edge windows padded) | pad to 128 |
+ *   LR tokens raster | pad to 128.   N_tot = number of slots, a multiple of 128.
+ *   Raster layout: tokens ordered text, HR raster (row i, column j), LR raster.
+ */
+#ifndef ULTRAGEN_H
+#define ULTRAGEN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;                       /* cudaStream_t is struct CUstream_st* */
+typedef struct CUstream_st* ultragen_stream_t;
+
+enum ultragen_status {
+  ULTRAGEN_OK = 0,
+  ULTRAGEN_ERR_INVALID_ARG = 1,   /* null pointer, negative or inconsistent size         */
+  ULTRAGEN_ERR_UNSUPPORTED = 2,   /* head_dim not 64/128, b > l, sizes past int32 limits */
+  ULTRAGEN_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed                   */
+  ULTRAGEN_ERR_OOM = 4,           /* device allocation failed                            */
+  ULTRAGEN_ERR_TIMEOUT = 5,       /* a device-side wait ran past its limit               */
+  ULTRAGEN_ERR_PLAN_MISMATCH = 6, /* plan built for another shape / device               */
+  ULTRAGEN_ERR_NO_DEVICE = 7      /* no sm_100 device is current                         */
+};
+
+enum ultragen_dtype { ULTRAGEN_BF16 = 0, ULTRAGEN_F32 = 1 };
+
+typedef struct ultragen_plan ultragen_plan_t;   /* opaque, owned by the library */
+
+typedef struct {
+  int32_t H, W, l, b, rho, text_len, heads, head_dim;
+  int32_t nWh, nWw;           /* windows per column / per row: ceil(H/l), ceil(W/l)   */
+  int32_t h, w;               /* LR grid: ceil(H/rho), ceil(W/rho); 0 when rho = 0      */
+  int64_t N_raster;           /* text_len + H*W + h*w                                   */
+  int64_t N_tot;              /* slots in the permuted layout                           */
+  int64_t off_hr, off_lr;     /* first slot of the HR and LR segments                   */
+  int32_t n_qtiles;           /* N_tot / 128                                            */
+  int32_t n_items;            /* work items per (batch, head) after pairing/splitting   */
+  int64_t n_entries;          /* tile-list entries (all query tiles)                    */
+  int64_t n_partial;          /* entries that need per-element masking                  */
+  int64_t useful_pairs;       /* visible (query, key) pairs of one head                 */
+  int32_t rope_axes[3];       /* RoPE dims per axis (text/time, row, column)            */
+  double rope_theta;
+  int32_t split_chunk;        /* key tiles per split of a long query group (0 = none)   */
+  int32_t n_split_groups;     /* query groups whose key list is split                   */
+  int32_t n_split_items;      /* items that write split partials (per head)             */
+  int64_t workspace_bytes_per_head; /* split partial storage per (batch, head)          */
+} ultragen_plan_info_t;
+
+/* Human-readable name of a status code.  Never NULL. */
+const char* ultragen_status_string(int status);
+
+/*
+ * ultragen_plan -- build the per-shape plan on the host: window geometry
+ * ([UG-note] 关键设计 1: l x l windows, ceil(H/l) ceil(W/l) of them), the window-first
+ * permutation, the block-sparse tile lists of the mask M ([UG-note] 关键设计 2, last
+ * paragraph; [UG-gist] 2.B "Attention Masking"), the RoPE tables with LR positions scaled
+ * by rho ([UG-note] 关键设计 2, (m,n) -> (rho m, rho n)), and the kernel schedule.
+ *   H, W      HR latent rows / columns (>= 1)
+ *   l         window side in latent tokens (>= 1)
+ *   b         halo width in tokens, 0 <= b <= l: an HR query sees HR keys inside its
+ *             window's box grown by b on each side, clipped to the image
+ *   rho       LR scale (>= 1), or 0 for no LR segment; LR grid is ceil(H/rho) x ceil(W/rho)
+ *   text_len  text tokens (>= 0)
+ *   heads     attention heads (>= 1);  head_dim  64 or 128
+ *   out       receives the plan; release it with ultragen_plan_destroy
+ * Host-only: needs no GPU.  Errors: INVALID_ARG, UNSUPPORTED, OOM (host).
+ */
+int ultragen_plan(int H, int W, int l, int b, int rho, int text_len, int heads,
+                  int head_dim, ultragen_plan_t** out);
+
+/* RoPE split (ax0 + ax1 + ax2 == head_dim, each even) and base theta (> 0).
+ * Default: head_dim 64 -> (16,24,24), 128 -> (16,56,56); theta 1e4.  Axis 0 always has
+ * position 0; axis 1 takes the row (rho*m for LR), axis 2 the column (rho*n for LR). */
+int ultragen_plan_set_rope(ultragen_plan_t* plan, int ax0, int ax1, int ax2, double theta);
+
+/* Split long query groups' key lists into chunks of `chunk` key tiles, merged by a
+ * log-sum-exp combine.  chunk = -1: automatic (the default; chunk = the longest HR/LR
+ * group, applied to groups at least 1.5x longer); chunk = 0: never split. */
+int ultragen_plan_set_split(ultragen_plan_t* plan, int chunk);
+
+int ultragen_plan_info(const ultragen_plan_t* plan, ultragen_plan_info_t* out);
+
+/*
+ * Host copies of the plan's integer tables (caller-allocated host buffers):
+ *   perm     [N_tot]       raster index of each permuted slot, -1 for pad slots
+ *   row_ptr  [n_qtiles+1]  CSR offsets of each query tile's entries
+ *   entries  [n_entries]   key-tile index | (1u << 31 if partial), ascending per tile.
+ * An entry exists iff some (real query row, key column) cell of the 128x128 block is
+ * visible; it is partial iff some such cell is not.  Any pointer may be NULL to skip it.
+ */
+int ultragen_plan_export(const ultragen_plan_t* plan, int32_t* perm, int32_t* row_ptr,
+                         int32_t* entries);
+
+/* Per-row visibility of query tile `qtile`: out[e][r][w] (uint32) for each of the tile's
+ * entries e, rows r in [0,128), words w in [0,4); bit c%32 of word c/32 = key column c of
+ * the entry's key tile visible to row r.  Rows of pad slots are 0.  `out` holds
+ * (row_ptr[qtile+1]-row_ptr[qtile]) * 512 words. */
+int ultragen_plan_export_rowmasks(const ultragen_plan_t* plan, int qtile, uint32_t* out);
+
+int ultragen_plan_destroy(ultragen_plan_t* plan);
+
+/*
+ * ultragen_permute_rope -- raster -> window-first gather of Q, K, V fused with axial 2D
+ * RoPE on Q and K ([UG-note] 关键设计 1 window-first order; 关键设计 2 position scaling).
+ *   q, k, v     [batch, N_raster, heads, head_dim], in_dtype BF16 or F32 (device)
+ *   qp, kp, vp  [batch, heads, N_tot, head_dim] BF16 (device); pad slots written as 0
+ * RoPE is computed in fp32 from fp32 tables and rounded to bf16 (nearest even); V and
+ * text tokens are copied (F32 input: rounded to bf16).
+ */
+int ultragen_permute_rope(const void* q, const void* k, const void* v, int in_dtype,
+                          void* qp, void* kp, void* vp, int batch,
+                          const ultragen_plan_t* plan, ultragen_stream_t stream);
+
+/*
+ * ultragen_hla_forward -- masked joint attention softmax(Q K^T / sqrt(d) + M) V
+ * ([UG-note] 关键设计 3, the MMA equation; M additive -inf on masked pairs) over the
+ * permuted layout, visiting only the key tiles of each query tile's list.
+ *   qp, kp, vp, op  [batch, heads, N_tot, head_dim] BF16 (device); op rows of pad slots = 0
+ * bf16 tensor-core products with fp32 accumulation and fp32 online softmax.  Uses the
+ * plan's split workspace (device memory the plan allocates and keeps) when the plan
+ * splits groups.  Errors: INVALID_ARG, NO_DEVICE, OOM, CUDA.
+ */
+int ultragen_hla_forward(const void* qp, const void* kp, const void* vp, void* op,
+                         const ultragen_plan_t* plan, int batch, ultragen_stream_t stream);
+
+/*
+ * ultragen_unpermute -- window-first -> raster: o[b, t, h, :] = op[b, h, slot(t), :].
+ *   op  [batch, heads, N_tot, head_dim] BF16 (device)
+ *   o   [batch, N_raster, heads, head_dim], out_dtype BF16 (bit copy) or F32 (device)
+ */
+int ultragen_unpermute(const void* op, void* o, int out_dtype, int batch,
+                       const ultragen_plan_t* plan, ultragen_stream_t stream);
+
+/* Wait for `stream`, then report (and clear) a device-side error raised by this plan's
+ * kernels since the last call: ULTRAGEN_ERR_TIMEOUT if a wait ran out. */
+int ultragen_sync_status(const ultragen_plan_t* plan, ultragen_stream_t stream);
+
+/* Kernel launches the last device call of this plan issued (for launch accounting). */
+int ultragen_last_launch_count(const ultragen_plan_t* plan);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ULTRAGEN_H */

@@ -24,6 +24,9 @@ What each function follows:
   * 2D RoPE on Q/K ......................... implied by [UG-note] 关键设计 1 and 3 ("RoPE"),
                                              convention fixed by the readings below
 
+Tables returned by the cached geometry helpers (raster_tokens, slot_of_tokens, perm_map,
+slot_info) are shared between calls: callers must not modify them.
+
 Readings taken where the pages are silent or garbled (each is listed in the design doc):
   R1  l counts latent tokens (l=16 <-> 256x256 pixels at a 16x VAE).
   R2  Halo: the query's own window box grown by b tokens on every side, clipped to the
@@ -49,6 +52,7 @@ the closed forms the pages state (the 256x window reduction at 4K, rho = H/h).
 """
 from __future__ import annotations
 
+import functools
 import math
 from dataclasses import dataclass
 
@@ -126,6 +130,7 @@ class Geometry:
 # Tokens, raster order and the window-first permutation
 # --------------------------------------------------------------------------------------
 
+@functools.lru_cache(maxsize=8)
 def raster_tokens(g: Geometry):
     """Every token of [C_T; X; X_lr] in raster order: (segment, a, b) per token.
 
@@ -151,6 +156,7 @@ def raster_tokens(g: Geometry):
     return seg, ca, cb
 
 
+@functools.lru_cache(maxsize=8)
 def slot_of_tokens(g: Geometry) -> np.ndarray:
     """Permuted slot of every raster token (window-first order, [UG-note] 关键设计 1; R8, R13).
 
@@ -170,6 +176,7 @@ def slot_of_tokens(g: Geometry) -> np.ndarray:
     return slot
 
 
+@functools.lru_cache(maxsize=8)
 def perm_map(g: Geometry) -> np.ndarray:
     """pi: permuted slot -> raster index, -1 for pad slots."""
     perm = np.full(g.N_tot, -1, np.int64)
@@ -177,6 +184,7 @@ def perm_map(g: Geometry) -> np.ndarray:
     return perm
 
 
+@functools.lru_cache(maxsize=8)
 def slot_info(g: Geometry):
     """Per permuted slot: segment (PAD for pad slots) and the token's two coordinates."""
     seg_r, ca_r, cb_r = raster_tokens(g)

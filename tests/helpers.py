@@ -1,0 +1,53 @@
+"""Shared test helpers: the tolerance check and oracle runs on sampled rows/heads."""
+import numpy as np
+
+from oracle import hla_oracle as O
+
+MAX_ABS = 2e-2      # attention output from bf16 inputs: max |gpu - oracle| over real rows
+MEAN_REL = 5e-3     # sum |gpu - oracle| / sum |oracle| over the same elements
+
+
+def to_np64(t):
+    import torch
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def geometry(wl):
+    return O.Geometry(wl.H, wl.W, wl.l, wl.b, wl.rho, wl.T)
+
+
+def check_attention(got, ref, what=""):
+    d = np.abs(got - ref)
+    max_abs = float(d.max()) if d.size else 0.0
+    mean_rel = float(d.sum() / max(np.abs(ref).sum(), 1e-30))
+    assert max_abs <= MAX_ABS and mean_rel <= MEAN_REL, (
+        f"{what}: max_abs {max_abs:.3e} (<= {MAX_ABS}), mean_rel {mean_rel:.3e} (<= {MEAN_REL})")
+    return max_abs, mean_rel
+
+
+def oracle_rows(q, k, v, wl, b, heads, rows):
+    """Oracle output [len(heads), len(rows), D] for batch b, the given heads and permuted rows."""
+    g = geometry(wl)
+    out = []
+    for h in heads:
+        qh = to_np64(q[b:b + 1, :, h:h + 1, :])
+        kh = to_np64(k[b:b + 1, :, h:h + 1, :])
+        vh = to_np64(v[b:b + 1, :, h:h + 1, :])
+        o, _ = O.forward(qh, kh, vh, g, wl.axes, rows=rows)
+        out.append(o[0, 0])
+    return np.stack(out)
+
+
+def sample_rows(wl, n_text=16, n_lr=32, windows="corners"):
+    """Permuted rows to check at full size: text rows, whole windows (corner, edge, interior,
+    and the last column for ragged grids), LR rows."""
+    g = geometry(wl)
+    rows = list(np.linspace(0, max(0, g.T - 1), min(n_text, g.T)).astype(int)) if g.T else []
+    l2 = g.l * g.l
+    wins = {0, g.nWw - 1, (g.nWh - 1) * g.nWw, g.nWh * g.nWw - 1,
+            (g.nWh // 2) * g.nWw + g.nWw // 2, g.nWw // 2, (g.nWh // 2) * g.nWw}
+    for w in sorted(wins):
+        rows += list(range(g.off_hr + w * l2, g.off_hr + (w + 1) * l2))
+    if g.N_lr:
+        rows += list(np.linspace(g.off_lr, g.off_lr + g.N_lr - 1, min(n_lr, g.N_lr)).astype(int))
+    return np.array(sorted(set(int(r) for r in rows)), np.int64)

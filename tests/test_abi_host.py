@@ -1,0 +1,156 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol of
+include/ultragen.h, rejects bad arguments, and its host plan (permutation, tile lists,
+per-row masks, pair counts) is bit-exact against the oracle's explicit mask."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import hla_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="session")
+def ffi():
+    from diffusion_transformer_ultra_b200 import build
+    build.build()
+    from diffusion_transformer_ultra_b200 import _ffi
+    return _ffi
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "ultragen.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\**\s+\**(ultragen_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_every_declared_symbol_is_exported(ffi):
+    names = header_functions()
+    assert len(names) >= 13
+    lib = ctypes.CDLL(ffi.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(ffi.SYMBOLS)
+
+
+def test_status_strings(ffi):
+    L = ffi.lib()
+    for code in range(8):
+        assert L.ultragen_status_string(code).decode()
+    assert L.ultragen_status_string(99).decode() == "unknown status"
+
+
+@pytest.mark.parametrize("args,status", [
+    ((0, 8, 4, 1, 2, 3, 1, 64), 1),     # H < 1
+    ((8, 8, 4, 5, 2, 3, 1, 64), 2),     # b > l
+    ((8, 8, 4, 1, -1, 3, 1, 64), 1),    # rho < 0
+    ((8, 8, 4, 1, 2, 3, 1, 96), 2),     # head_dim not 64/128
+    ((8, 8, 0, 0, 2, 3, 1, 64), 1),     # l < 1
+    ((8, 8, 4, 1, 2, -3, 1, 64), 1),    # text_len < 0
+])
+def test_plan_rejects_bad_arguments(ffi, args, status):
+    h = ctypes.c_void_p()
+    assert ffi.lib().ultragen_plan(*args, ctypes.byref(h)) == status
+    assert not h.value
+
+
+def test_set_rope_validation(ffi):
+    p = ffi.Plan(8, 8, 4, 1, 2, 3, 1, 64)
+    L = ffi.lib()
+    assert L.ultragen_plan_set_rope(p.handle, 16, 24, 22, 1e4) == 1   # sum != D
+    assert L.ultragen_plan_set_rope(p.handle, 15, 25, 24, 1e4) == 1   # odd
+    assert L.ultragen_plan_set_rope(p.handle, 16, 24, 24, -1.0) == 1
+    assert L.ultragen_plan_set_rope(p.handle, 0, 32, 32, 5e3) == 0
+    p._refresh()
+    assert p.info["rope_axes"] == (0, 32, 32) and p.info["rope_theta"] == 5e3
+
+
+def test_device_calls_without_device_fail_cleanly(ffi):
+    """On a host with no GPU the device entry points return an error status, never crash."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    p = ffi.Plan(8, 8, 4, 1, 2, 3, 1, 64)
+    L = ffi.lib()
+    buf = ctypes.create_string_buffer(1 << 16)
+    a = ctypes.addressof(buf) + (-ctypes.addressof(buf)) % 16
+    st = L.ultragen_hla_forward(a, a, a, a, p.handle, 1, None)
+    assert st in (3, 7)
+    assert L.ultragen_hla_forward(None, a, a, a, p.handle, 1, None) == 1
+    assert L.ultragen_permute_rope(a, a, a, 5, a, a, a, 1, p.handle, None) == 1
+
+
+GEOMS = {
+    "tiny": (32, 32, 8, 2, 4, 16),
+    "1k": (64, 64, 16, 4, 4, 512),
+    "ragged": (256, 135, 16, 16, 4, 256),
+    "odd": (37, 29, 12, 5, 3, 70),
+    "small_l": (20, 18, 4, 3, 5, 9),
+    "no_lr_text": (40, 24, 8, 8, 0, 0),
+}
+
+
+def sample_qtiles(g, n_hr=40, seed=0):
+    nq = g.N_tot // 128
+    text = list(range(0, g.off_hr // 128))
+    lr = list(range(g.off_lr // 128, nq))
+    hr = list(range(g.off_hr // 128, g.off_lr // 128))
+    rng = np.random.default_rng(seed)
+    pick = sorted(set(hr[:4] + hr[-4:] + list(rng.choice(hr, size=min(n_hr, len(hr)), replace=False))))
+    return sorted(set(text + lr[:3] + lr[-3:] + pick))
+
+
+def compare_plan(ffi, geom, qtiles=None):
+    g = O.Geometry(*geom)
+    p = ffi.Plan(*geom, 2, 64)
+    info = p.info
+    assert info["N_tot"] == g.N_tot and info["N_raster"] == g.N_raster
+    assert info["off_hr"] == g.off_hr and info["off_lr"] == g.off_lr
+    perm, row_ptr, entries = p.export()
+    np.testing.assert_array_equal(perm, O.perm_map(g))
+    qtiles = range(g.N_tot // 128) if qtiles is None else qtiles
+    for t in qtiles:
+        e_ref, m_ref = O.qtile_entries(g, t)
+        e_got = entries[row_ptr[t]:row_ptr[t + 1]].view(np.uint32)
+        np.testing.assert_array_equal(e_got, e_ref, err_msg=f"q-tile {t}")
+        np.testing.assert_array_equal(p.rowmasks(t, len(e_ref)), m_ref, err_msg=f"q-tile {t} masks")
+    return g, p
+
+
+@pytest.mark.parametrize("name", ["tiny", "1k", "odd", "small_l", "no_lr_text"])
+def test_plan_bit_exact_full(ffi, name):
+    g, p = compare_plan(ffi, GEOMS[name])
+    assert p.info["useful_pairs"] == O.visible_pair_count(g)
+
+
+@pytest.mark.parametrize("name", ["ragged"])
+def test_plan_bit_exact_sampled(ffi, name):
+    compare_plan(ffi, GEOMS[name], sample_qtiles(O.Geometry(*GEOMS[name])))
+
+
+def test_plan_4k_8k_sampled_and_pair_counts(ffi):
+    import sys
+    sys.path.insert(0, os.path.dirname(__file__))
+    from test_oracle_pins import closed_form_pairs
+    for side in (256, 512):
+        geom = (side, side, 16, 4, 4, 512)
+        g = O.Geometry(*geom)
+        _, p = compare_plan(ffi, geom, sample_qtiles(g, n_hr=12))
+        assert p.info["useful_pairs"] == sum(closed_form_pairs(*geom).values())
+    # the totals quoted for these layers: 390,873,088 (4K) and 4,988,354,560 (8K) pairs per head
+    assert sum(closed_form_pairs(256, 256, 16, 4, 4, 512).values()) == 390_873_088
+    assert sum(closed_form_pairs(512, 512, 16, 4, 4, 512).values()) == 4_988_354_560
+
+
+def test_split_policy(ffi):
+    p = ffi.Plan(256, 256, 16, 4, 4, 512, 24, 128)
+    i = p.info
+    assert i["split_chunk"] == 48 and i["n_split_groups"] == 2
+    p.set_split(0)
+    assert p.info["n_split_groups"] == 0 and p.info["workspace_bytes_per_head"] == 0
+    p.set_split(7)
+    assert p.info["split_chunk"] == 7 and p.info["n_split_groups"] > 2
+    assert p.info["workspace_bytes_per_head"] == p.info["n_split_items"] * 2 * 128 * 129 * 4
