@@ -38,6 +38,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="4k")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="override the workload's head count (smaller profiling captures)")
     ap.add_argument("--impl", default="ultragen", choices=["ultragen", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -209,6 +211,9 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
 
     wl = ug.WORKLOADS[args.workload]
+    if args.heads:
+        import dataclasses
+        wl = dataclasses.replace(wl, heads=args.heads)
     plan = ug.plan_for(wl)
     info = plan.info
     q, k, v = ug.make_qkv(wl)

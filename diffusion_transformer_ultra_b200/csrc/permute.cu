@@ -40,8 +40,10 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 
 }  // namespace
 
-// One thread = one 16-byte output chunk of one output row; a block covers ROWS rows per
-// pass and each thread handles U rows per pass so that U loads are in flight together.
+// One thread = one 16-byte chunk of one output row.  Rows are visited in (batch, slot, head)
+// order, so the heads of one token -- contiguous in the raster input -- are read together
+// (heads x D x 2 bytes in one run) while each output row is written whole.  Each thread
+// handles U rows per pass so that U loads are in flight together.
 template <typename Tin, int D>
 __global__ void __launch_bounds__(256) permute_rope_kernel(PermuteArgs a) {
   constexpr int CH = D / 8;
@@ -50,38 +52,41 @@ __global__ void __launch_bounds__(256) permute_rope_kernel(PermuteArgs a) {
   constexpr int HALF = D / 2;
   const int which = blockIdx.y;
   const bool do_rope = which < 2;
-  const Tin* __restrict__ in = static_cast<const Tin*>(a.in[which]);
-  __nv_bfloat16* __restrict__ out = a.out[which];
+  const Tin* __restrict__ in =
+      static_cast<const Tin*>(which == 0 ? a.in[0] : (which == 1 ? a.in[1] : a.in[2]));
+  __nv_bfloat16* __restrict__ out = which == 0 ? a.out[0] : (which == 1 ? a.out[1] : a.out[2]);
   const int c = threadIdx.x % CH;
   const int rsub = threadIdx.x / CH;
-  const int64_t step = (int64_t)gridDim.x * ROWS * U;
+  const int rows_total = (int)a.rows_total;          // < 2^31, checked by the caller
+  const int step = gridDim.x * ROWS * U;
 
-  for (int64_t row0 = (int64_t)blockIdx.x * ROWS * U; row0 < a.rows_total; row0 += step) {
+  for (int row0 = blockIdx.x * ROWS * U; row0 < rows_total; row0 += step) {
     float x[U][8];
     int pos_r[U], pos_c[U];
-    bool live[U], real[U];
+    int dst[U];                                       // output row, -1 when out of range
+    bool real[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int64_t row = row0 + u * ROWS + rsub;
-      live[u] = row < a.rows_total;
+      const int row = row0 + u * ROWS + rsub;         // (b, slot, h)
+      dst[u] = -1;
       real[u] = false;
-      if (!live[u]) continue;
-      const int slot = (int)(row % a.N_tot);
-      const int64_t bh = row / a.N_tot;
-      const int h = (int)(bh % a.heads);
-      const int b = (int)(bh / a.heads);
+      if (row >= rows_total) continue;
+      const int h = row % a.heads;
+      const int bs = row / a.heads;
+      const int slot = bs % a.N_tot;
+      const int b = bs / a.N_tot;
+      dst[u] = (b * a.heads + h) * a.N_tot + slot;
       const int r = __ldg(a.perm + slot);
       if (r < 0) continue;
       real[u] = true;
       const uint32_t sp = __ldg(a.slot_pos + slot);
       pos_r[u] = (int)(sp >> 16);
       pos_c[u] = (int)(sp & 0xffffu);
-      load8(in + (((int64_t)b * a.N_raster + r) * a.heads + h) * D + c * 8, x[u]);
+      load8(in + ((int64_t)(b * a.N_raster + r) * a.heads + h) * D + c * 8, x[u]);
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      if (!live[u]) continue;
-      const int64_t row = row0 + u * ROWS + rsub;
+      if (dst[u] < 0) continue;
       uint4 o = make_uint4(0u, 0u, 0u, 0u);
       if (real[u]) {
         if (do_rope) {
@@ -90,7 +95,7 @@ __global__ void __launch_bounds__(256) permute_rope_kernel(PermuteArgs a) {
             const int q = c * 4 + k;                       // rotation pair index
             const int pos = q < a.pair_a0 ? 0 : (q < a.pair_a01 ? pos_r[u] : pos_c[u]);
             if (pos != 0) {
-              const float2 cs = __ldg(reinterpret_cast<const float2*>(a.rope) + (int64_t)pos * HALF + q);
+              const float2 cs = __ldg(reinterpret_cast<const float2*>(a.rope) + pos * HALF + q);
               const float x0 = x[u][2 * k], x1 = x[u][2 * k + 1];
               x[u][2 * k] = x0 * cs.x - x1 * cs.y;
               x[u][2 * k + 1] = x0 * cs.y + x1 * cs.x;
@@ -102,7 +107,7 @@ __global__ void __launch_bounds__(256) permute_rope_kernel(PermuteArgs a) {
         o.z = pack_bf16(x[u][4], x[u][5]);
         o.w = pack_bf16(x[u][6], x[u][7]);
       }
-      *reinterpret_cast<uint4*>(out + row * D + c * 8) = o;
+      *reinterpret_cast<uint4*>(out + (int64_t)dst[u] * D + c * 8) = o;
     }
   }
 }
@@ -114,25 +119,26 @@ __global__ void __launch_bounds__(256) unpermute_kernel(UnpermuteArgs a) {
   constexpr int U = 4;
   const int c = threadIdx.x % CH;
   const int rsub = threadIdx.x / CH;
-  const int64_t step = (int64_t)gridDim.x * ROWS * U;
+  const int rows_total = (int)a.rows_total;          // < 2^31, checked by the caller
+  const int step = gridDim.x * ROWS * U;
   Tout* __restrict__ out = static_cast<Tout*>(a.out);
-  for (int64_t row0 = (int64_t)blockIdx.x * ROWS * U; row0 < a.rows_total; row0 += step) {
+  for (int row0 = blockIdx.x * ROWS * U; row0 < rows_total; row0 += step) {
     uint4 v[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int64_t row = row0 + u * ROWS + rsub;      // (b, t, h) raster row
-      if (row >= a.rows_total) continue;
-      const int h = (int)(row % a.heads);
-      const int64_t bt = row / a.heads;
-      const int t = (int)(bt % a.N_raster);
-      const int b = (int)(bt / a.N_raster);
+      const int row = row0 + u * ROWS + rsub;          // (b, t, h) raster row
+      if (row >= rows_total) continue;
+      const int h = row % a.heads;
+      const int bt = row / a.heads;
+      const int t = bt % a.N_raster;
+      const int b = bt / a.N_raster;
       const int slot = __ldg(a.inv_perm + t);
-      v[u] = __ldg(reinterpret_cast<const uint4*>(a.in + (((int64_t)b * a.heads + h) * a.N_tot + slot) * D + c * 8));
+      v[u] = __ldg(reinterpret_cast<const uint4*>(a.in + ((int64_t)(b * a.heads + h) * a.N_tot + slot) * D + c * 8));
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int64_t row = row0 + u * ROWS + rsub;
-      if (row >= a.rows_total) continue;
+      if (row >= rows_total) continue;
       if constexpr (sizeof(Tout) == 2) {
         *reinterpret_cast<uint4*>(out + row * D + c * 8) = v[u];
       } else {

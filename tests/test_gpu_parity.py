@@ -1,7 +1,8 @@
 """GPU parity of the CUDA path against the fp64 oracle, through the C ABI.
 
 Bars: permutation and V gather bit-exact; Q/K after RoPE within 1 bf16 ulp of the oracle's
-fp64 RoPE rounded to nearest-even; attention output within max-abs 2e-2 and mean-rel 5e-3
+fp64 RoPE rounded to nearest-even, plus the fp32 rotation error bound (see FP32_ROT);
+attention output within max-abs 2e-2 and mean-rel 5e-3
 of the oracle on every real row (pad rows exactly 0).
 """
 import dataclasses
@@ -64,13 +65,30 @@ def custom(name):
 
 
 def expected_qkv_perm(wl, q, k, v, b, h):
+    """Oracle RoPE'd, permuted Q, K (rounded to bf16), V, and the per-element pair magnitude
+    |x_2k| + |x_2k+1| of the unrotated inputs."""
     g = geometry(wl)
     pos = O.positions(g)
     qh, kh, vh = (to_np64(x[b:b + 1, :, h:h + 1, :]) for x in (q, k, v))
     qp = O.permute(O.rope(qh, pos, wl.axes), g)[0, 0]
     kp = O.permute(O.rope(kh, pos, wl.axes), g)[0, 0]
     vp = O.permute(vh, g)[0, 0]
-    return O.round_bf16(qp), O.round_bf16(kp), O.round_bf16(vp)
+
+    def pair_mag(x):
+        xp = np.abs(O.permute(x, g)[0, 0])
+        s = xp[:, 0::2] + xp[:, 1::2]
+        return np.repeat(s, 2, axis=1)
+
+    return (O.round_bf16(qp), O.round_bf16(kp), O.round_bf16(vp), pair_mag(qh), pair_mag(kh))
+
+
+# RoPE is evaluated in fp32 from fp32 cos/sin tables, then rounded to bf16 (nearest even).
+# Against the fp64 rotation rounded to bf16, an element may differ by one bf16 ulp (the
+# rounding of a value that moved across a tie) plus the fp32 evaluation error, which is
+# bounded by 2^-22 * (|x_2k| + |x_2k+1|): table rounding of cos and sin (2^-24 each, relative)
+# and at most two product/sum roundings.  The second term only matters where the rotation
+# cancels to a value far below the pair's magnitude.
+FP32_ROT = 2.0 ** -22
 
 
 def ulp_bf16(x):
@@ -86,12 +104,15 @@ def test_permute_rope_parity(ug, name):
     heads = range(wl.heads) if wl.heads <= 3 else (0, wl.heads // 2, wl.heads - 1)
     for b in range(wl.batch):
         for h in heads:
-            eq, ek, ev = expected_qkv_perm(wl, q, k, v, b, h)
+            eq, ek, ev, mq, mk = expected_qkv_perm(wl, q, k, v, b, h)
             gq, gk, gv = (to_np64(t[b, h]) for t in (lay.qp, lay.kp, lay.vp))
             np.testing.assert_array_equal(gv, ev, err_msg="V gather must be bit-exact")
-            for got, exp, nm in ((gq, eq, "Q"), (gk, ek, "K")):
-                bad = np.abs(got - exp) > ulp_bf16(exp) * 1.0000001
-                assert not bad.any(), f"{nm} off by more than 1 bf16 ulp at {np.argwhere(bad)[:5]}"
+            for got, exp, mag, nm in ((gq, eq, mq, "Q"), (gk, ek, mk, "K")):
+                tol = ulp_bf16(np.maximum(np.abs(got), np.abs(exp))) + FP32_ROT * mag
+                bad = np.abs(got - exp) > tol
+                assert not bad.any(), f"{nm} outside 1 ulp + fp32 bound at {np.argwhere(bad)[:5]}"
+                # almost every element is within one plain ulp
+                assert (np.abs(got - exp) > ulp_bf16(exp)).mean() < 1e-5
     # text tokens and axis-0 dims are copies
     g = geometry(wl)
     if g.T:
