@@ -5,12 +5,16 @@
 // pairs), visiting for each query tile only the key tiles its plan list names; masks are
 // applied per element on partial tiles only.
 //
-// CTA organisation (one persistent CTA per SM, 320 threads):
+// CTA organisation (one persistent CTA per SM, 384 threads = 3 warpgroups):
 //   warps 0-3   softmax group 0: owns query tile slot 0 (thread = row, TMEM lane = row)
 //   warps 4-7   softmax group 1: owns query tile slot 1
 //   warp  8     producer: TMA loads of Q (per item) and of K, V tiles into a ring
 //   warp  9     MMA issuer: tcgen05.mma for S = Q K^T (both operands in shared memory) and
 //               O += P V (P read from TMEM, V from shared memory); owns TMEM allocation
+//   warps 10-11 idle
+// The kernel is compiled for 168 registers per thread (384 x 168 = 64,512); the control
+// warpgroup gives registers back (setmaxnreg 56) so the softmax groups can hold a whole
+// 128-column S row in registers (setmaxnreg 224): 2 x 128 x 224 + 128 x 56 = 64,512.
 // A work item is one or two query tiles with the same key list (the two 128-row halves of
 // a 16x16 window, two text tiles, two LR tiles), so each K/V tile is loaded once per two
 // query tiles.  The issue order S0(j) / S1(j) / [P0 V(j)] / S0(j+1) ... lets one softmax
@@ -26,6 +30,7 @@
 
 #include <cstdint>
 
+#include "exp2_poly.h"
 #include "kernels.h"
 #include "ptx.cuh"
 
@@ -50,12 +55,43 @@ struct FwdCfg {
   static constexpr uint32_t O_COL = 256;
 };
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
+constexpr int kRegsLaunch = 168;      // per thread at launch: 65536 / 384, rounded down to 8
+constexpr int kRegsSoftmax = 224;
+constexpr int kRegsControl = 56;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kThreads * kRegsLaunch,
+              "register split exceeds the launch allocation");
 constexpr int kWarpProducer = 8;
 constexpr int kWarpMma = 9;
 constexpr uint64_t kDrainNs = 50ull * 1000 * 1000;   // bounded drain on the abort path
 
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
+
+// 2^x for a pair of arguments on the FMA pipe (Cody-Waite range reduction + minimax
+// polynomial): n = round(x) by the 1.5 * 2^23 shifter, f = x - n in [-1/2, 1/2],
+// 2^x = 2^n * p(f), with n added to the exponent field as an integer.  x is clamped at -125
+// so the result stays a normal float; 2^-125 then stands for 0 (masked entries), far below
+// any visible weight.
+__device__ __forceinline__ float2 ex2_fma2(float2 x) {
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 t = fadd2(x, make_float2(12582912.0f, 12582912.0f));
+  const float2 u = fadd2(t, make_float2(-12582912.0f, -12582912.0f));
+  const float2 f = ffma2(u, make_float2(-1.0f, -1.0f), x);
+  float2 p = ffma2(f, make_float2(UG_EXP2_C3, UG_EXP2_C3), make_float2(UG_EXP2_C2, UG_EXP2_C2));
+  p = ffma2(f, p, make_float2(UG_EXP2_C1, UG_EXP2_C1));
+  p = ffma2(f, p, make_float2(UG_EXP2_C0, UG_EXP2_C0));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
+// Which exponential pairs (of the 64 in a row of a tile) go to ex2_fma2 instead of the SFU.
+#ifndef UG_FMA_EXP_MASK
+#define UG_FMA_EXP_MASK 0
+#endif
+__device__ __forceinline__ constexpr bool pair_on_fma(int c2) {
+  return ((UG_FMA_EXP_MASK >> (c2 & 7)) & 1) != 0;
+}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -272,18 +308,22 @@ __device__ void softmax_role(const FwdParams& p, uint32_t sbase, uint32_t tbase,
       tc_fence_after();
       uint32_t s[128];
       tmem_ld128_sync(tS, s);
-      float mx = neg_inf();
+      // row max (the row is thread-local: no shuffles), 4 chains of three-input max
       if (ent < 0) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const float v = ((mw[c >> 5] >> (c & 31)) & 1u) ? __uint_as_float(s[c]) : neg_inf();
-          s[c] = __float_as_uint(v);
-          mx = fmaxf(mx, v);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
+        for (int c = 0; c < 128; ++c)
+          if (!((mw[c >> 5] >> (c & 31)) & 1u)) s[c] = 0xff800000u;   // -inf
       }
+      float mx4[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) mx4[i] = neg_inf();
+#pragma unroll
+      for (int c = 0; c < 128; c += 8) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          mx4[i] = fmax3(mx4[i], __uint_as_float(s[c + 2 * i]), __uint_as_float(s[c + 2 * i + 1]));
+      }
+      const float mx = fmax3(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]);
       const float mnew = fmaxf(m, mx * scale);
       if (j == 0) {
         m = mnew;
@@ -309,19 +349,33 @@ __device__ void softmax_role(const FwdParams& p, uint32_t sbase, uint32_t tbase,
         }
       }
       const float mu = (m == neg_inf()) ? 0.f : m;
+      const float2 scale2 = make_float2(scale, scale), nmu2 = make_float2(-mu, -mu);
+      float2 ls[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) ls[i] = make_float2(0.f, 0.f);
 #pragma unroll
       for (int c2 = 0; c2 < 64; ++c2) {
-        const float p0 = ex2(fmaf(__uint_as_float(s[2 * c2]), scale, -mu));
-        const float p1 = ex2(fmaf(__uint_as_float(s[2 * c2 + 1]), scale, -mu));
-        lsum += p0 + p1;
-        s[c2] = pack_bf16x2(p0, p1);
+        const float2 x =
+            ffma2(make_float2(__uint_as_float(s[2 * c2]), __uint_as_float(s[2 * c2 + 1])), scale2, nmu2);
+        float2 pp;
+        if (pair_on_fma(c2)) {
+          pp = ex2_fma2(x);
+        } else {
+          pp.x = ex2(x.x);
+          pp.y = ex2(x.y);
+        }
+        ls[c2 & 3] = fadd2(ls[c2 & 3], pp);
+        s[c2] = pack_bf16x2(pp.x, pp.y);
       }
+      const float2 l2 = fadd2(fadd2(ls[0], ls[1]), fadd2(ls[2], ls[3]));
+      lsum += l2.x + l2.y;
       __syncwarp();
       tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(&s[0]));
       tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(&s[32]));
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar + 8 * (C::B_PF + t));
+      __syncwarp();
+      if ((threadIdx.x & 31) == 0) mbar_arrive(bar + 8 * (C::B_PF + t));
     }
     bool ok = mbar_wait(bar + 8 * (C::B_OF + t), oc & 1, abort_flag, p.err, DEV_TIMEOUT_SOFTMAX,
                         p.timeout_ns);
@@ -391,7 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar + 8 * (C::B_SF + t), 1);
-      mbar_init(bar + 8 * (C::B_PF + t), 128);
+      mbar_init(bar + 8 * (C::B_PF + t), 4);      // one arrive per softmax warp
       mbar_init(bar + 8 * (C::B_OF + t), 1);
     }
     mbar_init(bar + 8 * C::B_DRAIN, 1);
@@ -412,11 +466,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tbase = misc[0];
 
-  if (warp == kWarpProducer) {
-    if (lane == 0) producer_role<D>(&tmQ, &tmK, &tmV, p, sbase, abort_flag);
-  } else if (warp == kWarpMma) {
-    if (lane == 0) mma_role<D>(p, sbase, tbase, abort_flag);
+  if (warp >= 8) {
+    regs_shrink<kRegsControl>();
+    if (warp == kWarpProducer) {
+      if (lane == 0) producer_role<D>(&tmQ, &tmK, &tmV, p, sbase, abort_flag);
+    } else if (warp == kWarpMma) {
+      if (lane == 0) mma_role<D>(p, sbase, tbase, abort_flag);
+    }
   } else {
+    regs_grow<kRegsSoftmax>();
     softmax_role<D>(p, sbase, tbase, abort_flag);
   }
 
@@ -435,7 +493,13 @@ static cudaError_t launch_d(const void* tmQ, const void* tmK, const void* tmV, c
   static bool attr_set = false;
   const int smem = FwdCfg<D>::SMEM_BYTES;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(hla_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    // The register split above is only sound if the kernel really launches with
+    // kRegsLaunch registers per thread; refuse to launch otherwise.
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, hla_fwd_kernel<D>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != kRegsLaunch) return cudaErrorInvalidConfiguration;
+    e = cudaFuncSetAttribute(hla_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
