@@ -109,6 +109,22 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def max_over_ranks(x: float, world: int, device) -> float:
+    """Largest value of x over all ranks (the job is as slow as its slowest rank)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(flops_per_rank: float, world: int, ms_per_step: float) -> float:
+    """Whole-job useful TFLOP/s: every rank runs its own layer (weak scaling)."""
+    return flops_per_rank * world / (ms_per_step * 1e-3) / 1e12
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     for f in ("hla_fwd.cu", "ptx.cuh", "kernels.h"):
@@ -268,13 +284,10 @@ def main():
     ms_perm = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     ms_attn = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     ms_unperm = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
-    t = torch.tensor([ms_total], device="cuda")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_step = float(t.item()) / args.steps
+    ms_step = max_over_ranks(ms_total, world, "cuda") / args.steps
 
     flops = 4.0 * wl.D * info["useful_pairs"] * wl.heads * wl.batch
-    value = flops * world / (ms_step * 1e-3) / 1e12
+    value = job_tflops(flops, world, ms_step)
     pk, src = peaks()
     attn_tflops = flops / (ms_attn * 1e-3) / 1e12
     peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
@@ -301,11 +314,8 @@ def main():
             oh.copy_(o, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
-        t2 = torch.tensor([e0.elapsed_time(e1) / n_e2e], device="cuda")
-        if world > 1:
-            dist.all_reduce(t2, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t2.item())
-        e2e = {"value": flops * world / (ms_e2e * 1e-3) / 1e12, "unit": "useful TFLOP/s",
+        ms_e2e = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world, "cuda")
+        e2e = {"value": job_tflops(flops, world, ms_e2e), "unit": "useful TFLOP/s",
                "ms_per_step": ms_e2e,
                "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
                "d2h_bytes_per_step": o.numel() * o.element_size()}
