@@ -4,8 +4,8 @@ The compute lives in ``libultragen.so`` (hand-written CUDA behind a C ABI, see
 ``include/ultragen.h``); this package holds its ctypes binding, the in-tree build script and
 the seeded synthetic-input generator.
 """
-from ._ffi import (BF16, F32, Layer, Plan, UltragenError, hla_forward, lib,  # noqa: F401
-                   permute_rope, unpermute)
+from ._ffi import (BF16, F32, Layer, Plan, UltragenError, hla_forward,  # noqa: F401
+                   hla_forward_noalloc, lib, permute_rope, unpermute)
 from .inputs import WORKLOADS, Workload, make_qkv  # noqa: F401
 
 

@@ -28,6 +28,7 @@ SYMBOLS = (
     "ultragen_plan_info", "ultragen_plan_export", "ultragen_plan_export_rowmasks",
     "ultragen_plan_destroy", "ultragen_permute_rope", "ultragen_hla_forward",
     "ultragen_unpermute", "ultragen_sync_status", "ultragen_last_launch_count",
+    "ultragen_hla_forward_noalloc",
 )
 
 
@@ -81,6 +82,7 @@ def lib() -> ctypes.CDLL:
     L.ultragen_plan_destroy.argtypes = [vp]
     L.ultragen_permute_rope.argtypes = [vp, vp, vp, cint, vp, vp, vp, cint, vp, vp]
     L.ultragen_hla_forward.argtypes = [vp, vp, vp, vp, vp, cint, vp]
+    L.ultragen_hla_forward_noalloc.argtypes = [vp, vp, vp, vp, vp, cint, vp]
     L.ultragen_unpermute.argtypes = [vp, vp, cint, cint, vp, vp]
     L.ultragen_sync_status.argtypes = [vp, vp]
     L.ultragen_last_launch_count.argtypes = [vp]
@@ -202,6 +204,21 @@ def hla_forward(qp, kp, vp, op, plan: Plan, stream=None):
     for t, n in ((qp, "qp"), (kp, "kp"), (vp, "vp"), (op, "op")):
         _need(t, shape, (torch.bfloat16,), n)
     _check("ultragen_hla_forward", lib().ultragen_hla_forward(
+        qp.data_ptr(), kp.data_ptr(), vp.data_ptr(), op.data_ptr(), plan.handle, B,
+        _stream_ptr(stream)))
+
+
+def hla_forward_noalloc(qp, kp, vp, op, plan: Plan, stream=None):
+    """hla_forward without any device allocation: split partials go to the library's fixed
+    scratch array.  The plan's tables must already be on the device (any earlier device call
+    with this plan uploads them)."""
+    import torch
+    i = plan.info
+    B = qp.shape[0]
+    shape = (B, i["heads"], i["N_tot"], i["head_dim"])
+    for t, n in ((qp, "qp"), (kp, "kp"), (vp, "vp"), (op, "op")):
+        _need(t, shape, (torch.bfloat16,), n)
+    _check("ultragen_hla_forward_noalloc", lib().ultragen_hla_forward_noalloc(
         qp.data_ptr(), kp.data_ptr(), vp.data_ptr(), op.data_ptr(), plan.handle, B,
         _stream_ptr(stream)))
 

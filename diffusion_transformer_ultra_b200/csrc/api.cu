@@ -86,6 +86,20 @@ int ensure_device(ultragen_plan_t* p) {
   return ULTRAGEN_OK;
 }
 
+int grid_for(int64_t rows, int rows_per_block) {
+  const int64_t need = (rows + rows_per_block - 1) / rows_per_block;
+  const int64_t cap = (int64_t)sm_count() * 8;
+  return (int)std::max<int64_t>(1, std::min(need, cap));
+}
+
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return ULTRAGEN_OK;
+  cudaGetLastError();
+  return e == cudaErrorMemoryAllocation ? ULTRAGEN_ERR_OOM : ULTRAGEN_ERR_CUDA;
+}
+
+}  // namespace
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -128,19 +142,6 @@ int sm_count() {
   return n > 0 ? n : 148;
 }
 
-int grid_for(int64_t rows, int rows_per_block) {
-  const int64_t need = (rows + rows_per_block - 1) / rows_per_block;
-  const int64_t cap = (int64_t)sm_count() * 8;
-  return (int)std::max<int64_t>(1, std::min(need, cap));
-}
-
-int cuda_status(cudaError_t e) {
-  if (e == cudaSuccess) return ULTRAGEN_OK;
-  cudaGetLastError();
-  return e == cudaErrorMemoryAllocation ? ULTRAGEN_ERR_OOM : ULTRAGEN_ERR_CUDA;
-}
-
-}  // namespace
 }  // namespace ug
 
 using namespace ug;

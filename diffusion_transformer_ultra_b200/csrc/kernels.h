@@ -1,6 +1,7 @@
 // Argument blocks and launchers of the device kernels (host side includes this).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -59,6 +60,10 @@ cudaError_t launch_permute_rope(const PermuteArgs& a, int in_dtype, int D, int g
 cudaError_t launch_unpermute(const UnpermuteArgs& a, int out_dtype, int D, int grid_x,
                              cudaStream_t st);
 cudaError_t launch_combine(const CombineArgs& a, int D, cudaStream_t st);
+// 2D bf16 tensor map [rows, D] with [128 x 64] boxes and the 128-byte swizzle (api.cu).
+int make_tmap(CUtensorMap* m, const void* base, uint64_t rows, int D);
+// Streaming multiprocessors of the current device (api.cu).
+int sm_count();
 // Launches the block-sparse attention kernel; tensor maps are built by the caller.
 cudaError_t launch_hla_fwd(const void* tmQ, const void* tmK, const void* tmV,
                            const FwdParams& p, int D, int grid, cudaStream_t st);

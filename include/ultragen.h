@@ -159,6 +159,31 @@ int ultragen_hla_forward(const void* qp, const void* kp, const void* vp, void* o
 int ultragen_unpermute(const void* op, void* o, int out_dtype, int batch,
                        const ultragen_plan_t* plan, ultragen_stream_t stream);
 
+/*
+ * ultragen_hla_forward_noalloc -- the same attention as ultragen_hla_forward, for callers that
+ * cannot allocate device memory when they call it: code running while a framework's caching
+ * allocator owns the whole device, real-time loops that must not hit cudaMalloc's implicit
+ * synchronisation, or processes held to a fixed memory budget.  The pages have no counterpart
+ * of this call; it exists for those callers only.
+ *   Arguments, layouts and results are those of ultragen_hla_forward.
+ *   It calls no cudaMalloc, cudaFree or other allocating routine.  The split partials live in
+ *   one file-scope device array of ULTRAGEN_NOALLOC_SCRATCH_BYTES that every GPU which loads
+ *   the library holds until the process exits.  No part of it needs to start at zero (each
+ *   partial the merge reads is written earlier in the same call), it keeps the last call's
+ *   contents, and all calls share it: calls that overlap on the GPU (two streams, two
+ *   threads) race on it and give wrong results.
+ *   The first call on a device looks up the array's device address (cudaGetSymbolAddress);
+ *   make that first call before any stream capture.
+ *   The plan's tables must already be on the current device: any earlier device call with
+ *   this plan (e.g. ultragen_permute_rope) uploads them; otherwise ULTRAGEN_ERR_PLAN_MISMATCH.
+ *   ULTRAGEN_ERR_UNSUPPORTED when batch * heads * workspace_bytes_per_head (see
+ *   ultragen_plan_info) exceeds ULTRAGEN_NOALLOC_SCRATCH_BYTES; a larger split chunk
+ *   (ultragen_plan_set_split) or no split (0) lowers it.
+ */
+#define ULTRAGEN_NOALLOC_SCRATCH_BYTES (64u << 20)
+int ultragen_hla_forward_noalloc(const void* qp, const void* kp, const void* vp, void* op,
+                                 const ultragen_plan_t* plan, int batch, ultragen_stream_t stream);
+
 /* Wait for `stream`, then report (and clear) a device-side error raised by this plan's
  * kernels since the last call: ULTRAGEN_ERR_TIMEOUT if a wait ran out. */
 int ultragen_sync_status(const ultragen_plan_t* plan, ultragen_stream_t stream);
