@@ -40,14 +40,17 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
   (void)state;
 }
 
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+// One bounded wait on a barrier phase: the thread sleeps until the phase completes or about
+// `suspend_ns` pass (then it returns false), instead of spinning on the issue slots that the
+// other warps of its SM sub-partition need.
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity, uint32_t suspend_ns) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(suspend_ns)
       : "memory");
   return ok != 0;
 }
@@ -61,22 +64,22 @@ enum DevErr : int {
   DEV_TIMEOUT_DRAIN = 0x104,
 };
 
-// Bounded wait: spins on the barrier phase; every 256 polls it checks the CTA abort flag and
-// the wall clock.  Returns false when the CTA is aborting or when `timeout_ns` passed (then it
-// raises the abort flag and records `code` in the global error word).
+// Bounded wait: sleeps on the barrier phase in slices of 20 us; between slices it checks the
+// CTA abort flag and the wall clock.  Returns false when the CTA is aborting or when
+// `timeout_ns` passed (then it raises the abort flag and records `code` in the global error
+// word).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           int* err, int code, uint64_t timeout_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
-  uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0) {
-      if (abort_flag && *abort_flag) return false;
-      if (globaltimer_ns() - t0 > timeout_ns) {
-        if (abort_flag) *abort_flag = 1;
-        atomicExch(err, code);
-        return false;
-      }
+  constexpr uint32_t kSliceNs = 20000;
+  if (mbar_try_wait(bar, parity, kSliceNs)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    if (mbar_try_wait(bar, parity, kSliceNs)) return true;
+    if (abort_flag && *abort_flag) return false;
+    if (globaltimer_ns() - t0 > timeout_ns) {
+      if (abort_flag) *abort_flag = 1;
+      atomicExch(err, code);
+      return false;
     }
   }
 }
