@@ -181,9 +181,11 @@ int ultragen_permute_rope(const void* q, const void* k, const void* v, int in_dt
   a.N_tot = (int)p->N_tot;
   a.N_raster = (int)p->N_raster;
   a.heads = p->heads;
+  a.div_heads = FastDiv((uint32_t)p->heads);
+  a.div_ntot = FastDiv((uint32_t)p->N_tot);
   a.pair_a0 = p->axes[0] / 2;
   a.pair_a01 = (p->axes[0] + p->axes[1]) / 2;
-  const int rows_per_block = (256 / (p->D / 8)) * 4;
+  const int rows_per_block = 256 / (p->D / 8);
   p->last_launches = 1;
   return cuda_status(launch_permute_rope(a, in_dtype, p->D, grid_for(a.rows_total, rows_per_block),
                                          reinterpret_cast<cudaStream_t>(stream)));
@@ -283,7 +285,9 @@ int ultragen_unpermute(const void* op, void* o, int out_dtype, int batch,
   a.N_tot = (int)p->N_tot;
   a.N_raster = (int)p->N_raster;
   a.heads = p->heads;
-  const int rows_per_block = (256 / (p->D / 8)) * 4;
+  a.div_heads = FastDiv((uint32_t)p->heads);
+  a.div_nraster = FastDiv((uint32_t)p->N_raster);
+  const int rows_per_block = 256 / (p->D / 8);
   p->last_launches = 1;
   return cuda_status(launch_unpermute(a, out_dtype, p->D, grid_for(a.rows_total, rows_per_block),
                                       reinterpret_cast<cudaStream_t>(stream)));

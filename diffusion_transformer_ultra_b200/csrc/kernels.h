@@ -9,6 +9,22 @@
 
 namespace ug {
 
+// Division of 0 <= n < 2^31 by a fixed divisor d >= 1 as a multiply-high and a shift (the
+// round-up method of Granlund and Montgomery, "Division by invariant integers using
+// multiplication", 1994): with s = ceil(log2 d) and m = floor(2^32 (2^s - d) / d) + 1,
+// n / d = (mulhi(n, m) + n) >> s.  The sum stays below 2^32 because n < 2^31.
+struct FastDiv {
+  uint32_t d, m, s;
+  FastDiv() : d(1), m(0), s(0) {}
+  explicit FastDiv(uint32_t div) : d(div), m(0), s(0) {
+    while ((1ull << s) < div) ++s;
+    m = (uint32_t)((((1ull << 32) * ((1ull << s) - div)) / div) + 1);
+  }
+#ifdef __CUDACC__
+  __device__ __forceinline__ uint32_t div(uint32_t n) const { return (__umulhi(n, m) + n) >> s; }
+#endif
+};
+
 struct PermuteArgs {
   const void* in[3];               // q, k, v raster [B, N_raster, heads, D]
   __nv_bfloat16* out[3];           // qp, kp, vp window-first [B, heads, N_tot, D]
@@ -17,6 +33,7 @@ struct PermuteArgs {
   const float* rope;               // [max(H,W)][D/2][2] (cos, sin)
   int64_t rows_total;              // B * heads * N_tot
   int N_tot, N_raster, heads;
+  FastDiv div_heads, div_ntot;
   int pair_a0, pair_a01;           // pairs [0,a0) axis 0, [a0,a01) axis 1, rest axis 2
 };
 
@@ -26,6 +43,7 @@ struct UnpermuteArgs {
   const int32_t* inv_perm;         // raster -> slot
   int64_t rows_total;              // B * N_raster * heads
   int N_tot, N_raster, heads;
+  FastDiv div_heads, div_nraster;
 };
 
 struct CombineArgs {
