@@ -28,7 +28,7 @@ SYMBOLS = (
     "ultragen_plan_info", "ultragen_plan_export", "ultragen_plan_export_rowmasks",
     "ultragen_plan_destroy", "ultragen_permute_rope", "ultragen_hla_forward",
     "ultragen_unpermute", "ultragen_sync_status", "ultragen_last_launch_count",
-    "ultragen_hla_forward_noalloc",
+    "ultragen_hla_forward_noalloc", "ultragen_plan_set_diagnostics",
 )
 
 
@@ -86,6 +86,7 @@ def lib() -> ctypes.CDLL:
     L.ultragen_unpermute.argtypes = [vp, vp, cint, cint, vp, vp]
     L.ultragen_sync_status.argtypes = [vp, vp]
     L.ultragen_last_launch_count.argtypes = [vp]
+    L.ultragen_plan_set_diagnostics.argtypes = [vp, cint, ctypes.c_double]
     for name in SYMBOLS:
         if name != "ultragen_status_string":
             getattr(L, name).restype = cint
@@ -138,6 +139,10 @@ class Plan:
         _check("ultragen_plan_export_rowmasks",
                lib().ultragen_plan_export_rowmasks(self._h, int(qtile), out.ctypes.data))
         return out[:n_entries]
+
+    def set_diagnostics(self, fault: int = 0, wait_limit_s: float = 2.0):
+        _check("ultragen_plan_set_diagnostics",
+               lib().ultragen_plan_set_diagnostics(self._h, int(fault), float(wait_limit_s)))
 
     def sync_status(self, stream=None) -> int:
         return lib().ultragen_sync_status(self._h, _stream_ptr(stream))

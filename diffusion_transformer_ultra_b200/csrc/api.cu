@@ -13,7 +13,6 @@
 namespace ug {
 namespace {
 
-constexpr unsigned long long kDefaultTimeoutNs = 2000ull * 1000 * 1000;   // 2 s per wait
 
 template <typename T>
 int upload(T** dst, const std::vector<T>& src) {
@@ -243,7 +242,8 @@ int ultragen_hla_forward(const void* qp, const void* kp, const void* vp, void* o
   f.l2 = p->l * p->l;
   f.n_ws_head = p->n_split_items;
   f.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)p->D));
-  f.timeout_ns = kDefaultTimeoutNs;
+  f.timeout_ns = p->wait_limit_ns;
+  f.fault = p->fault;
   const int grid = (int)std::min<int64_t>(items, sm_count());
   p->last_launches = 0;
   if (grid > 0) {
@@ -310,5 +310,13 @@ int ultragen_sync_status(const ultragen_plan_t* cplan, ultragen_stream_t stream)
 }
 
 int ultragen_last_launch_count(const ultragen_plan_t* p) { return p ? p->last_launches : -1; }
+
+int ultragen_plan_set_diagnostics(ultragen_plan_t* p, int fault, double wait_limit_s) {
+  if (!p || fault < 0 || fault > 1 || !(wait_limit_s >= 1e-3 && wait_limit_s <= 60.0))
+    return ULTRAGEN_ERR_INVALID_ARG;
+  p->fault = fault;
+  p->wait_limit_ns = (unsigned long long)(wait_limit_s * 1e9);
+  return ULTRAGEN_OK;
+}
 
 }  // extern "C"

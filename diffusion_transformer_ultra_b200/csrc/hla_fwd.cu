@@ -190,6 +190,7 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t tbase,
   using C = FwdCfg<D>;
   const uint32_t sQ = sbase + C::Q_OFF, sKV = sbase + C::KV_OFF, bar = sbase + C::BAR_OFF;
   uint32_t ld = 0, qi = 0, pc0 = 0, pc1 = 0;
+  bool withhold = p.fault == 1;   // injected fault: drop the first item's first "S ready"
   auto wait = [&](int b, uint32_t par) {
     return mbar_wait(bar + 8 * b, par, abort_flag, p.err, DEV_TIMEOUT_MMA, p.timeout_ns);
   };
@@ -208,7 +209,11 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t tbase,
       tc_fence_after();
       for (int t = 0; t < ntile; ++t) {
         issue_s<D>(tbase + 128 * t, sQ + t * C::TILE_BYTES, sKV + s * C::TILE_BYTES);
-        mma_commit(bar + 8 * (C::B_SF + t));
+        if (withhold && t == 0) {
+          withhold = false;     // nothing completes this barrier: its waiters time out
+        } else {
+          mma_commit(bar + 8 * (C::B_SF + t));
+        }
       }
       mma_commit(bar + 8 * (C::B_KVE + s));
     }

@@ -71,6 +71,7 @@ struct FwdParams {
   int n_ws_head;
   float scale_log2;                // log2(e) / sqrt(D)
   unsigned long long timeout_ns;   // limit of every device-side wait
+  int fault = 0;                   // 1: withhold one "S ready" signal (tests the timeout path)
 };
 
 cudaError_t launch_permute_rope(const PermuteArgs& a, int in_dtype, int D, int grid_x,

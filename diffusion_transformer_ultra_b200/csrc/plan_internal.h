@@ -59,6 +59,9 @@ struct ultragen_plan {
   // split policy (-1 auto, 0 off, >0 chunk) and the chunk in effect
   int split_req = -1;
   int split_chunk = 0;
+  // diagnostics: device wait limit and injected fault (ultragen_plan_set_diagnostics)
+  unsigned long long wait_limit_ns = 2000ull * 1000 * 1000;
+  int fault = 0;
 
   // host tables
   std::vector<int32_t> perm;       // slot -> raster (-1 pad)

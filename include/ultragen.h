@@ -188,6 +188,13 @@ int ultragen_hla_forward_noalloc(const void* qp, const void* kp, const void* vp,
  * kernels since the last call: ULTRAGEN_ERR_TIMEOUT if a wait ran out. */
 int ultragen_sync_status(const ultragen_plan_t* plan, ultragen_stream_t stream);
 
+/* Diagnostics (no counterpart in the pages).  wait_limit_s (1 ms .. 60 s, default 2 s) bounds
+ * every device-side wait of ultragen_hla_forward; past it the kernel stops cleanly and
+ * ultragen_sync_status reports ULTRAGEN_ERR_TIMEOUT.  fault = 1 makes the MMA warp of every
+ * CTA withhold one "S ready" signal, so a wait runs out on purpose (tests of that path);
+ * fault = 0 is normal operation.  INVALID_ARG outside these ranges. */
+int ultragen_plan_set_diagnostics(ultragen_plan_t* plan, int fault, double wait_limit_s);
+
 /* Kernel launches the last device call of this plan issued (for launch accounting). */
 int ultragen_last_launch_count(const ultragen_plan_t* plan);
 

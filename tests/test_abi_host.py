@@ -154,3 +154,13 @@ def test_split_policy(ffi):
     p.set_split(7)
     assert p.info["split_chunk"] == 7 and p.info["n_split_groups"] > 2
     assert p.info["workspace_bytes_per_head"] == p.info["n_split_items"] * 2 * 128 * 129 * 4
+
+
+def test_diagnostics_validation(ffi):
+    p = ffi.Plan(8, 8, 4, 1, 2, 3, 1, 64)
+    L = ffi.lib()
+    assert L.ultragen_plan_set_diagnostics(p.handle, 2, 1.0) == 1
+    assert L.ultragen_plan_set_diagnostics(p.handle, 0, 0.0) == 1
+    assert L.ultragen_plan_set_diagnostics(p.handle, 0, 61.0) == 1
+    assert L.ultragen_plan_set_diagnostics(p.handle, 1, 0.05) == 0
+    assert L.ultragen_plan_set_diagnostics(p.handle, 0, 2.0) == 0
