@@ -40,6 +40,8 @@ def parse():
     ap.add_argument("--workload", default="4k")
     ap.add_argument("--heads", type=int, default=0,
                     help="override the workload's head count (smaller profiling captures)")
+    ap.add_argument("--lr-radius", type=int, default=-1,
+                    help="HR->LR scope: -1 all LR tokens (default); r >= 0 the window's anchors grown by r")
     ap.add_argument("--impl", default="ultragen", choices=["ultragen", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -231,6 +233,8 @@ def main():
         import dataclasses
         wl = dataclasses.replace(wl, heads=args.heads)
     plan = ug.plan_for(wl)
+    if args.lr_radius != -1:
+        plan.set_lr_scope(args.lr_radius)
     info = plan.info
     q, k, v = ug.make_qkv(wl)
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
@@ -330,8 +334,9 @@ def main():
             "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) + smooth 2D sinusoid Q/K/V; no weights needed)",
-            "config": {"workload": wl.name, "H": wl.H, "W": wl.W, "l": wl.l, "b": wl.b,
-                       "rho": wl.rho, "text_len": wl.T, "heads": wl.heads, "head_dim": wl.D,
+            "config": {"workload": wl.name + ("" if args.lr_radius < 0 else f"-lr-region-r{args.lr_radius}"),
+                       "H": wl.H, "W": wl.W, "l": wl.l, "b": wl.b,
+                       "rho": wl.rho, "text_len": wl.T, "lr_radius": args.lr_radius, "heads": wl.heads, "head_dim": wl.D,
                        "batch": wl.batch, "N_tot": info["N_tot"], "useful_pairs_per_head": info["useful_pairs"],
                        "l2": "inputs larger than L2 (Q, K, V permuted: 3 x %.0f MB); no flush" % (elem * 2 / 1e6),
                        "parallelism": f"independent layer per rank x{world}"},

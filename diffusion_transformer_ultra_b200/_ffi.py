@@ -28,7 +28,7 @@ SYMBOLS = (
     "ultragen_plan_info", "ultragen_plan_export", "ultragen_plan_export_rowmasks",
     "ultragen_plan_destroy", "ultragen_permute_rope", "ultragen_hla_forward",
     "ultragen_unpermute", "ultragen_sync_status", "ultragen_last_launch_count",
-    "ultragen_hla_forward_noalloc", "ultragen_plan_set_diagnostics",
+    "ultragen_hla_forward_noalloc", "ultragen_plan_set_diagnostics", "ultragen_plan_set_lr_scope",
 )
 
 
@@ -44,6 +44,7 @@ class PlanInfo(ctypes.Structure):
         ("rope_axes", ctypes.c_int32 * 3), ("rope_theta", ctypes.c_double),
         ("split_chunk", ctypes.c_int32), ("n_split_groups", ctypes.c_int32),
         ("n_split_items", ctypes.c_int32), ("workspace_bytes_per_head", ctypes.c_int64),
+        ("lr_radius", ctypes.c_int32),
     ]
 
     def as_dict(self):
@@ -76,6 +77,7 @@ def lib() -> ctypes.CDLL:
     L.ultragen_plan.argtypes = [cint] * 8 + [ctypes.POINTER(vp)]
     L.ultragen_plan_set_rope.argtypes = [vp, cint, cint, cint, ctypes.c_double]
     L.ultragen_plan_set_split.argtypes = [vp, cint]
+    L.ultragen_plan_set_lr_scope.argtypes = [vp, cint]
     L.ultragen_plan_info.argtypes = [vp, ctypes.POINTER(PlanInfo)]
     L.ultragen_plan_export.argtypes = [vp, vp, vp, vp]
     L.ultragen_plan_export_rowmasks.argtypes = [vp, cint, vp]
@@ -123,6 +125,10 @@ class Plan:
 
     def set_split(self, chunk: int):
         _check("ultragen_plan_set_split", lib().ultragen_plan_set_split(self._h, int(chunk)))
+        self._refresh()
+
+    def set_lr_scope(self, radius: int):
+        _check("ultragen_plan_set_lr_scope", lib().ultragen_plan_set_lr_scope(self._h, int(radius)))
         self._refresh()
 
     def export(self):

@@ -29,6 +29,7 @@ int cdiv(int a, int b) { return (a + b - 1) / b; }
 struct ClassDesc {
   int kind;              // SEG_TEXT, SEG_HR, SEG_LR
   int r0, r1, c0, c1;    // HR halo box [r0, r1) x [c0, c1)
+  int lr0, lr1, lc0, lc1;  // scaled LR positions visible to the window (lr_radius >= 0)
 };
 
 inline bool visible(const ultragen_plan_t* p, const ClassDesc& c, int64_t s) {
@@ -39,7 +40,12 @@ inline bool visible(const ultragen_plan_t* p, const ClassDesc& c, int64_t s) {
     case SEG_LR:
       return sg == SEG_LR || sg == SEG_TEXT;
     default:
-      if (sg == SEG_TEXT || sg == SEG_LR) return true;
+      if (sg == SEG_TEXT) return true;
+      if (sg == SEG_LR) {
+        if (p->lr_radius < 0) return true;
+        const int pm = p->rho * p->ci[s], pn = p->rho * p->cj[s];
+        return pm >= c.lr0 && pm < c.lr1 && pn >= c.lc0 && pn < c.lc1;
+      }
       if (sg != SEG_HR) return false;
       return p->ci[s] >= c.r0 && p->ci[s] < c.r1 && p->cj[s] >= c.c0 && p->cj[s] < c.c1;
   }
@@ -53,6 +59,11 @@ ClassDesc window_class(const ultragen_plan_t* p, int wid) {
   c.r1 = std::min(p->H, (wr + 1) * p->l + p->b);
   c.c0 = std::max(0, wc * p->l - p->b);
   c.c1 = std::min(p->W, (wc + 1) * p->l + p->b);
+  // the "corresponding" LR region: the window's l x l box grown by lr_radius
+  c.lr0 = wr * p->l - p->lr_radius;
+  c.lr1 = (wr + 1) * p->l + p->lr_radius;
+  c.lc0 = wc * p->l - p->lr_radius;
+  c.lc1 = (wc + 1) * p->l + p->lr_radius;
   return c;
 }
 
@@ -149,7 +160,7 @@ int build_tables(ultragen_plan_t* p) {
       const int wlast = (int)((std::min<int64_t>(s0 + kTile, hr_end) - 1 - p->off_hr) / l2);
       for (int wid = wfirst; wid <= wlast; ++wid) classes.push_back(window_class(p, wid));
     } else {
-      ClassDesc c{kind, 0, 0, 0, 0};
+      ClassDesc c{kind, 0, 0, 0, 0, 0, 0, 0, 0};
       classes.push_back(c);
       if (kind == SEG_HR) wfirst = -1;   // pad-only tile between HR and LR segments
     }
@@ -175,7 +186,21 @@ int build_tables(ultragen_plan_t* p) {
     cand.clear();
     add_range(cand, 0, p->T);
     if (kind == SEG_TEXT) add_range(cand, p->off_hr, hr_end);
-    if (kind == SEG_HR || kind == SEG_LR) add_range(cand, p->off_lr, p->off_lr + p->N_lr);
+    if (kind == SEG_LR || (kind == SEG_HR && p->lr_radius < 0))
+      add_range(cand, p->off_lr, p->off_lr + p->N_lr);
+    if (kind == SEG_HR && p->lr_radius >= 0 && p->rho > 0) {
+      for (int c = 0; c < C; ++c) {
+        if (class_real[c] == 0) continue;
+        const ClassDesc& cd = classes[c];
+        // LR rows m with lr0 <= rho*m < lr1, columns n with lc0 <= rho*n < lc1
+        const int m0 = std::max(0, cd.lr0 > 0 ? cdiv(cd.lr0, p->rho) : 0);
+        const int m1 = std::min(p->h - 1, (cd.lr1 - 1) / p->rho);
+        const int n0 = std::max(0, cd.lc0 > 0 ? cdiv(cd.lc0, p->rho) : 0);
+        const int n1 = std::min(p->w - 1, (cd.lc1 - 1) / p->rho);
+        for (int m = m0; m <= m1 && n0 <= n1; ++m)
+          add_range(cand, p->off_lr + (int64_t)m * p->w + n0, p->off_lr + (int64_t)m * p->w + n1 + 1);
+      }
+    }
     if (kind == SEG_HR) {
       for (int c = 0; c < C; ++c) {
         if (class_real[c] == 0) continue;
@@ -410,6 +435,25 @@ int ultragen_plan_set_split(ultragen_plan_t* p, int chunk) {
   return ULTRAGEN_OK;
 }
 
+int ultragen_plan_set_lr_scope(ultragen_plan_t* p, int radius) {
+  if (!p || radius < -1 || radius > (1 << 20)) return ULTRAGEN_ERR_INVALID_ARG;
+  const int old = p->lr_radius;
+  p->lr_radius = radius;
+  int st;
+  try {
+    st = ug::build_tables(p);
+  } catch (const std::bad_alloc&) {
+    st = ULTRAGEN_ERR_OOM;
+  }
+  if (st != ULTRAGEN_OK) {
+    p->lr_radius = old;
+    ug::build_tables(p);
+    return st;
+  }
+  p->dirty = true;
+  return ULTRAGEN_OK;
+}
+
 int ultragen_plan_info(const ultragen_plan_t* p, ultragen_plan_info_t* o) {
   if (!p || !o) return ULTRAGEN_ERR_INVALID_ARG;
   std::memset(o, 0, sizeof(*o));
@@ -429,6 +473,7 @@ int ultragen_plan_info(const ultragen_plan_t* p, ultragen_plan_info_t* o) {
   o->n_split_groups = (int32_t)p->combine.size();
   o->n_split_items = p->n_split_items;
   o->workspace_bytes_per_head = (int64_t)p->n_split_items * 2 * ug::kTile * (p->D + 1) * 4;
+  o->lr_radius = p->lr_radius;
   return ULTRAGEN_OK;
 }
 

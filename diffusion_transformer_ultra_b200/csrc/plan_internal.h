@@ -59,6 +59,8 @@ struct ultragen_plan {
   // split policy (-1 auto, 0 off, >0 chunk) and the chunk in effect
   int split_req = -1;
   int split_chunk = 0;
+  // HR -> LR scope: -1 all LR tokens; r >= 0 the anchors within r of the query's window
+  int lr_radius = -1;
   // diagnostics: device wait limit and injected fault (ultragen_plan_set_diagnostics)
   unsigned long long wait_limit_ns = 2000ull * 1000 * 1000;
   int fault = 0;

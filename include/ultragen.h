@@ -72,6 +72,7 @@ typedef struct {
   int32_t n_split_groups;     /* query groups whose key list is split                   */
   int32_t n_split_items;      /* items that write split partials (per head)             */
   int64_t workspace_bytes_per_head; /* split partial storage per (batch, head)          */
+  int32_t lr_radius;          /* HR -> LR scope (ultragen_plan_set_lr_scope)            */
 } ultragen_plan_info_t;
 
 /* Human-readable name of a status code.  Never NULL. */
@@ -105,6 +106,14 @@ int ultragen_plan_set_rope(ultragen_plan_t* plan, int ax0, int ax1, int ax2, dou
  * log-sum-exp combine.  chunk = -1: automatic (the default; chunk = the longest HR/LR
  * group, applied to groups at least 1.5x longer); chunk = 0: never split. */
 int ultragen_plan_set_split(ultragen_plan_t* plan, int chunk);
+
+/* Scope of the LR tokens an HR query sees.  radius = -1 (default): all LR tokens, the
+ * reading of [UG-gist] 2.B ("the scaled global guidance tokens").  radius = r >= 0: the
+ * "corresponding" anchors of [UG-note] 关键设计 2 (and the German summary's "entsprechenden
+ * skalierten Regionen"): LR token (m, n) is visible to the HR queries of window (wr, wc) iff
+ * (rho m, rho n) lies in [wr l - r, (wr+1) l + r) x [wc l - r, (wc+1) l + r).  Rebuilds the
+ * tile lists; rope and split settings are kept.  INVALID_ARG for radius < -1. */
+int ultragen_plan_set_lr_scope(ultragen_plan_t* plan, int radius);
 
 int ultragen_plan_info(const ultragen_plan_t* plan, ultragen_plan_info_t* out);
 

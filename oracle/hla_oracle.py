@@ -31,7 +31,11 @@ Readings taken where the pages are silent or garbled (each is listed in DESIGN.m
   R1  l counts latent tokens (l=16 <-> 256x256 pixels at a 16x VAE).
   R2  Halo: the query's own window box grown by b tokens on every side, clipped to the
       image; every query of a window sees the same set.  0 <= b <= l.
-  R3  HR queries see ALL low-resolution tokens.
+  R3  HR queries see ALL low-resolution tokens (lr_radius = -1, the default).  The variant
+      lr_radius = r >= 0 follows the other reading of the pages (the "corresponding" LR
+      anchors, [UG-note] 关键设计 2 and the German summary's "entsprechenden skalierten
+      Regionen"): an HR query of window (wr, wc) sees LR token (m, n) iff its scaled position
+      (rho m, rho n) lies in the window's l x l box grown by r tokens on every side.
   R4  LR queries see LR and text.  R5 text queries see text and HR, not LR.
   R6  The "* M" inside the softmax is read as an additive -inf on masked pairs; the
       scale is 1/sqrt(head_dim).
@@ -80,6 +84,7 @@ class Geometry:
     b: int          # halo width in tokens (R2)
     rho: int        # LR down-scale factor, rho = H / h ([UG-note] 关键设计 2); 0 = no LR
     T: int          # text tokens
+    lr_radius: int = -1   # -1: HR sees all LR (R3); r >= 0: only the window's region grown by r
 
     @property
     def nWh(self) -> int:
@@ -297,11 +302,23 @@ def visible_rows(g: Geometry, q_slots: np.ndarray) -> np.ndarray:
 
     hr = np.nonzero(qs == HR)[0]
     if len(hr):
-        r0, r1, c0, c1 = window_box(g, ca[q_slots[hr]], cb[q_slots[hr]])
+        qi, qj = ca[q_slots[hr]], cb[q_slots[hr]]
+        r0, r1, c0, c1 = window_box(g, qi, qj)
         ki, kj = ca[None, :], cb[None, :]
         in_box = ((kseg == HR) & (ki >= r0[:, None]) & (ki < r1[:, None])
                   & (kj >= c0[:, None]) & (kj < c1[:, None]))
-        vis[hr] = in_box | (kseg == TEXT) | (kseg == LR)
+        if g.lr_radius < 0:
+            lr_vis = kseg == LR
+        else:
+            # LR anchors whose scaled position lies in the window grown by lr_radius
+            rr0 = (qi // g.l) * g.l - g.lr_radius
+            rr1 = (qi // g.l + 1) * g.l + g.lr_radius
+            cc0 = (qj // g.l) * g.l - g.lr_radius
+            cc1 = (qj // g.l + 1) * g.l + g.lr_radius
+            pm, pn = g.rho * ki, g.rho * kj
+            lr_vis = ((kseg == LR) & (pm >= rr0[:, None]) & (pm < rr1[:, None])
+                      & (pn >= cc0[:, None]) & (pn < cc1[:, None]))
+        vis[hr] = in_box | (kseg == TEXT) | lr_vis
     return vis
 
 

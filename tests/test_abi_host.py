@@ -164,3 +164,37 @@ def test_diagnostics_validation(ffi):
     assert L.ultragen_plan_set_diagnostics(p.handle, 0, 61.0) == 1
     assert L.ultragen_plan_set_diagnostics(p.handle, 1, 0.05) == 0
     assert L.ultragen_plan_set_diagnostics(p.handle, 0, 2.0) == 0
+
+
+def compare_region_plan(ffi, geom, r, qtiles=None):
+    g = O.Geometry(*geom, lr_radius=r)
+    p = ffi.Plan(*geom, 2, 64)
+    p.set_lr_scope(r)
+    assert p.info["lr_radius"] == r
+    perm, row_ptr, entries = p.export()
+    np.testing.assert_array_equal(perm, O.perm_map(g))
+    for t in (range(g.N_tot // 128) if qtiles is None else qtiles):
+        e_ref, m_ref = O.qtile_entries(g, t)
+        np.testing.assert_array_equal(entries[row_ptr[t]:row_ptr[t + 1]].view(np.uint32), e_ref,
+                                      err_msg=f"q-tile {t}")
+        np.testing.assert_array_equal(p.rowmasks(t, len(e_ref)), m_ref, err_msg=f"q-tile {t} masks")
+    return g, p
+
+
+@pytest.mark.parametrize("name,r", [("tiny", 0), ("1k", 4), ("odd", 3), ("small_l", 1)])
+def test_region_plan_bit_exact(ffi, name, r):
+    g, p = compare_region_plan(ffi, GEOMS[name], r)
+    assert p.info["useful_pairs"] == O.visible_pair_count(g)
+
+
+def test_region_plan_large_sampled(ffi):
+    import sys
+    sys.path.insert(0, os.path.dirname(__file__))
+    from test_oracle_pins import closed_form_pairs
+    for geom, r in (((256, 256, 16, 4, 4, 512), 4), ((512, 512, 16, 4, 4, 512), 0),
+                    ((256, 135, 16, 16, 4, 256), 16)):
+        g = O.Geometry(*geom, lr_radius=r)
+        _, p = compare_region_plan(ffi, geom, r, sample_qtiles(g, n_hr=10))
+        assert p.info["useful_pairs"] == sum(closed_form_pairs(*geom, lr_radius=r).values())
+    p = ffi.Plan(64, 64, 16, 4, 4, 512, 2, 64)
+    assert ffi.lib().ultragen_plan_set_lr_scope(p.handle, -2) == 1

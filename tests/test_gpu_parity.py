@@ -29,9 +29,11 @@ def _wl(name, **kw):
     return dataclasses.replace(WORKLOADS[name], **kw) if kw else WORKLOADS[name]
 
 
-def run_layer(ug, wl, split=None, poison=True):
+def run_layer(ug, wl, split=None, poison=True, lr_radius=-1):
     import torch
     plan = ug.plan_for(wl)
+    if lr_radius != -1:
+        plan.set_lr_scope(lr_radius)
     if split is not None:
         plan.set_split(split)
     q, k, v = ug.make_qkv(wl)
@@ -177,6 +179,24 @@ def test_attention_full_size_sampled(ug, name, heads):
         got = np.stack([to_np64(lay.op[b, h, torch.as_tensor(rows, device="cuda")]) for h in heads])
         assert np.all(got[:, ~real] == 0)
         check_attention(got[:, real], ref[:, real], f"{name} b={b}")
+
+
+@pytest.mark.parametrize("name,r,heads", [("1k", 4, (0, 11, 23)), ("tiny", 0, (0,)),
+                                          ("4k", 4, (9,)), ("8k", 0, (2,))])
+def test_attention_lr_region_parity(ug, name, r, heads):
+    """The LR-region reading (HR queries see only the anchors of their window, grown by r)."""
+    import torch
+    wl = _wl(name)
+    plan, (q, k, v), lay, o = run_layer(ug, wl, lr_radius=r)
+    assert plan.info["lr_radius"] == r
+    assert not torch.isnan(lay.op).any()
+    g = geometry(wl, r)
+    rows = np.arange(g.N_tot) if name in ("1k", "tiny") else sample_rows(wl)
+    real = O.perm_map(g)[rows] >= 0
+    ref = oracle_rows(q, k, v, wl, 0, heads, rows, lr_radius=r)
+    got = np.stack([to_np64(lay.op[0, h, torch.as_tensor(rows, device="cuda")]) for h in heads])
+    assert np.all(got[:, ~real] == 0)
+    check_attention(got[:, real], ref[:, real], f"{name} lr_radius={r}")
 
 
 def test_deterministic(ug):

@@ -61,7 +61,7 @@ def bf_slots(H, W, l, rho, T):
     return seq
 
 
-def bf_visible(qt, kt, l, b):
+def bf_visible(qt, kt, l, b, rho=0, lr_radius=-1):
     """Visibility of key token kt to query token qt (None = pad)."""
     if qt is None or kt is None:
         return False
@@ -70,12 +70,19 @@ def bf_visible(qt, kt, l, b):
         return kk in ("text", "hr")
     if qk == "lr":
         return kk in ("lr", "text")
-    # HR query: text, all LR, and HR keys within b of its window rectangle
-    if kk in ("text", "lr"):
-        return True
+    # HR query: text, LR (all, or the anchors within lr_radius of its window), and HR keys
+    # within b of its window rectangle
     wr, wc = qt[1] // l, qt[2] // l
     top, bottom = wr * l, (wr + 1) * l - 1
     left, right = wc * l, (wc + 1) * l - 1
+    if kk == "text":
+        return True
+    if kk == "lr":
+        if lr_radius < 0:
+            return True
+        ym, xn = rho * kt[1], rho * kt[2]
+        return (max(0, top - ym, ym - bottom) <= lr_radius and
+                max(0, left - xn, xn - right) <= lr_radius)
     dr = max(0, top - kt[1], kt[1] - bottom)
     dc = max(0, left - kt[2], kt[2] - right)
     return dr <= b and dc <= b
@@ -105,7 +112,7 @@ def bf_rope_vec(x, pos, axes, theta=1e4):
     return y
 
 
-def bf_forward(q, k, v, H, W, l, b, rho, T, axes):
+def bf_forward(q, k, v, H, W, l, b, rho, T, axes, lr_radius=-1):
     """Pure-Python HLA on raster inputs [B, N, Hh, D]; returns raster output."""
     toks = bf_tokens(H, W, rho, T)
     B, N, Hh, D = q.shape
@@ -116,7 +123,7 @@ def bf_forward(q, k, v, H, W, l, b, rho, T, axes):
         for t, tok in enumerate(toks):
             logits = []
             for u, utok in enumerate(toks):
-                if bf_visible(tok, utok, l, b):
+                if bf_visible(tok, utok, l, b, rho, lr_radius):
                     logits.append((u, sum(a * c for a, c in zip(qr[t], kr[u])) / math.sqrt(D)))
             mx = max(s for _, s in logits)
             wts = [(u, math.exp(s - mx)) for u, s in logits]
@@ -337,7 +344,7 @@ def test_rope_invariants():
 # pair counts: closed forms and the pages' numbers
 # ----------------------------------------------------------------------------------------
 
-def closed_form_pairs(H, W, l, b, rho, T):
+def closed_form_pairs(H, W, l, b, rho, T, lr_radius=-1):
     """Visible pairs of one head, segment by segment, from closed forms."""
     h = math.ceil(H / rho) if rho else 0
     w = math.ceil(W / rho) if rho else 0
@@ -351,9 +358,20 @@ def closed_form_pairs(H, W, l, b, rho, T):
             s += rows_in * box
         return s
 
+    def axis_lr(n, nl):
+        # sum over windows of (HR rows in the window) x (LR anchors rho*m in its grown range)
+        s = 0
+        for wi in range(math.ceil(n / l)):
+            rows_in = min(n, (wi + 1) * l) - wi * l
+            anchors = sum(1 for m in range(nl) if wi * l - lr_radius <= rho * m < (wi + 1) * l + lr_radius)
+            s += rows_in * anchors
+        return s
+
+    hr_lr = Nhr * Nlr if lr_radius < 0 else axis_lr(H, h) * axis_lr(W, w)
+
     return {
         "hr_hr": axis_sum(H) * axis_sum(W),
-        "hr_text": Nhr * T, "hr_lr": Nhr * Nlr,
+        "hr_text": Nhr * T, "hr_lr": hr_lr,
         "text_text": T * T, "text_hr": T * Nhr,
         "lr_lr": Nlr * Nlr, "lr_text": Nlr * T,
     }
@@ -417,3 +435,49 @@ def test_round_bf16_ties_and_no_double_rounding():
     # if the extra bit were below fp32 precision; here 2^-30 is kept by fp64)
     assert O.round_bf16(np.array([1.0 + 2.0 ** -8 + 2.0 ** -30]))[0] == 1.0 + 2.0 ** -7
     assert O.round_bf16(np.array([1.0 + 2.0 ** -8 + 2.0 ** -40]))[0] == 1.0 + 2.0 ** -7
+
+
+# ----------------------------------------------------------------------------------------
+# the LR-region reading (lr_radius >= 0)
+# ----------------------------------------------------------------------------------------
+
+REGION_GEOMS = [
+    # H, W, l, b, rho, T, axes, lr_radius
+    (8, 8, 4, 1, 2, 3, (4, 6, 6), 0),
+    (7, 10, 4, 2, 3, 5, (2, 4, 4), 2),
+    (12, 9, 4, 0, 4, 2, (2, 2, 4), 5),
+]
+
+
+@pytest.mark.parametrize("geom", REGION_GEOMS)
+def test_region_mask_matches_brute_force(geom):
+    H, W, l, b, rho, T, _, r = geom
+    g = O.Geometry(H, W, l, b, rho, T, r)
+    seq = bf_slots(H, W, l, rho, T)
+    expect = np.array([[bf_visible(qt, kt, l, b, rho, r) for kt in seq] for qt in seq])
+    np.testing.assert_array_equal(O.visible_rows(g, np.arange(g.N_tot)), expect)
+
+
+@pytest.mark.parametrize("geom", REGION_GEOMS[:2])
+def test_region_forward_matches_brute_force(geom):
+    H, W, l, b, rho, T, axes, r = geom
+    g = O.Geometry(H, W, l, b, rho, T, r)
+    rng = np.random.default_rng(11)
+    q, k, v = (rng.standard_normal((1, g.N_raster, 2, sum(axes))) for _ in range(3))
+    expect = bf_forward(q, k, v, H, W, l, b, rho, T, axes, lr_radius=r)
+    got = O.unpermute(O.forward(q, k, v, g, axes)[0], g)
+    np.testing.assert_allclose(got, expect, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("geom", [(32, 32, 8, 2, 4, 16, 0), (64, 64, 16, 4, 4, 512, 4),
+                                  (40, 27, 16, 16, 4, 64, 16), (19, 23, 8, 3, 3, 9, 1)])
+def test_region_pair_count_equals_closed_form(geom):
+    g = O.Geometry(*geom)
+    assert O.visible_pair_count(g) == sum(closed_form_pairs(*geom).values())
+
+
+def test_region_radius_covering_the_image_is_all_lr():
+    base = O.Geometry(20, 24, 8, 2, 4, 7)
+    wide = O.Geometry(20, 24, 8, 2, 4, 7, 64)
+    rows = np.arange(base.N_tot)
+    np.testing.assert_array_equal(O.visible_rows(base, rows), O.visible_rows(wide, rows))
