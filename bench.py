@@ -1,4 +1,5 @@
-"""Benchmark of the HLA hot path: permute_rope -> hla_forward (+ split combine) -> unpermute.
+"""Benchmark of the HLA hot path: permute_rope -> hla_forward (+ split combine) -> unpermute
+(folded into the attention epilogue unless --unfused).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 4k|8k|1k|ragged]
                     [--impl ultragen|reference]
@@ -43,6 +44,8 @@ def parse():
     ap.add_argument("--lr-radius", type=int, default=-1,
                     help="HR->LR scope: -1 all LR tokens (default); r >= 0 the window's anchors grown by r")
     ap.add_argument("--impl", default="ultragen", choices=["ultragen", "reference"])
+    ap.add_argument("--unfused", action="store_true",
+                    help="run unpermute as its own pass instead of in the attention epilogue")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -249,12 +252,16 @@ def main():
         n = 1
         if evs:
             evs[1].record(stream)
-        ug.hla_forward(lay.qp, lay.kp, lay.vp, lay.op, plan)
+        if args.unfused:
+            ug.hla_forward(lay.qp, lay.kp, lay.vp, lay.op, plan)
+        else:
+            ug.hla_forward_raster(lay.qp, lay.kp, lay.vp, o, plan)   # unpermute in the epilogue
         n += plan.last_launch_count()
         if evs:
             evs[2].record(stream)
-        ug.unpermute(lay.op, o, plan)
-        n += 1
+        if args.unfused:
+            ug.unpermute(lay.op, o, plan)
+            n += 1
         if evs:
             evs[3].record(stream)
         return n
@@ -340,10 +347,13 @@ def main():
                        "batch": wl.batch, "N_tot": info["N_tot"], "useful_pairs_per_head": info["useful_pairs"],
                        "l2": "inputs larger than L2 (Q, K, V permuted: 3 x %.0f MB); no flush" % (elem * 2 / 1e6),
                        "parallelism": f"independent layer per rank x{world}"},
-            "ms_per_kernel": {"permute_rope": ms_perm, "hla_forward": ms_attn, "unpermute": ms_unperm},
+            "ms_per_kernel": {"permute_rope": ms_perm, "hla_forward": ms_attn,
+                              "unpermute": ms_unperm if args.unfused else "in hla_forward's epilogue"},
+            "path": "permute_rope + hla_forward + unpermute" if args.unfused
+                    else "permute_rope + hla_forward_raster (unpermute fused)",
             "hla_forward_tflops": attn_tflops,
             "permute_rope_gbs": perm_bytes / (ms_perm * 1e-3) / 1e9,
-            "unpermute_gbs": unperm_bytes / (ms_unperm * 1e-3) / 1e9,
+            "unpermute_gbs": unperm_bytes / (ms_unperm * 1e-3) / 1e9 if args.unfused else None,
             "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
                          "frac": attn_tflops / peak, "traffic": traffic,
                          "peak_source": f"{src} bf16 dense, sustained (kernel timed inside a repeated step)",

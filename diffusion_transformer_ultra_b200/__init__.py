@@ -5,7 +5,8 @@ The compute lives in ``libultragen.so`` (hand-written CUDA behind a C ABI, see
 the seeded synthetic-input generator.
 """
 from ._ffi import (BF16, F32, Layer, Plan, UltragenError, hla_forward,  # noqa: F401
-                   hla_forward_noalloc, lib, permute_rope, unpermute)
+                   hla_forward_noalloc, hla_forward_raster, lib, permute_rope,
+                   unpermute)
 from .inputs import WORKLOADS, Workload, make_qkv  # noqa: F401
 
 

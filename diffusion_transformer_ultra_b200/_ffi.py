@@ -29,6 +29,7 @@ SYMBOLS = (
     "ultragen_plan_destroy", "ultragen_permute_rope", "ultragen_hla_forward",
     "ultragen_unpermute", "ultragen_sync_status", "ultragen_last_launch_count",
     "ultragen_hla_forward_noalloc", "ultragen_plan_set_diagnostics", "ultragen_plan_set_lr_scope",
+    "ultragen_hla_forward_raster",
 )
 
 
@@ -85,6 +86,7 @@ def lib() -> ctypes.CDLL:
     L.ultragen_permute_rope.argtypes = [vp, vp, vp, cint, vp, vp, vp, cint, vp, vp]
     L.ultragen_hla_forward.argtypes = [vp, vp, vp, vp, vp, cint, vp]
     L.ultragen_hla_forward_noalloc.argtypes = [vp, vp, vp, vp, vp, cint, vp]
+    L.ultragen_hla_forward_raster.argtypes = [vp, vp, vp, vp, vp, cint, vp]
     L.ultragen_unpermute.argtypes = [vp, vp, cint, cint, vp, vp]
     L.ultragen_sync_status.argtypes = [vp, vp]
     L.ultragen_last_launch_count.argtypes = [vp]
@@ -219,6 +221,20 @@ def hla_forward(qp, kp, vp, op, plan: Plan, stream=None):
         _stream_ptr(stream)))
 
 
+def hla_forward_raster(qp, kp, vp, o, plan: Plan, stream=None):
+    """hla_forward writing O straight to the raster layout [B, N_raster, H, D] (bf16)."""
+    import torch
+    i = plan.info
+    B = qp.shape[0]
+    shape = (B, i["heads"], i["N_tot"], i["head_dim"])
+    for t, n in ((qp, "qp"), (kp, "kp"), (vp, "vp")):
+        _need(t, shape, (torch.bfloat16,), n)
+    _need(o, (B, i["N_raster"], i["heads"], i["head_dim"]), (torch.bfloat16,), "o")
+    _check("ultragen_hla_forward_raster", lib().ultragen_hla_forward_raster(
+        qp.data_ptr(), kp.data_ptr(), vp.data_ptr(), o.data_ptr(), plan.handle, B,
+        _stream_ptr(stream)))
+
+
 def hla_forward_noalloc(qp, kp, vp, op, plan: Plan, stream=None):
     """hla_forward without any device allocation: split partials go to the library's fixed
     scratch array.  The plan's tables must already be on the device (any earlier device call
@@ -258,8 +274,17 @@ class Layer:
         self.qp, self.kp, self.vp, self.op = (torch.empty(shape, dtype=torch.bfloat16, device=device)
                                               for _ in range(4))
 
-    def __call__(self, q, k, v, o, stream=None):
+    def __call__(self, q, k, v, o, stream=None, fused=None):
+        """o: raster [B, N_raster, H, D].  With a bf16 o the unpermute runs inside the
+        attention epilogue (fused=None or True); fused=False, or an fp32 o, keeps the three
+        separate passes (the permuted output stays in self.op)."""
+        import torch
         permute_rope(q, k, v, self.qp, self.kp, self.vp, self.plan, stream)
-        hla_forward(self.qp, self.kp, self.vp, self.op, self.plan, stream)
-        unpermute(self.op, o, self.plan, stream)
+        if fused is None:
+            fused = o.dtype == torch.bfloat16
+        if fused:
+            hla_forward_raster(self.qp, self.kp, self.vp, o, self.plan, stream)
+        else:
+            hla_forward(self.qp, self.kp, self.vp, self.op, self.plan, stream)
+            unpermute(self.op, o, self.plan, stream)
         return o

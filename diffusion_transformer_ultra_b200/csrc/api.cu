@@ -190,8 +190,10 @@ int ultragen_permute_rope(const void* q, const void* k, const void* v, int in_dt
                                          reinterpret_cast<cudaStream_t>(stream)));
 }
 
-int ultragen_hla_forward(const void* qp, const void* kp, const void* vp, void* op,
-                         const ultragen_plan_t* cplan, int batch, ultragen_stream_t stream) {
+// The attention forward; `raster` selects the output layout (0: permuted, 1: raster).
+static int hla_forward_impl(const void* qp, const void* kp, const void* vp, void* op,
+                            const ultragen_plan_t* cplan, int batch, ultragen_stream_t stream,
+                            int raster) {
   ultragen_plan_t* p = const_cast<ultragen_plan_t*>(cplan);
   if (!p || !qp || !kp || !vp || !op || batch < 1) return ULTRAGEN_ERR_INVALID_ARG;
   const void* ptrs[] = {qp, kp, vp, op};
@@ -244,6 +246,9 @@ int ultragen_hla_forward(const void* qp, const void* kp, const void* vp, void* o
   f.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)p->D));
   f.timeout_ns = p->wait_limit_ns;
   f.fault = p->fault;
+  f.raster = raster;
+  f.N_raster = (int)p->N_raster;
+  f.heads = p->heads;
   const int grid = (int)std::min<int64_t>(items, sm_count());
   p->last_launches = 0;
   if (grid > 0) {
@@ -261,11 +266,26 @@ int ultragen_hla_forward(const void* qp, const void* kp, const void* vp, void* o
     c.n_ws_head = p->n_split_items;
     c.N_tot = (int)p->N_tot;
     c.BH = batch * p->heads;
+    c.raster = raster;
+    c.N_raster = (int)p->N_raster;
+    c.heads = p->heads;
     st = cuda_status(launch_combine(c, p->D, s));
     if (st) return st;
     p->last_launches++;
   }
   return ULTRAGEN_OK;
+}
+
+int ultragen_hla_forward(const void* qp, const void* kp, const void* vp, void* op,
+                         const ultragen_plan_t* plan, int batch, ultragen_stream_t stream) {
+  return hla_forward_impl(qp, kp, vp, op, plan, batch, stream, 0);
+}
+
+int ultragen_hla_forward_raster(const void* qp, const void* kp, const void* vp, void* o,
+                                const ultragen_plan_t* plan, int batch, ultragen_stream_t stream) {
+  if (plan && (int64_t)batch * plan->heads * plan->N_raster >= ((int64_t)1 << 31))
+    return ULTRAGEN_ERR_UNSUPPORTED;
+  return hla_forward_impl(qp, kp, vp, o, plan, batch, stream, 1);
 }
 
 int ultragen_unpermute(const void* op, void* o, int out_dtype, int batch,

@@ -291,8 +291,17 @@ __device__ void softmax_role(const FwdParams& p, uint32_t sbase, uint32_t tbase,
       cls = (slot - p.off_hr) / p.l2 - wfirst;
       cls = cls < 0 ? 0 : (cls > ncls - 1 ? ncls - 1 : cls);
     }
-    __nv_bfloat16* orow = p.out + ((size_t)bh * p.N_tot + slot) * D;
+    // output row: permuted [bh][slot], or raster [b][token][h] (pad rows have no raster row)
+    __nv_bfloat16* orow;
+    if (p.raster) {
+      const int tok = __ldg(p.perm + slot);
+      const int b = bh / p.heads, hh = bh - (bh / p.heads) * p.heads;
+      orow = tok >= 0 ? p.out + (((size_t)b * p.N_raster + tok) * p.heads + hh) * D : nullptr;
+    } else {
+      orow = p.out + ((size_t)bh * p.N_tot + slot) * D;
+    }
     if (n == 0) {
+      if (!orow) continue;
 #pragma unroll
       for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(orow)[c] = make_uint4(0, 0, 0, 0);
       continue;
@@ -390,20 +399,24 @@ __device__ void softmax_role(const FwdParams& p, uint32_t sbase, uint32_t tbase,
     __syncwarp();
     const float inv = (lsum > 0.f) ? 1.0f / lsum : 0.f;
     if (ws_slot < 0) {
+      // every lane loads (tcgen05.ld is warp-wide); rows without a raster row store nothing
       const float f = real ? inv : 0.f;
 #pragma unroll
       for (int ch = 0; ch < D / 32; ++ch) {
         uint32_t o[32];
+        __syncwarp();
         tmem_ld32_sync(tO + ch * 32, o);
-        uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+        if (orow) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint4 v;
-          v.x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * f, __uint_as_float(o[8 * q + 1]) * f);
-          v.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * f, __uint_as_float(o[8 * q + 3]) * f);
-          v.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * f, __uint_as_float(o[8 * q + 5]) * f);
-          v.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * f, __uint_as_float(o[8 * q + 7]) * f);
-          dst[q] = v;
+          for (int q = 0; q < 4; ++q) {
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * f, __uint_as_float(o[8 * q + 1]) * f);
+            v.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * f, __uint_as_float(o[8 * q + 3]) * f);
+            v.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * f, __uint_as_float(o[8 * q + 5]) * f);
+            v.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * f, __uint_as_float(o[8 * q + 7]) * f);
+            dst[q] = v;
+          }
         }
       }
     } else {

@@ -52,6 +52,8 @@ struct CombineArgs {
   const int32_t* groups;           // 4 ints per split group: qt0, qt1, ws_first, nsplit
   const int32_t* perm;
   int n_groups, n_ws_head, N_tot, BH;
+  int raster = 0;                  // 1: out is raster [B, N_raster, heads, D] (pad rows skipped)
+  int N_raster = 0, heads = 1;
 };
 
 struct FwdParams {
@@ -72,6 +74,8 @@ struct FwdParams {
   float scale_log2;                // log2(e) / sqrt(D)
   unsigned long long timeout_ns;   // limit of every device-side wait
   int fault = 0;                   // 1: withhold one "S ready" signal (tests the timeout path)
+  int raster = 0;                  // 1: out is raster [B, N_raster, heads, D] (pad rows skipped)
+  int N_raster = 0, heads = 1;
 };
 
 cudaError_t launch_permute_rope(const PermuteArgs& a, int in_dtype, int D, int grid_x,

@@ -181,14 +181,18 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
   const int qt = t ? G[1] : G[0];
   if (qt < 0) return;
   const int slot = qt * 128 + row;
-  __nv_bfloat16* dst = a.out + (bh * a.N_tot + slot) * D + lane * PER;
+  const int tok = __ldg(a.perm + slot);
+  if (a.raster && tok < 0) return;                 // pad rows have no raster row
+  __nv_bfloat16* dst =
+      a.raster ? a.out + (((bh / a.heads) * a.N_raster + tok) * a.heads + bh % a.heads) * D + lane * PER
+               : a.out + (bh * a.N_tot + slot) * D + lane * PER;
   const size_t item_floats = (size_t)2 * 128 * (D + 1);
   const float* base = a.ws + (size_t)(bh * a.n_ws_head) * item_floats;
   float acc[PER];
 #pragma unroll
   for (int i = 0; i < PER; ++i) acc[i] = 0.f;
   float M = -INFINITY;
-  if (__ldg(a.perm + slot) >= 0) {
+  if (tok >= 0) {
     for (int s = 0; s < G[3]; ++s) {
       const float* it = base + (size_t)(G[2] + s) * item_floats;
       M = fmaxf(M, __ldg(it + 2 * 128 * D + t * 128 + row));

@@ -161,6 +161,17 @@ int ultragen_hla_forward(const void* qp, const void* kp, const void* vp, void* o
                          const ultragen_plan_t* plan, int batch, ultragen_stream_t stream);
 
 /*
+ * ultragen_hla_forward_raster -- ultragen_hla_forward with the unpermute folded into its
+ * epilogue: each output row goes straight to its raster place.
+ *   qp, kp, vp  [batch, heads, N_tot, head_dim] BF16 (device, permuted)
+ *   o           [batch, N_raster, heads, head_dim] BF16 (device, raster); pad slots write nothing
+ * Same arithmetic as ultragen_hla_forward + ultragen_unpermute (bit for bit), one pass less
+ * over HBM.  Errors as ultragen_hla_forward.
+ */
+int ultragen_hla_forward_raster(const void* qp, const void* kp, const void* vp, void* o,
+                                const ultragen_plan_t* plan, int batch, ultragen_stream_t stream);
+
+/*
  * ultragen_unpermute -- window-first -> raster: o[b, t, h, :] = op[b, h, slot(t), :].
  *   op  [batch, heads, N_tot, head_dim] BF16 (device)
  *   o   [batch, N_raster, heads, head_dim], out_dtype BF16 (bit copy) or F32 (device)

@@ -44,7 +44,7 @@ def run_layer(ug, wl, split=None, poison=True, lr_radius=-1):
             t.fill_(float("nan"))
     o = torch.full((wl.batch, plan.info["N_raster"], wl.heads, wl.D), float("nan"),
                    dtype=torch.bfloat16, device="cuda")
-    lay(qd, kd, vd, o)
+    lay(qd, kd, vd, o, fused=False)
     assert plan.sync_status() == 0
     torch.cuda.synchronize()
     return plan, (q, k, v), lay, o
@@ -197,6 +197,23 @@ def test_attention_lr_region_parity(ug, name, r, heads):
     got = np.stack([to_np64(lay.op[0, h, torch.as_tensor(rows, device="cuda")]) for h in heads])
     assert np.all(got[:, ~real] == 0)
     check_attention(got[:, real], ref[:, real], f"{name} lr_radius={r}")
+
+
+@pytest.mark.parametrize("name,split,r", [("1k", None, -1), ("1k", 5, -1), ("ragged", None, -1),
+                                          ("odd", 3, -1), ("tiny", 2, -1), ("4k", None, 4),
+                                          ("text_only_pad", 1, -1)])
+def test_fused_raster_equals_forward_then_unpermute(ug, name, split, r):
+    """The unpermute folded into the attention epilogue gives the same bits as the two passes."""
+    import torch
+    wl = _wl(name) if name in ("tiny", "1k", "ragged", "4k") else custom(name)
+    plan, (q, k, v), lay, o_two = run_layer(ug, wl, split=split, lr_radius=r)
+    o_one = torch.full_like(o_two, float("nan"))
+    if o_one.dtype != torch.bfloat16:
+        o_one = torch.full(o_two.shape, float("nan"), dtype=torch.bfloat16, device="cuda")
+    ug.hla_forward_raster(lay.qp, lay.kp, lay.vp, o_one, plan)
+    assert plan.sync_status() == 0
+    torch.cuda.synchronize()
+    assert torch.equal(o_one.view(torch.int16), o_two.to(torch.bfloat16).view(torch.int16))
 
 
 def test_deterministic(ug):
