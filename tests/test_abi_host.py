@@ -90,6 +90,8 @@ GEOMS = {
     "odd": (37, 29, 12, 5, 3, 70),
     "small_l": (20, 18, 4, 3, 5, 9),
     "no_lr_text": (40, 24, 8, 8, 0, 0),
+    # window-size / rho ablation shapes of the pages (ws 512 px -> l = 32; rho = 2)
+    "win32_rho2": (96, 96, 32, 8, 2, 64),
 }
 
 
@@ -120,7 +122,7 @@ def compare_plan(ffi, geom, qtiles=None):
     return g, p
 
 
-@pytest.mark.parametrize("name", ["tiny", "1k", "odd", "small_l", "no_lr_text"])
+@pytest.mark.parametrize("name", ["tiny", "1k", "odd", "small_l", "no_lr_text", "win32_rho2"])
 def test_plan_bit_exact_full(ffi, name):
     g, p = compare_plan(ffi, GEOMS[name])
     assert p.info["useful_pairs"] == O.visible_pair_count(g)

@@ -56,6 +56,8 @@ CUSTOM = {
     "small_l": dict(name="small_l", cfg=12, H=20, W=18, l=4, b=3, rho=5, T=9, heads=2, D=64,
                     batch=1, axes=(16, 24, 24), dtype="f32", sinusoid=False),
     "no_lr_text": dict(name="no_lr_text", cfg=13, H=40, W=24, l=8, b=8, rho=0, T=0, heads=2, D=128, batch=1),
+    # ablation shapes of the pages: 512-px windows (l = 32) and rho = 2
+    "win32_rho2": dict(name="win32_rho2", cfg=15, H=96, W=96, l=32, b=8, rho=2, T=64, heads=2, D=128, batch=1),
     "text_only_pad": dict(name="text_only_pad", cfg=14, H=16, W=16, l=16, b=0, rho=2, T=200, heads=2, D=64,
                           batch=1, axes=(8, 28, 28)),
 }
@@ -140,7 +142,7 @@ def test_unpermute_inverts_permute_bitwise(ug, name):
 # ------------------------------------------------------------------ attention
 @pytest.mark.parametrize("name,split", [("tiny", None), ("tiny", 0), ("tiny", 2), ("1k", None),
                                         ("1k", 0), ("1k", 5), ("odd", None), ("odd", 3),
-                                        ("small_l", None), ("no_lr_text", None),
+                                        ("small_l", None), ("no_lr_text", None), ("win32_rho2", None),
                                         ("text_only_pad", 1)])
 def test_attention_full_parity(ug, name, split):
     wl = _wl(name) if name in ("tiny", "1k") else custom(name)
