@@ -51,7 +51,7 @@ def build(verbose: bool = False, force: bool = False) -> str:
             cmd += ["-Xptxas", "-v"]
         if src.endswith(".cpp"):
             cmd = [nvcc(), "-x", "c++", "-c", path, "-o", obj, "-O3", "-std=c++17",
-                   "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC]
+                   "-Wno-deprecated-gpu-targets", "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC]
         if verbose:
             print(" ".join(cmd), flush=True)
         subprocess.run(cmd, check=True)
