@@ -12,6 +12,11 @@ independent layer (no collective on the data path); timing is the max over ranks
 
 --impl reference times the fp64 CPU oracle (the plain restatement the tests check against) on
 a bounded row sample of the same workload, on rank 0 only.
+
+--op warm_start measures the warm-start initialisation instead (one launch per step over a
+synthetic 16-channel latent, --workload warm_8k by default): HBM GB/s of its algorithmic
+bytes (noise read unless --drawn-noise, output written, low-resolution latent read), with L2
+flushed between launches.
 """
 from __future__ import annotations
 
@@ -38,7 +43,8 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="4k")
+    ap.add_argument("--workload", default=None,
+                    help="4k (default), 8k, 1k, ragged; warm_8k (default for --op warm_start), warm_4k")
     ap.add_argument("--heads", type=int, default=0,
                     help="override the workload's head count (smaller profiling captures)")
     ap.add_argument("--lr-radius", type=int, default=-1,
@@ -46,9 +52,15 @@ def parse():
     ap.add_argument("--impl", default="ultragen", choices=["ultragen", "reference"])
     ap.add_argument("--unfused", action="store_true",
                     help="run unpermute as its own pass instead of in the attention epilogue")
+    ap.add_argument("--op", default="hla", choices=["hla", "warm_start"])
+    ap.add_argument("--drawn-noise", action="store_true",
+                    help="warm_start: draw X_T in the kernel instead of reading a noise buffer")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    return ap.parse_args()
+    args = ap.parse_args()
+    if args.workload is None:
+        args.workload = "warm_8k" if args.op == "warm_start" else "4k"
+    return args
 
 
 def peaks():
@@ -213,11 +225,172 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+WARM_METRIC = "warm-start initialisation: HBM GB/s of algorithmic bytes"
+
+
+def warm_bytes(wl, drawn: bool) -> int:
+    n_hr = wl.batch * wl.C * wl.H * wl.W
+    return 4 * n_hr * (1 if drawn else 2) + 4 * wl.batch * wl.C * wl.h * wl.w
+
+
+def warm_cpu_baseline(wl, x_lr, noise, budget_s: float = 10.0):
+    """The warm-start oracle on this host: whole planes, growing until about budget_s."""
+    from oracle import warm_start_oracle as WO
+    t0 = time.perf_counter()
+    planes = 0
+    while True:
+        c = planes % wl.C
+        WO.warm_start(x_lr[:1, c:c + 1].double().numpy(), wl.H, wl.W, wl.alpha, wl.sharpen,
+                      noise=noise[:1, c:c + 1].double().numpy())
+        planes += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    one = warm_bytes(type(wl)(wl.name, wl.cfg, 1, 1, wl.h, wl.w, wl.H, wl.W, wl.alpha, wl.sharpen),
+                     False)
+    return {"value": one * planes / dt / 1e9, "unit": "GB/s", "cores": os.cpu_count(),
+            "kind": "oracle",
+            "sample": f"{planes} plane(s) of {wl.H}x{wl.W} (noise given), fp64 NumPy, "
+                      f"{dt / planes:.2f} s each"}
+
+
+def main_warm(args, rank, world, local):
+    import torch
+    import torch.distributed as dist
+
+    import diffusion_transformer_ultra_b200 as ug
+    wl = ug.WARM_WORKLOADS[args.workload]
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        x_lr, noise = ug.make_warm(wl)
+        per = []
+        for i in range(args.warmup + args.steps):
+            r = warm_cpu_baseline(wl, x_lr, noise, budget_s=0.0)
+            if i >= args.warmup:
+                per.append(r)
+        value = statistics.mean(r["value"] for r in per)
+        print(json.dumps({
+            "impl": "reference", "metric": WARM_METRIC, "value": value, "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * warm_bytes(wl, False) / (value * 1e9),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": wl.name},
+            "cpu_baseline": {"kind": "oracle", "cores": per[-1]["cores"], "sample": per[-1]["sample"],
+                             "value": value, "unit": "GB/s"},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }), flush=True)
+        return
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    x_lr, noise = ug.make_warm(wl)
+    xd, nd = x_lr.cuda(), (None if args.drawn_noise else noise.cuda())
+    out = torch.empty((wl.batch, wl.C, wl.H, wl.W), device="cuda")
+    # L2 flush between launches: writing 256 MB evicts everything, and reading another 256 MB
+    # then replaces those dirty lines with clean ones, so their write-back to HBM happens here
+    # and not inside the next timed launch
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    flush_rd = torch.zeros(64 << 20, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ug.warm_start(xd, out, wl.alpha, wl.sharpen, noise=nd, seed=1234, offset=0)
+        return 1
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    launches = 0
+    for i in range(args.steps):
+        flush.zero_()
+        flush_rd.sum()
+        evs[i][0].record(stream)
+        launches += step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    ms = max_over_ranks(ms, world, "cuda")
+    nbytes = warm_bytes(wl, args.drawn_noise)
+    value = nbytes * world / (ms * 1e-3) / 1e9
+    pk, src = peaks()
+
+    e2e = None
+    if not args.no_e2e:
+        xh = x_lr.pin_memory()
+        nh = noise.pin_memory()
+        oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        nd2 = torch.empty_like(out) if not args.drawn_noise else None
+
+        def e2e_step():
+            xd.copy_(xh, non_blocking=True)
+            if nd2 is not None:
+                nd2.copy_(nh, non_blocking=True)
+            ug.warm_start(xd, out, wl.alpha, wl.sharpen, noise=nd2, seed=1234, offset=0)
+            oh.copy_(out, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(3, args.steps // 4)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms_e2e = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world, "cuda")
+        h2d = x_lr.numel() * 4 + (0 if args.drawn_noise else noise.numel() * 4)
+        e2e = {"value": nbytes * world / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s",
+               "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": out.numel() * 4}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = warm_cpu_baseline(wl, x_lr, noise)
+    if rank == 0:
+        achieved = nbytes / (ms * 1e-3) / 1e9
+        peak = pk["hbm_gbs"]
+        print(json.dumps({
+            "metric": WARM_METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded N(0,1) + smooth sinusoid latent, N(0,1) noise)",
+            "config": {"workload": wl.name, "batch": wl.batch, "channels": wl.C, "h": wl.h,
+                       "w": wl.w, "H": wl.H, "W": wl.W, "alpha": wl.alpha, "sharpen": wl.sharpen,
+                       "noise": "drawn in the kernel (Philox4x32-10)" if args.drawn_noise else "read",
+                       "l2": "flushed before every launch (256 MB written, then 256 MB read)",
+                       "parallelism": f"independent latent per rank x{world}"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "peak_source": f"{src} copy bandwidth",
+                         "algorithmic_bytes_per_launch": nbytes},
+            "e2e": e2e, "gpu_launches": launches, "clocks": clocks, "cpu_baseline": cpu,
+        }), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.op == "warm_start":
+        main_warm(args, rank, world, local)
+        return
     if args.impl == "reference":
         run_reference(args, rank, world)
         return

@@ -6,8 +6,9 @@ the seeded synthetic-input generator.
 """
 from ._ffi import (BF16, F32, Layer, Plan, UltragenError, hla_forward,  # noqa: F401
                    hla_forward_noalloc, hla_forward_raster, lib, permute_rope,
-                   unpermute)
-from .inputs import WORKLOADS, Workload, make_qkv  # noqa: F401
+                   unpermute, warm_start)
+from .inputs import (WARM_WORKLOADS, WORKLOADS, WarmWorkload, Workload,  # noqa: F401
+                     make_qkv, make_warm)
 
 
 def plan_for(wl: "Workload") -> "Plan":

@@ -29,7 +29,7 @@ SYMBOLS = (
     "ultragen_plan_destroy", "ultragen_permute_rope", "ultragen_hla_forward",
     "ultragen_unpermute", "ultragen_sync_status", "ultragen_last_launch_count",
     "ultragen_hla_forward_noalloc", "ultragen_plan_set_diagnostics", "ultragen_plan_set_lr_scope",
-    "ultragen_hla_forward_raster",
+    "ultragen_hla_forward_raster", "ultragen_warm_start",
 )
 
 
@@ -91,6 +91,8 @@ def lib() -> ctypes.CDLL:
     L.ultragen_sync_status.argtypes = [vp, vp]
     L.ultragen_last_launch_count.argtypes = [vp]
     L.ultragen_plan_set_diagnostics.argtypes = [vp, cint, ctypes.c_double]
+    L.ultragen_warm_start.argtypes = [vp, vp, vp] + [cint] * 6 + [ctypes.c_float] * 2 + \
+        [ctypes.c_uint64] * 2 + [vp]
     for name in SYMBOLS:
         if name != "ultragen_status_string":
             getattr(L, name).restype = cint
@@ -260,6 +262,26 @@ def unpermute(op, o, plan: Plan, stream=None):
     dt = BF16 if o.dtype == torch.bfloat16 else F32
     _check("ultragen_unpermute", lib().ultragen_unpermute(
         op.data_ptr(), o.data_ptr(), dt, B, plan.handle, _stream_ptr(stream)))
+
+
+def warm_start(x_lr, x_hr, alpha: float, sharpen: float = 1.0, noise=None, seed: int = 0,
+               offset: int = 0, stream=None):
+    """Warm-start latent x_hr [B, C, H, W] = alpha * X_T + (1 - alpha) * sharpen(upsample(x_lr))
+    (fp32).  X_T is `noise` [B, C, H, W], or the Philox/Box-Muller stream (seed, offset) drawn
+    in the kernel when noise is None."""
+    import torch
+    if x_lr.dim() != 4 or x_hr.dim() != 4:
+        raise ValueError("x_lr and x_hr must be [B, C, h, w] and [B, C, H, W]")
+    B, C, h, w = x_lr.shape
+    H, W = x_hr.shape[2:]
+    _need(x_lr, (B, C, h, w), (torch.float32,), "x_lr")
+    _need(x_hr, (B, C, H, W), (torch.float32,), "x_hr")
+    if noise is not None:
+        _need(noise, (B, C, H, W), (torch.float32,), "noise")
+    _check("ultragen_warm_start", lib().ultragen_warm_start(
+        x_lr.data_ptr(), None if noise is None else noise.data_ptr(), x_hr.data_ptr(), B, C, h, w,
+        H, W, float(alpha), float(sharpen), int(seed), int(offset), _stream_ptr(stream)))
+    return x_hr
 
 
 class Layer:

@@ -331,6 +331,41 @@ int ultragen_sync_status(const ultragen_plan_t* cplan, ultragen_stream_t stream)
 
 int ultragen_last_launch_count(const ultragen_plan_t* p) { return p ? p->last_launches : -1; }
 
+int ultragen_warm_start(const float* x_lr, const float* noise, float* x_hr, int batch,
+                        int channels, int h, int w, int H, int W, float alpha, float sharpen,
+                        uint64_t seed, uint64_t offset, ultragen_stream_t stream) {
+  if (!x_lr || !x_hr || batch < 1 || channels < 1 || h < 1 || w < 1 || H < 1 || W < 1)
+    return ULTRAGEN_ERR_INVALID_ARG;
+  if (!std::isfinite(alpha) || !std::isfinite(sharpen) || sharpen < 0.0f)
+    return ULTRAGEN_ERR_INVALID_ARG;
+  const void* ptrs[] = {x_lr, noise, x_hr};
+  for (const void* x : ptrs)
+    if (reinterpret_cast<uintptr_t>(x) & 3u) return ULTRAGEN_ERR_INVALID_ARG;
+  const int64_t planes = (int64_t)batch * channels;
+  if (planes > 65535 || H > 65535 * 32 || (int64_t)h * w >= ((int64_t)1 << 31))
+    return ULTRAGEN_ERR_UNSUPPORTED;
+  int dev;
+  int st = check_device(&dev);
+  if (st) return st;
+  WarmArgs a;
+  a.lr = x_lr;
+  a.noise = noise;
+  a.out = x_hr;
+  a.planes = (int)planes;
+  a.h = h;
+  a.w = w;
+  a.H = H;
+  a.W = W;
+  a.sy = (float)h / (float)H;
+  a.sx = (float)w / (float)W;
+  a.alpha = alpha;
+  a.amount = sharpen;
+  a.seed = seed;
+  a.offset = offset;
+  a.vec = (W % 4 == 0) && aligned16(x_hr) && (!noise || aligned16(noise));
+  return cuda_status(launch_warm_start(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int ultragen_plan_set_diagnostics(ultragen_plan_t* p, int fault, double wait_limit_s) {
   if (!p || fault < 0 || fault > 1 || !(wait_limit_s >= 1e-3 && wait_limit_s <= 60.0))
     return ULTRAGEN_ERR_INVALID_ARG;

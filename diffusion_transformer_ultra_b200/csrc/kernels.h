@@ -78,6 +78,17 @@ struct FwdParams {
   int N_raster = 0, heads = 1;
 };
 
+struct WarmArgs {
+  const float* lr;                 // [planes, h, w] low-resolution latent
+  const float* noise;              // [planes, H, W] X_T, or null: drawn in the kernel
+  float* out;                      // [planes, H, W]
+  int planes, h, w, H, W;          // planes = batch * channels
+  float sy, sx;                    // h / H, w / W in fp32
+  float alpha, amount;             // blend weight of the noise, unsharp-mask amount
+  unsigned long long seed, offset; // Philox key and the high counter words
+  int vec;                         // 1: W % 4 == 0 and 16-byte aligned noise / out
+};
+
 cudaError_t launch_permute_rope(const PermuteArgs& a, int in_dtype, int D, int grid_x,
                                 cudaStream_t st);
 cudaError_t launch_unpermute(const UnpermuteArgs& a, int out_dtype, int D, int grid_x,
@@ -87,6 +98,7 @@ cudaError_t launch_combine(const CombineArgs& a, int D, cudaStream_t st);
 int make_tmap(CUtensorMap* m, const void* base, uint64_t rows, int D);
 // Streaming multiprocessors of the current device (api.cu).
 int sm_count();
+cudaError_t launch_warm_start(const WarmArgs& a, cudaStream_t st);
 // Launches the block-sparse attention kernel; tensor maps are built by the caller.
 cudaError_t launch_hla_fwd(const void* tmQ, const void* tmK, const void* tmV,
                            const FwdParams& p, int D, int grid, cudaStream_t st);

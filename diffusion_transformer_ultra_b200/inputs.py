@@ -14,6 +14,11 @@ Recipe (per tensor, raster layout [B, N_raster, heads, D], segment order text | 
   * bf16 workloads are rounded to bfloat16 (round to nearest even); the tiny workload
     stays float32.
 Seeds: Q/K/V = 1000*cfg + {1, 2, 3}; sinusoid parameters = 1000*cfg + 7.
+
+Warm-start latents (``make_warm``): the low-resolution latent [B, C, h, w] is i.i.d. N(0, 1)
+plus a smooth per-channel 2D sinusoid of amplitude 1 (a stand-in for generated image
+structure); the noise X_T [B, C, H, W] is i.i.d. N(0, 1); both float32.  Seeds
+1000*cfg + 11 (latent), + 12 (noise), + 13 (sinusoid).
 """
 from __future__ import annotations
 
@@ -134,3 +139,45 @@ def make_tensor(wl: Workload, which: str, threads: int | None = None):
 
 def make_qkv(wl: Workload, threads: int | None = None):
     return tuple(make_tensor(wl, w, threads) for w in ("q", "k", "v"))
+
+
+@dataclass(frozen=True)
+class WarmWorkload:
+    name: str
+    cfg: int
+    batch: int
+    C: int              # latent channels
+    h: int
+    w: int
+    H: int
+    W: int
+    alpha: float        # t / T of the starting timestep
+    sharpen: float      # unsharp-mask amount
+
+
+WARM_WORKLOADS = {
+    "warm_tiny": WarmWorkload("warm_tiny", 20, 1, 4, 16, 16, 64, 64, 0.7, 1.0),
+    "warm_ragged": WarmWorkload("warm_ragged", 21, 2, 3, 13, 11, 50, 47, 0.3, 0.5),
+    # 4K / 8K images: 16-channel latents at 1/8 of the pixel grid, guide at rho = 4
+    "warm_4k": WarmWorkload("warm_4k", 22, 1, 16, 128, 128, 512, 512, 0.7, 1.0),
+    "warm_8k": WarmWorkload("warm_8k", 23, 1, 16, 256, 256, 1024, 1024, 0.7, 1.0),
+}
+
+
+def make_warm(wl: WarmWorkload):
+    """(x_lr [B, C, h, w], noise [B, C, H, W]) as CPU float32 torch tensors."""
+    import torch
+
+    rng = np.random.default_rng(1000 * wl.cfg + 11)
+    x = rng.standard_normal((wl.batch, wl.C, wl.h, wl.w), dtype=np.float32)
+    prm = np.random.default_rng(1000 * wl.cfg + 13)
+    u = prm.integers(1, 4, size=wl.C)
+    v = prm.integers(1, 4, size=wl.C)
+    phi = prm.uniform(0.0, 2.0 * np.pi, size=wl.C)
+    yy = np.arange(wl.h)[:, None] / wl.h
+    xx = np.arange(wl.w)[None, :] / wl.w
+    for c in range(wl.C):
+        x[:, c] += np.sin(2.0 * np.pi * (u[c] * yy + v[c] * xx) + phi[c]).astype(np.float32)
+    noise = np.random.default_rng(1000 * wl.cfg + 12).standard_normal(
+        (wl.batch, wl.C, wl.H, wl.W), dtype=np.float32)
+    return torch.from_numpy(x), torch.from_numpy(noise)

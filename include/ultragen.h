@@ -218,6 +218,31 @@ int ultragen_plan_set_diagnostics(ultragen_plan_t* plan, int fault, double wait_
 /* Kernel launches the last device call of this plan issued (for launch accounting). */
 int ultragen_last_launch_count(const ultragen_plan_t* plan);
 
+/*
+ * ultragen_warm_start -- warm-start initialisation of the high-resolution latent
+ * ([UG-note] 关键设计 4 and its blend equation; [UG-gist] 2.D "Warm-Start Initialization"):
+ *     U     = bilinear upsampling of x_lr to H x W: along each axis output index i reads
+ *             source coordinate max((i + 1/2) * n_in / n_out - 1/2, 0), taps floor() and the
+ *             next index (both clamped to n_in - 1), weighted by the fractional part;
+ *     X_ref = U + sharpen * (U - B(U)), B the 3x3 binomial blur (1 2 1)^T (1 2 1) / 16 per
+ *             channel with replicated edges (sharpen = 0: plain interpolation);
+ *     x_hr  = alpha * X_T + (1 - alpha) * X_ref, alpha = t / T of the starting timestep.
+ *   x_lr   [batch, channels, h, w] F32 (device)
+ *   noise  [batch, channels, H, W] F32 (device) X_T, or NULL: X_T is drawn in the kernel from
+ *          Philox4x32-10 (key = seed, counter = (g, offset) for 4-element block g of the flat
+ *          output index) and the Box-Muller transform of the words mapped to
+ *          (floor(x / 2^9) + 1/2) * 2^-23; lanes 0..3 of a block are r cos, r sin of words
+ *          (0, 1), then of words (2, 3).
+ *   x_hr   [batch, channels, H, W] F32 (device), written in full.
+ *   Pointers need 4-byte alignment; W % 4 == 0 with 16-byte aligned noise and x_hr takes the
+ *   vector path.  INVALID_ARG: null x_lr / x_hr, a size < 1, a non-finite alpha or sharpen,
+ *   sharpen < 0.  UNSUPPORTED: batch * channels > 65535 or H > 2,097,120.  Computed in fp32.
+ *   One kernel launch; asynchronous on `stream`.
+ */
+int ultragen_warm_start(const float* x_lr, const float* noise, float* x_hr, int batch,
+                        int channels, int h, int w, int H, int W, float alpha, float sharpen,
+                        uint64_t seed, uint64_t offset, ultragen_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -130,10 +130,11 @@ def box_muller(u1, u2):
     return r * np.cos(2.0 * np.pi * u2), r * np.sin(2.0 * np.pi * u2)
 
 
-def philox_normals(seed: int, offset: int, n: int) -> np.ndarray:
-    """The first n standard normals of the stream (seed, offset), in fp64 (reading W3)."""
-    n_blocks = (n + 3) // 4
-    g = np.arange(n_blocks, dtype=np.uint64)
+def philox_normals(seed: int, offset: int, n: int, first: int = 0) -> np.ndarray:
+    """Normals first .. first + n - 1 of the stream (seed, offset), in fp64 (reading W3)."""
+    g0 = first // 4
+    n_blocks = (first + n + 3) // 4 - g0
+    g = np.arange(g0, g0 + n_blocks, dtype=np.uint64)
     zeros = np.zeros_like(g)
     ctr = (g & _MASK32, g >> np.uint64(32), zeros + np.uint64(offset & 0xFFFFFFFF),
            zeros + np.uint64(offset >> 32))
@@ -141,7 +142,8 @@ def philox_normals(seed: int, offset: int, n: int) -> np.ndarray:
     x0, x1, x2, x3 = philox4x32_10(ctr, key)
     z0, z1 = box_muller(uniform_open(x0), uniform_open(x1))
     z2, z3 = box_muller(uniform_open(x2), uniform_open(x3))
-    return np.stack([z0, z1, z2, z3], axis=1).reshape(-1)[:n]
+    z = np.stack([z0, z1, z2, z3], axis=1).reshape(-1)
+    return z[first - 4 * g0:first - 4 * g0 + n]
 
 
 # ---------------------------------------------------------------------------- blend

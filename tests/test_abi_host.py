@@ -81,6 +81,31 @@ def test_device_calls_without_device_fail_cleanly(ffi):
     assert st in (3, 7)
     assert L.ultragen_hla_forward(None, a, a, a, p.handle, 1, None) == 1
     assert L.ultragen_permute_rope(a, a, a, 5, a, a, a, 1, p.handle, None) == 1
+    assert L.ultragen_warm_start(a, None, a, 1, 1, 4, 4, 16, 16, 0.5, 1.0, 0, 0, None) in (3, 7)
+
+
+def test_warm_start_argument_checks(ffi):
+    """Argument errors come back before any device work (safe with or without a GPU)."""
+    L = ffi.lib()
+    buf = ctypes.create_string_buffer(1 << 12)
+    a = ctypes.addressof(buf) + (-ctypes.addressof(buf)) % 16
+    ok = (a, None, a, 1, 4, 8, 8, 32, 32, 0.5, 1.0, 7, 0, None)
+
+    def call(**kw):
+        args = list(ok)
+        for i, name in enumerate(("lr", "noise", "out", "B", "C", "h", "w", "H", "W", "alpha",
+                                  "sharpen", "seed", "offset", "stream")):
+            if name in kw:
+                args[i] = kw[name]
+        return L.ultragen_warm_start(*args)
+
+    assert call(lr=None) == 1
+    assert call(out=None) == 1
+    assert call(B=0) == 1 and call(C=-1) == 1 and call(h=0) == 1 and call(W=0) == 1
+    assert call(sharpen=-0.5) == 1
+    assert call(alpha=float("nan")) == 1 and call(sharpen=float("inf")) == 1
+    assert call(lr=a + 2) == 1 and call(noise=a + 1) == 1
+    assert call(B=300, C=300) == 2
 
 
 GEOMS = {

@@ -106,6 +106,7 @@ def test_philox_normals_are_standard_normal():
     assert not np.allclose(WO.philox_normals(1234, 1, 64), z[:64])
     assert not np.allclose(WO.philox_normals(1235, 0, 64), z[:64])
     np.testing.assert_array_equal(WO.philox_normals(1234, 0, 7), z[:7])
+    np.testing.assert_array_equal(WO.philox_normals(1234, 0, 9, first=1001), z[1001:1010])
 
 
 def test_blend_special_cases():
