@@ -56,6 +56,8 @@ def parse():
     ap.add_argument("--drawn-noise", action="store_true",
                     help="warm_start: draw X_T in the kernel instead of reading a noise buffer")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-heads-per-chunk", type=int, default=3,
+                    help="head slice per pipelined unit of the host-buffer (e2e) measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.workload is None:
@@ -482,27 +484,30 @@ def main():
 
     e2e = None
     if not args.no_e2e:
-        qh, kh, vh = (x.pin_memory() for x in (q, k, v))
+        # the public host-buffer call: page-locked Q/K/V in, O out, copies overlapped with the
+        # kernels of other head slices
+        qh, kh, vh = (x.to(torch.bfloat16).pin_memory() for x in (q, k, v))
         oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        runner = ug.HostRunner(plan, wl.batch, args.e2e_heads_per_chunk)
         for _ in range(2):
-            qd.copy_(qh, non_blocking=True); kd.copy_(kh, non_blocking=True); vd.copy_(vh, non_blocking=True)
-            step()
-            oh.copy_(o, non_blocking=True)
+            runner(qh, kh, vh, oh)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         n_e2e = max(3, args.steps // 4)
         e0.record(stream)
         for _ in range(n_e2e):
-            qd.copy_(qh, non_blocking=True); kd.copy_(kh, non_blocking=True); vd.copy_(vh, non_blocking=True)
-            step()
-            oh.copy_(o, non_blocking=True)
+            runner(qh, kh, vh, oh)
         e1.record(stream)
         torch.cuda.synchronize()
+        if plan.sync_status() != 0:
+            raise RuntimeError("device error during the end-to-end steps")
         ms_e2e = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world, "cuda")
         e2e = {"value": job_tflops(flops, world, ms_e2e), "unit": "useful TFLOP/s",
-               "ms_per_step": ms_e2e,
-               "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
-               "d2h_bytes_per_step": o.numel() * o.element_size()}
+               "ms_per_step": ms_e2e, "api": "ultragen_host_runner_forward (host buffers)",
+               "heads_per_chunk": args.e2e_heads_per_chunk,
+               "h2d_bytes_per_step": 3 * qh.numel() * qh.element_size(),
+               "d2h_bytes_per_step": oh.numel() * oh.element_size()}
+        runner.close()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

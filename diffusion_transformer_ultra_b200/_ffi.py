@@ -29,7 +29,9 @@ SYMBOLS = (
     "ultragen_plan_destroy", "ultragen_permute_rope", "ultragen_hla_forward",
     "ultragen_unpermute", "ultragen_sync_status", "ultragen_last_launch_count",
     "ultragen_hla_forward_noalloc", "ultragen_plan_set_diagnostics", "ultragen_plan_set_lr_scope",
-    "ultragen_hla_forward_raster", "ultragen_warm_start",
+    "ultragen_hla_forward_raster", "ultragen_warm_start", "ultragen_host_runner_create",
+    "ultragen_host_runner_forward", "ultragen_host_runner_last_launch_count",
+    "ultragen_host_runner_destroy",
 )
 
 
@@ -93,6 +95,10 @@ def lib() -> ctypes.CDLL:
     L.ultragen_plan_set_diagnostics.argtypes = [vp, cint, ctypes.c_double]
     L.ultragen_warm_start.argtypes = [vp, vp, vp] + [cint] * 6 + [ctypes.c_float] * 2 + \
         [ctypes.c_uint64] * 2 + [vp]
+    L.ultragen_host_runner_create.argtypes = [vp, cint, cint, ctypes.POINTER(vp)]
+    L.ultragen_host_runner_forward.argtypes = [vp, vp, vp, vp, vp, vp]
+    L.ultragen_host_runner_last_launch_count.argtypes = [vp]
+    L.ultragen_host_runner_destroy.argtypes = [vp]
     for name in SYMBOLS:
         if name != "ultragen_status_string":
             getattr(L, name).restype = cint
@@ -282,6 +288,46 @@ def warm_start(x_lr, x_hr, alpha: float, sharpen: float = 1.0, noise=None, seed:
         x_lr.data_ptr(), None if noise is None else noise.data_ptr(), x_hr.data_ptr(), B, C, h, w,
         H, W, float(alpha), float(sharpen), int(seed), int(offset), _stream_ptr(stream)))
     return x_hr
+
+
+class HostRunner:
+    """The whole layer for Q/K/V and O in host memory, PCIe copies overlapped with the kernels
+    (units of heads_per_chunk heads; see ultragen_host_runner_create)."""
+
+    def __init__(self, plan: Plan, batch: int, heads_per_chunk: int = 3):
+        self.plan = plan
+        self.batch = batch
+        self._h = ctypes.c_void_p()
+        _check("ultragen_host_runner_create", lib().ultragen_host_runner_create(
+            plan.handle, int(batch), int(heads_per_chunk), ctypes.byref(self._h)))
+
+    def __call__(self, q, k, v, o, stream=None):
+        """q, k, v, o: CPU bf16 [batch, N_raster, heads, D] (page-locked for overlap)."""
+        import torch
+        i = self.plan.info
+        shape = (self.batch, i["N_raster"], i["heads"], i["head_dim"])
+        for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+            if not isinstance(t, torch.Tensor) or t.is_cuda:
+                raise ValueError(f"{n} must be a host tensor")
+            if tuple(t.shape) != shape or t.dtype != torch.bfloat16 or not t.is_contiguous():
+                raise ValueError(f"{n} must be contiguous bf16 {shape}")
+        _check("ultragen_host_runner_forward", lib().ultragen_host_runner_forward(
+            self._h, q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), _stream_ptr(stream)))
+        return o
+
+    def last_launch_count(self) -> int:
+        return lib().ultragen_host_runner_last_launch_count(self._h)
+
+    def close(self):
+        if self._h:
+            lib().ultragen_host_runner_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 class Layer:

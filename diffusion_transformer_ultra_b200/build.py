@@ -16,7 +16,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libultragen.so")
 
-SOURCES = ["plan.cpp", "api.cu", "permute.cu", "hla_fwd.cu", "noalloc.cu", "warm_start.cu"]
+SOURCES = ["plan.cpp", "api.cu", "permute.cu", "hla_fwd.cu", "noalloc.cu", "warm_start.cu", "host_runner.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -141,6 +141,98 @@ int sm_count() {
   return n > 0 ? n : 148;
 }
 
+int ensure_device_tables(ultragen_plan_t* p) { return ensure_device(p); }
+
+size_t split_workspace_bytes(const ultragen_plan_t* p, int64_t units) {
+  return (size_t)units * p->n_split_items * 2 * kTile * (p->D + 1) * sizeof(float);
+}
+
+// Attention over `units` (batch, head) pairs whose permuted Q/K/V start at qp/kp/vp; a raster
+// output is laid out [units / heads][N_raster][heads][D].  The plan's tables must already be on
+// the device and `ws` must hold split_workspace_bytes(p, units).
+int launch_attention(const ultragen_plan_t* p, const void* qp, const void* kp, const void* vp,
+                     void* op, int units, int heads, int raster, float* ws, cudaStream_t s,
+                     int* launches) {
+  const int64_t rows = (int64_t)units * p->N_tot;
+  const int64_t items = (int64_t)units * (int64_t)p->items.size();
+  alignas(64) CUtensorMap tq, tk, tv;
+  int st;
+  if ((st = make_tmap(&tq, qp, rows, p->D)) || (st = make_tmap(&tk, kp, rows, p->D)) ||
+      (st = make_tmap(&tv, vp, rows, p->D)))
+    return st;
+  FwdParams f;
+  f.items = p->dev.items;
+  f.entries = p->dev.entries;
+  f.mask_off = p->dev.mask_off;
+  f.mask_pool = p->dev.mask_pool;
+  f.perm = p->dev.perm;
+  f.out = static_cast<__nv_bfloat16*>(op);
+  f.ws = ws;
+  f.err = p->dev.error;
+  f.n_items_head = (int)p->items.size();
+  f.total_items = (int)items;
+  f.N_tot = (int)p->N_tot;
+  f.off_hr = (int)p->off_hr;
+  f.l2 = p->l * p->l;
+  f.n_ws_head = p->n_split_items;
+  f.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)p->D));
+  f.timeout_ns = p->wait_limit_ns;
+  f.fault = p->fault;
+  f.raster = raster;
+  f.N_raster = (int)p->N_raster;
+  f.heads = heads;
+  const int grid = (int)std::min<int64_t>(items, sm_count());
+  *launches = 0;
+  if (grid > 0) {
+    st = cuda_status(launch_hla_fwd(&tq, &tk, &tv, f, p->D, grid, s));
+    if (st) return st;
+    ++*launches;
+  }
+  if (!p->combine.empty()) {
+    CombineArgs c;
+    c.ws = ws;
+    c.out = f.out;
+    c.groups = p->dev.combine;
+    c.perm = p->dev.perm;
+    c.n_groups = (int)p->combine.size();
+    c.n_ws_head = p->n_split_items;
+    c.N_tot = (int)p->N_tot;
+    c.BH = units;
+    c.raster = raster;
+    c.N_raster = (int)p->N_raster;
+    c.heads = heads;
+    st = cuda_status(launch_combine(c, p->D, s));
+    if (st) return st;
+    ++*launches;
+  }
+  return ULTRAGEN_OK;
+}
+
+// permute_rope over `batch` raster blocks of `heads` heads: raster [batch][N_raster][heads][D]
+// -> permuted [batch][heads][N_tot][D].  The plan's tables must already be on the device.
+int launch_permute(const ultragen_plan_t* p, const void* q, const void* k, const void* v,
+                   int in_dtype, void* qp, void* kp, void* vp, int batch, int heads,
+                   cudaStream_t s) {
+  PermuteArgs a;
+  a.in[0] = q; a.in[1] = k; a.in[2] = v;
+  a.out[0] = static_cast<__nv_bfloat16*>(qp);
+  a.out[1] = static_cast<__nv_bfloat16*>(kp);
+  a.out[2] = static_cast<__nv_bfloat16*>(vp);
+  a.perm = p->dev.perm;
+  a.slot_pos = p->dev.slot_pos;
+  a.rope = p->dev.rope;
+  a.rows_total = (int64_t)batch * heads * p->N_tot;
+  a.N_tot = (int)p->N_tot;
+  a.N_raster = (int)p->N_raster;
+  a.heads = heads;
+  a.div_heads = FastDiv((uint32_t)heads);
+  a.div_ntot = FastDiv((uint32_t)p->N_tot);
+  a.pair_a0 = p->axes[0] / 2;
+  a.pair_a01 = (p->axes[0] + p->axes[1]) / 2;
+  const int rows_per_block = 256 / (p->D / 8);
+  return cuda_status(launch_permute_rope(a, in_dtype, p->D, grid_for(a.rows_total, rows_per_block), s));
+}
+
 }  // namespace ug
 
 using namespace ug;
@@ -168,26 +260,9 @@ int ultragen_permute_rope(const void* q, const void* k, const void* v, int in_dt
     return ULTRAGEN_ERR_UNSUPPORTED;
   int st = ensure_device(p);
   if (st) return st;
-  PermuteArgs a;
-  a.in[0] = q; a.in[1] = k; a.in[2] = v;
-  a.out[0] = static_cast<__nv_bfloat16*>(qp);
-  a.out[1] = static_cast<__nv_bfloat16*>(kp);
-  a.out[2] = static_cast<__nv_bfloat16*>(vp);
-  a.perm = p->dev.perm;
-  a.slot_pos = p->dev.slot_pos;
-  a.rope = p->dev.rope;
-  a.rows_total = (int64_t)batch * p->heads * p->N_tot;
-  a.N_tot = (int)p->N_tot;
-  a.N_raster = (int)p->N_raster;
-  a.heads = p->heads;
-  a.div_heads = FastDiv((uint32_t)p->heads);
-  a.div_ntot = FastDiv((uint32_t)p->N_tot);
-  a.pair_a0 = p->axes[0] / 2;
-  a.pair_a01 = (p->axes[0] + p->axes[1]) / 2;
-  const int rows_per_block = 256 / (p->D / 8);
   p->last_launches = 1;
-  return cuda_status(launch_permute_rope(a, in_dtype, p->D, grid_for(a.rows_total, rows_per_block),
-                                         reinterpret_cast<cudaStream_t>(stream)));
+  return launch_permute(p, q, k, v, in_dtype, qp, kp, vp, batch, p->heads,
+                        reinterpret_cast<cudaStream_t>(stream));
 }
 
 // The attention forward; `raster` selects the output layout (0: permuted, 1: raster).
@@ -207,7 +282,7 @@ static int hla_forward_impl(const void* qp, const void* kp, const void* vp, void
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 
   // split workspace, owned by the plan and grown on demand
-  const size_t ws_need = (size_t)batch * p->heads * p->n_split_items * 2 * kTile * (p->D + 1) * sizeof(float);
+  const size_t ws_need = ug::split_workspace_bytes(p, batch * p->heads);
   if (ws_need > p->dev.ws_bytes) {
     if (p->dev.ws) {
       cudaStreamSynchronize(s);
@@ -222,58 +297,11 @@ static int hla_forward_impl(const void* qp, const void* kp, const void* vp, void
     }
     p->dev.ws_bytes = ws_need;
   }
-
-  alignas(64) CUtensorMap tq, tk, tv;
-  if ((st = make_tmap(&tq, qp, rows, p->D)) || (st = make_tmap(&tk, kp, rows, p->D)) ||
-      (st = make_tmap(&tv, vp, rows, p->D)))
-    return st;
-
-  FwdParams f;
-  f.items = p->dev.items;
-  f.entries = p->dev.entries;
-  f.mask_off = p->dev.mask_off;
-  f.mask_pool = p->dev.mask_pool;
-  f.perm = p->dev.perm;
-  f.out = static_cast<__nv_bfloat16*>(op);
-  f.ws = p->dev.ws;
-  f.err = p->dev.error;
-  f.n_items_head = (int)p->items.size();
-  f.total_items = (int)items;
-  f.N_tot = (int)p->N_tot;
-  f.off_hr = (int)p->off_hr;
-  f.l2 = p->l * p->l;
-  f.n_ws_head = p->n_split_items;
-  f.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)p->D));
-  f.timeout_ns = p->wait_limit_ns;
-  f.fault = p->fault;
-  f.raster = raster;
-  f.N_raster = (int)p->N_raster;
-  f.heads = p->heads;
-  const int grid = (int)std::min<int64_t>(items, sm_count());
-  p->last_launches = 0;
-  if (grid > 0) {
-    st = cuda_status(launch_hla_fwd(&tq, &tk, &tv, f, p->D, grid, s));
-    if (st) return st;
-    p->last_launches++;
-  }
-  if (!p->combine.empty()) {
-    CombineArgs c;
-    c.ws = p->dev.ws;
-    c.out = f.out;
-    c.groups = p->dev.combine;
-    c.perm = p->dev.perm;
-    c.n_groups = (int)p->combine.size();
-    c.n_ws_head = p->n_split_items;
-    c.N_tot = (int)p->N_tot;
-    c.BH = batch * p->heads;
-    c.raster = raster;
-    c.N_raster = (int)p->N_raster;
-    c.heads = p->heads;
-    st = cuda_status(launch_combine(c, p->D, s));
-    if (st) return st;
-    p->last_launches++;
-  }
-  return ULTRAGEN_OK;
+  int launches = 0;
+  st = ug::launch_attention(p, qp, kp, vp, op, batch * p->heads, p->heads, raster, p->dev.ws, s,
+                            &launches);
+  p->last_launches = launches;
+  return st;
 }
 
 int ultragen_hla_forward(const void* qp, const void* kp, const void* vp, void* op,

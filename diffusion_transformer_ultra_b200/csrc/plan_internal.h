@@ -99,4 +99,16 @@ int build_tables(ultragen_plan_t* p);
 void build_schedule(ultragen_plan_t* p);
 // Fills the RoPE table on the host: [max(H,W)][D/2][2] (cos, sin) floats (plan.cpp).
 std::vector<float> rope_table(const ultragen_plan_t* p);
+
+// Device-side launch helpers shared by the entry points (api.cu).  They take the number of
+// (batch, head) units and the raster head count explicitly, so a caller can run a slice of the
+// heads; the plan's tables must already be on the current device.
+int ensure_device_tables(ultragen_plan_t* p);
+size_t split_workspace_bytes(const ultragen_plan_t* p, int64_t units);
+int launch_permute(const ultragen_plan_t* p, const void* q, const void* k, const void* v,
+                   int in_dtype, void* qp, void* kp, void* vp, int batch, int heads,
+                   ultragen_stream_t s);
+int launch_attention(const ultragen_plan_t* p, const void* qp, const void* kp, const void* vp,
+                     void* op, int units, int heads, int raster, float* ws, ultragen_stream_t s,
+                     int* launches);
 }  // namespace ug

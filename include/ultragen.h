@@ -219,6 +219,43 @@ int ultragen_plan_set_diagnostics(ultragen_plan_t* plan, int fault, double wait_
 int ultragen_last_launch_count(const ultragen_plan_t* plan);
 
 /*
+ * Host-buffer runner -- the whole layer for Q/K/V and O in HOST memory, with the PCIe copies
+ * overlapped with the kernels (no counterpart in the pages; it serves callers whose
+ * activations live on the host).  The heads are independent problems, so the layer runs as
+ * units of (batch element, heads_per_chunk heads): each unit's slice is copied in with one 2D
+ * copy per tensor, permuted and attended exactly as ultragen_permute_rope +
+ * ultragen_hla_forward_raster would (the same kernels, bit for bit), and copied out, while the
+ * next unit's copy-in and the previous unit's copy-out proceed on their own streams.
+ *
+ * ultragen_host_runner_create(plan, batch, heads_per_chunk, &runner)
+ *   Allocates every device buffer the runner needs: double-buffered staging for 3 inputs and
+ *   1 output of one unit (2 x 4 x N_raster x heads_per_chunk x head_dim x 2 bytes), permuted
+ *   Q/K/V of one unit, split partials of one unit; three streams and their events.  Uploads the
+ *   plan's tables.  heads_per_chunk is clamped to the plan's head count.  The plan must outlive
+ *   the runner.  INVALID_ARG for a null plan / out, batch < 1, heads_per_chunk < 1;
+ *   NO_DEVICE, OOM, CUDA as usual.
+ * ultragen_host_runner_forward(runner, q, k, v, o, stream)
+ *   q, k, v  [batch, N_raster, heads, head_dim] BF16 in HOST memory (page-locked memory lets
+ *            the copies overlap the kernels; pageable memory works, serialised)
+ *   o        [batch, N_raster, heads, head_dim] BF16 in HOST memory, written in full
+ *   Asynchronous: the work is ordered after what `stream` holds at the call, and `stream`
+ *   waits for all of it, so o is complete once `stream` is synchronised.  Calls on one runner
+ *   must not overlap (one call at a time per runner).  PLAN_MISMATCH when called on another
+ *   device than the one the runner was created on, or when the plan's split schedule now needs
+ *   more partial storage than was allocated.  Device-side wait timeouts are reported by
+ *   ultragen_sync_status(plan, stream).
+ * ultragen_host_runner_last_launch_count(runner): kernels the last forward launched.
+ * ultragen_host_runner_destroy(runner): waits for the runner's streams, frees everything.
+ */
+typedef struct ultragen_host_runner ultragen_host_runner_t;   /* opaque */
+int ultragen_host_runner_create(ultragen_plan_t* plan, int batch, int heads_per_chunk,
+                                ultragen_host_runner_t** out);
+int ultragen_host_runner_forward(ultragen_host_runner_t* runner, const void* q, const void* k,
+                                 const void* v, void* o, ultragen_stream_t stream);
+int ultragen_host_runner_last_launch_count(const ultragen_host_runner_t* runner);
+int ultragen_host_runner_destroy(ultragen_host_runner_t* runner);
+
+/*
  * ultragen_warm_start -- warm-start initialisation of the high-resolution latent
  * ([UG-note] 关键设计 4 and its blend equation; [UG-gist] 2.D "Warm-Start Initialization"):
  *     U     = bilinear upsampling of x_lr to H x W: along each axis output index i reads

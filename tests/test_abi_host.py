@@ -82,6 +82,25 @@ def test_device_calls_without_device_fail_cleanly(ffi):
     assert L.ultragen_hla_forward(None, a, a, a, p.handle, 1, None) == 1
     assert L.ultragen_permute_rope(a, a, a, 5, a, a, a, 1, p.handle, None) == 1
     assert L.ultragen_warm_start(a, None, a, 1, 1, 4, 4, 16, 16, 0.5, 1.0, 0, 0, None) in (3, 7)
+    r = ctypes.c_void_p()
+    assert L.ultragen_host_runner_create(p.handle, 1, 4, ctypes.byref(r)) in (3, 7)
+    assert not r.value
+
+
+def test_host_runner_argument_checks(ffi):
+    """Argument errors of the host runner come back before any device work."""
+    L = ffi.lib()
+    p = ffi.Plan(8, 8, 4, 1, 2, 3, 2, 64)
+    r = ctypes.c_void_p()
+    assert L.ultragen_host_runner_create(None, 1, 1, ctypes.byref(r)) == 1
+    assert L.ultragen_host_runner_create(p.handle, 0, 1, ctypes.byref(r)) == 1
+    assert L.ultragen_host_runner_create(p.handle, 1, 0, ctypes.byref(r)) == 1
+    assert L.ultragen_host_runner_create(p.handle, 1, 1, None) == 1
+    buf = ctypes.create_string_buffer(64)
+    a = ctypes.addressof(buf)
+    assert L.ultragen_host_runner_forward(None, a, a, a, a, None) == 1
+    assert L.ultragen_host_runner_destroy(None) == 1
+    assert L.ultragen_host_runner_last_launch_count(None) == -1
 
 
 def test_warm_start_argument_checks(ffi):
