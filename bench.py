@@ -56,7 +56,7 @@ def parse():
     ap.add_argument("--drawn-noise", action="store_true",
                     help="warm_start: draw X_T in the kernel instead of reading a noise buffer")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--e2e-heads-per-chunk", type=int, default=3,
+    ap.add_argument("--e2e-heads-per-chunk", type=int, default=2,
                     help="head slice per pipelined unit of the host-buffer (e2e) measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

@@ -294,7 +294,7 @@ class HostRunner:
     """The whole layer for Q/K/V and O in host memory, PCIe copies overlapped with the kernels
     (units of heads_per_chunk heads; see ultragen_host_runner_create)."""
 
-    def __init__(self, plan: Plan, batch: int, heads_per_chunk: int = 3):
+    def __init__(self, plan: Plan, batch: int, heads_per_chunk: int = 2):
         self.plan = plan
         self.batch = batch
         self._h = ctypes.c_void_p()
