@@ -67,6 +67,8 @@ WORKLOADS = {
     "4k": Workload("4k", 2, 256, 256, 16, 4, 4, 512, 24, 128, 1, "bf16"),
     "8k": Workload("8k", 3, 512, 512, 16, 4, 4, 512, 24, 128, 1, "bf16"),
     "ragged": Workload("ragged", 4, 256, 135, 16, 16, 4, 256, 24, 128, 2, "bf16"),
+    # the largest layer considered: a 16K image (1024 x 1024 HR tokens, 256 x 256 LR)
+    "16k": Workload("16k", 5, 1024, 1024, 16, 4, 4, 512, 24, 128, 1, "bf16"),
 }
 
 

@@ -136,6 +136,12 @@ GEOMS = {
     "no_lr_text": (40, 24, 8, 8, 0, 0),
     # window-size / rho ablation shapes of the pages (ws 512 px -> l = 32; rho = 2)
     "win32_rho2": (96, 96, 32, 8, 2, 64),
+    # degenerate cases: one token; a window larger than the image; rho larger than the image
+    # (one LR token); a 3-row strip with a text segment one past a tile boundary
+    "single": (1, 1, 1, 0, 1, 0),
+    "win_exceeds": (5, 7, 16, 3, 8, 3),
+    "rho_exceeds": (4, 4, 2, 2, 8, 1),
+    "thin": (3, 130, 4, 1, 2, 129),
 }
 
 
@@ -166,7 +172,8 @@ def compare_plan(ffi, geom, qtiles=None):
     return g, p
 
 
-@pytest.mark.parametrize("name", ["tiny", "1k", "odd", "small_l", "no_lr_text", "win32_rho2"])
+@pytest.mark.parametrize("name", ["tiny", "1k", "odd", "small_l", "no_lr_text", "win32_rho2",
+                                  "single", "win_exceeds", "rho_exceeds", "thin"])
 def test_plan_bit_exact_full(ffi, name):
     g, p = compare_plan(ffi, GEOMS[name])
     assert p.info["useful_pairs"] == O.visible_pair_count(g)
@@ -244,3 +251,23 @@ def test_region_plan_large_sampled(ffi):
         assert p.info["useful_pairs"] == sum(closed_form_pairs(*geom, lr_radius=r).values())
     p = ffi.Plan(64, 64, 16, 4, 4, 512, 2, 64)
     assert ffi.lib().ultragen_plan_set_lr_scope(p.handle, -2) == 1
+
+
+def test_plan_at_16k_maximum_size(ffi):
+    """The largest layer considered (a 16K image: 1024 x 1024 HR tokens, 256 x 256 LR): the plan
+    builds, stays inside the int32 limits of the launch arithmetic for 24 heads, and its visible
+    pair count equals the closed form."""
+    import importlib.util
+    import os
+    spec = importlib.util.spec_from_file_location(
+        "pins", os.path.join(os.path.dirname(__file__), "test_oracle_pins.py"))
+    pins = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(pins)
+    geom = (1024, 1024, 16, 4, 4, 512)
+    p = ffi.Plan(*geom, 24, 128)
+    i = p.info
+    assert sum(pins.closed_form_pairs(*geom).values()) == i["useful_pairs"]
+    assert 24 * i["N_tot"] < 2 ** 31 and 24 * i["N_raster"] < 2 ** 31
+    assert 24 * i["n_items"] < 2 ** 31
+    g = O.Geometry(*geom)
+    assert (i["N_tot"], i["N_raster"], i["off_hr"], i["off_lr"]) == (g.N_tot, g.N_raster, g.off_hr, g.off_lr)

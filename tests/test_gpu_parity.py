@@ -60,6 +60,13 @@ CUSTOM = {
     "win32_rho2": dict(name="win32_rho2", cfg=15, H=96, W=96, l=32, b=8, rho=2, T=64, heads=2, D=128, batch=1),
     "text_only_pad": dict(name="text_only_pad", cfg=14, H=16, W=16, l=16, b=0, rho=2, T=200, heads=2, D=64,
                           batch=1, axes=(8, 28, 28)),
+    # degenerate cases: one HR token (and one LR token); a window larger than the image; rho
+    # larger than the image; a 3-row strip whose text segment ends one past a tile boundary
+    "single": dict(name="single", cfg=16, H=1, W=1, l=1, b=0, rho=1, T=0, heads=2, D=128, batch=1),
+    "win_exceeds": dict(name="win_exceeds", cfg=17, H=5, W=7, l=16, b=3, rho=8, T=3, heads=2, D=64,
+                        batch=2, axes=(16, 24, 24)),
+    "rho_exceeds": dict(name="rho_exceeds", cfg=18, H=4, W=4, l=2, b=2, rho=8, T=1, heads=1, D=128, batch=1),
+    "thin": dict(name="thin", cfg=19, H=3, W=130, l=4, b=1, rho=2, T=129, heads=2, D=128, batch=1),
 }
 
 
@@ -101,7 +108,8 @@ def ulp_bf16(x):
     return np.where(a > 0, 2.0 ** (np.maximum(e, -126) - 7), 2.0 ** -133)
 
 
-@pytest.mark.parametrize("name", ["tiny", "1k", "ragged", "odd", "small_l", "text_only_pad"])
+@pytest.mark.parametrize("name", ["tiny", "1k", "ragged", "odd", "small_l", "text_only_pad", "single",
+                                  "win_exceeds", "thin"])
 def test_permute_rope_parity(ug, name):
     wl = _wl(name) if name in ("tiny", "1k", "ragged") else custom(name)
     plan, (q, k, v), lay, _ = run_layer(ug, wl)
@@ -143,7 +151,8 @@ def test_unpermute_inverts_permute_bitwise(ug, name):
 @pytest.mark.parametrize("name,split", [("tiny", None), ("tiny", 0), ("tiny", 2), ("1k", None),
                                         ("1k", 0), ("1k", 5), ("odd", None), ("odd", 3),
                                         ("small_l", None), ("no_lr_text", None), ("win32_rho2", None),
-                                        ("text_only_pad", 1)])
+                                        ("text_only_pad", 1), ("single", None), ("win_exceeds", None),
+                                        ("rho_exceeds", None), ("thin", None), ("thin", 1)])
 def test_attention_full_parity(ug, name, split):
     wl = _wl(name) if name in ("tiny", "1k") else custom(name)
     plan, (q, k, v), lay, o = run_layer(ug, wl, split=split)
@@ -166,11 +175,13 @@ def test_attention_full_parity(ug, name, split):
                            lay.op[b][:, torch.as_tensor(slot, device="cuda")].view(torch.int16))
 
 
-@pytest.mark.parametrize("name,heads", [("4k", (0, 13)), ("ragged", (5,)), ("8k", (23,))])
+@pytest.mark.parametrize("name,heads", [("4k", (0, 13)), ("ragged", (5,)), ("8k", (23,)),
+                                        ("16k", (1,))])
 def test_attention_full_size_sampled(ug, name, heads):
-    """Full-size layers in the configuration the benchmark runs, checked on sampled rows."""
+    """Full-size layers in the configuration the benchmark runs, checked on sampled rows; the
+    16K layer (the largest considered, 1024 x 1024 HR tokens) runs with 2 heads."""
     import torch
-    wl = _wl(name)
+    wl = _wl(name, heads=2) if name == "16k" else _wl(name)
     plan, (q, k, v), lay, o = run_layer(ug, wl)
     assert not torch.isnan(lay.op).any()
     rows = sample_rows(wl)
