@@ -38,15 +38,23 @@ def oracle_rows(q, k, v, wl, b, heads, rows, lr_radius=-1):
     return np.stack(out)
 
 
-def sample_rows(wl, n_text=16, n_lr=32, windows="corners"):
-    """Permuted rows to check at full size: text rows, whole windows (corner, edge, interior,
-    and the last column for ragged grids), LR rows."""
+def sample_rows(wl, n_text=512, n_lr=512, windows="all12"):
+    """Permuted rows checked at full size: all text rows (up to n_text, evenly spaced beyond),
+    every row of 12 windows (the 4 corners, the 4 edge middles, 4 interior windows at the
+    quarter points; at a ragged right edge the corner and edge windows are the partial ones;
+    windows="corners" keeps the corners and the centre), and n_lr evenly spaced LR rows."""
     g = geometry(wl)
     rows = list(np.linspace(0, max(0, g.T - 1), min(n_text, g.T)).astype(int)) if g.T else []
     l2 = g.l * g.l
-    wins = {0, g.nWw - 1, (g.nWh - 1) * g.nWw, g.nWh * g.nWw - 1,
-            (g.nWh // 2) * g.nWw + g.nWw // 2, g.nWw // 2, (g.nWh // 2) * g.nWw}
-    for w in sorted(wins):
+    R, C = g.nWh - 1, g.nWw - 1
+    cells = {(0, 0), (0, C), (R, 0), (R, C)}                     # corners
+    if windows == "all12":
+        cells |= {(0, C // 2), (R, C // 2), (R // 2, 0), (R // 2, C),   # edge middles
+                  (R // 4, C // 4), (R // 4, 3 * C // 4), (3 * R // 4, C // 4), (3 * R // 4, 3 * C // 4)}
+    else:
+        cells |= {(R // 2, C // 2)}
+    for (wr, wc) in sorted(cells):
+        w = wr * g.nWw + wc
         rows += list(range(g.off_hr + w * l2, g.off_hr + (w + 1) * l2))
     if g.N_lr:
         rows += list(np.linspace(g.off_lr, g.off_lr + g.N_lr - 1, min(n_lr, g.N_lr)).astype(int))
