@@ -281,16 +281,16 @@ static int hla_forward_impl(const void* qp, const void* kp, const void* vp, void
   if (st) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 
-  // split workspace, owned by the plan and grown on demand
+  // split workspace, owned by the plan and grown on demand with stream-ordered allocation (no
+  // device-wide synchronisation, and capturable in a CUDA graph)
   const size_t ws_need = ug::split_workspace_bytes(p, batch * p->heads);
   if (ws_need > p->dev.ws_bytes) {
     if (p->dev.ws) {
-      cudaStreamSynchronize(s);
-      cudaFree(p->dev.ws);
+      cudaFreeAsync(p->dev.ws, s);
       p->dev.ws = nullptr;
       p->dev.ws_bytes = 0;
     }
-    if (cudaMalloc(reinterpret_cast<void**>(&p->dev.ws), ws_need) != cudaSuccess) {
+    if (cudaMallocAsync(reinterpret_cast<void**>(&p->dev.ws), ws_need, s) != cudaSuccess) {
       cudaGetLastError();
       p->dev.ws = nullptr;
       return ULTRAGEN_ERR_OOM;

@@ -8,7 +8,6 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
-#include <cmath>
 #include <mutex>
 
 #include "kernels.h"
@@ -18,7 +17,6 @@ namespace {
 
 constexpr size_t kScratchBytes = ULTRAGEN_NOALLOC_SCRATCH_BYTES;
 constexpr int kMaxDevices = 64;
-constexpr unsigned long long kTimeoutNs = 2000ull * 1000 * 1000;
 
 // Split partials of the no-allocation forward.  Every GPU that loads this library holds it
 // until the process exits.  All calls share it and it keeps the last call's contents.
@@ -61,8 +59,8 @@ extern "C" int ultragen_hla_forward_noalloc(const void* qp, const void* kp, cons
   if (rows >= ((int64_t)1 << 31) || items >= ((int64_t)1 << 31)) return ULTRAGEN_ERR_UNSUPPORTED;
 
   // the scratch bound: split partials of every (batch, head)
-  const size_t need = (size_t)batch * p->heads * p->n_split_items * 2 * ug::kTile * (p->D + 1) * sizeof(float);
-  if (need > kScratchBytes) return ULTRAGEN_ERR_UNSUPPORTED;
+  if (ug::split_workspace_bytes(p, (int64_t)batch * p->heads) > kScratchBytes)
+    return ULTRAGEN_ERR_UNSUPPORTED;
 
   // the plan's tables must already be on this device: this call uploads nothing
   int dev = -1, major = 0;
@@ -77,57 +75,11 @@ extern "C" int ultragen_hla_forward_noalloc(const void* qp, const void* kp, cons
   float* scratch = nullptr;
   int st = scratch_for_device(dev, &scratch);
   if (st) return st;
-
-  alignas(64) CUtensorMap tq, tk, tv;
-  if ((st = ug::make_tmap(&tq, qp, rows, p->D)) || (st = ug::make_tmap(&tk, kp, rows, p->D)) ||
-      (st = ug::make_tmap(&tv, vp, rows, p->D)))
-    return st;
-
-  ug::FwdParams f;
-  f.items = p->dev.items;
-  f.entries = p->dev.entries;
-  f.mask_off = p->dev.mask_off;
-  f.mask_pool = p->dev.mask_pool;
-  f.perm = p->dev.perm;
-  f.out = static_cast<__nv_bfloat16*>(op);
-  f.ws = scratch;
-  f.err = p->dev.error;
-  f.n_items_head = (int)p->items.size();
-  f.total_items = (int)items;
-  f.N_tot = (int)p->N_tot;
-  f.off_hr = (int)p->off_hr;
-  f.l2 = p->l * p->l;
-  f.n_ws_head = p->n_split_items;
-  f.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)p->D));
-  f.timeout_ns = kTimeoutNs;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int grid = (int)std::min<int64_t>(items, ug::sm_count());
+  // the same launches as ultragen_hla_forward (tensor maps, attention, split merge): none of
+  // them allocates
   int launches = 0;
-  if (grid > 0) {
-    cudaError_t e = ug::launch_hla_fwd(&tq, &tk, &tv, f, p->D, grid, s);
-    if (e != cudaSuccess) {
-      cudaGetLastError();
-      return ULTRAGEN_ERR_CUDA;
-    }
-    ++launches;
-  }
-  if (!p->combine.empty()) {
-    ug::CombineArgs c;
-    c.ws = scratch;
-    c.out = f.out;
-    c.groups = p->dev.combine;
-    c.perm = p->dev.perm;
-    c.n_groups = (int)p->combine.size();
-    c.n_ws_head = p->n_split_items;
-    c.N_tot = (int)p->N_tot;
-    c.BH = batch * p->heads;
-    cudaError_t e = ug::launch_combine(c, p->D, s);
-    if (e != cudaSuccess) {
-      cudaGetLastError();
-      return ULTRAGEN_ERR_CUDA;
-    }
-    ++launches;
-  }
+  st = ug::launch_attention(p, qp, kp, vp, op, batch * p->heads, p->heads, 0, scratch, stream,
+                            &launches);
   p->last_launches = launches;
-  return ULTRAGEN_OK;
+  return st;
 }

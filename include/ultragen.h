@@ -155,7 +155,9 @@ int ultragen_permute_rope(const void* q, const void* k, const void* v, int in_dt
  *   qp, kp, vp, op  [batch, heads, N_tot, head_dim] BF16 (device); op rows of pad slots = 0
  * bf16 tensor-core products with fp32 accumulation and fp32 online softmax.  Uses the
  * plan's split workspace (device memory the plan allocates and keeps) when the plan
- * splits groups.  Errors: INVALID_ARG, NO_DEVICE, OOM, CUDA.
+ * splits groups; a call that needs more than the plan holds grows it with stream-ordered
+ * allocation on `stream` (cudaFreeAsync / cudaMallocAsync from the device's default pool),
+ * so no call synchronises the device.  Errors: INVALID_ARG, NO_DEVICE, OOM, CUDA.
  */
 int ultragen_hla_forward(const void* qp, const void* kp, const void* vp, void* op,
                          const ultragen_plan_t* plan, int batch, ultragen_stream_t stream);
@@ -209,7 +211,8 @@ int ultragen_hla_forward_noalloc(const void* qp, const void* kp, const void* vp,
 int ultragen_sync_status(const ultragen_plan_t* plan, ultragen_stream_t stream);
 
 /* Diagnostics (no counterpart in the pages).  wait_limit_s (1 ms .. 60 s, default 2 s) bounds
- * every device-side wait of ultragen_hla_forward; past it the kernel stops cleanly and
+ * every device-side wait of the attention kernel (ultragen_hla_forward, _raster, _noalloc and
+ * the host runner); past it the kernel stops cleanly and
  * ultragen_sync_status reports ULTRAGEN_ERR_TIMEOUT.  fault = 1 makes the MMA warp of every
  * CTA withhold one "S ready" signal, so a wait runs out on purpose (tests of that path);
  * fault = 0 is normal operation.  INVALID_ARG outside these ranges. */
