@@ -476,7 +476,6 @@ def main():
     value = job_tflops(flops, world, ms_step)
     pk, src = peaks()
     attn_tflops = flops / (ms_attn * 1e-3) / 1e12
-    peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
     elem = wl.batch * wl.heads * info["N_tot"] * wl.D
     perm_bytes = 3 * (wl.batch * info["N_raster"] * wl.heads * wl.D * (2 if wl.dtype == "bf16" else 4)) + 3 * elem * 2
     unperm_bytes = elem * 2 + wl.batch * info["N_raster"] * wl.heads * wl.D * 2
@@ -513,6 +512,17 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl, q, k, v)
 
+    # roofline denominator: the burst bf16 figure while the SM clock held its maximum during
+    # the timed steps, the sustained (power-capped) one once the power cap throttled it
+    capped = "sw_power_cap" in clocks.get("reasons", []) or (
+        clocks.get("sm_mhz") and clocks.get("sm_max_mhz")
+        and clocks["sm_mhz"] < 0.97 * clocks["sm_max_mhz"])
+    if capped:
+        peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+        peak_note = f"{src} bf16 dense, sustained (the power cap held the SM clock at {clocks.get('sm_mhz')} MHz)"
+    else:
+        peak = pk["bf16_tflops"]
+        peak_note = f"{src} bf16 dense, burst (SM clock at its maximum during the timed steps)"
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "useful TFLOP/s", "n_gpus": world,
@@ -534,7 +544,7 @@ def main():
             "unpermute_gbs": unperm_bytes / (ms_unperm * 1e-3) / 1e9 if args.unfused else None,
             "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
                          "frac": attn_tflops / peak, "traffic": traffic,
-                         "peak_source": f"{src} bf16 dense, sustained (kernel timed inside a repeated step)",
+                         "peak_source": peak_note,
                          "algorithmic_flops_per_launch": flops},
             "e2e": e2e,
             "gpu_launches": launches,
