@@ -48,6 +48,12 @@ Readings taken where the pages are silent or garbled (each is listed in DESIGN.m
   R13 Windows in row-major order; raster order inside a window.
   R15 Pad slots are not tokens: never visible as keys; pad query rows output 0; tile lists
       are derived from the mask rows of real tokens only.
+  R18 Optional compact halo blocks (halo_copy): the K/V layout appends, per window w, a block
+      of G slots (G = the largest halo padded to 128) holding w's halo tokens -- the HR tokens
+      of its grown box outside the window, in raster order of the box.  An HR query of window
+      w then takes the other windows' tokens of its box from w's block instead of their
+      window segments; halo blocks are visible to nothing else.  Every query sees the same
+      tokens as without them, so the attention output is the same function.
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py`` (brute force
 on tiny grids, closed forms, textbook special cases, invariants).  The pages print no
@@ -85,6 +91,7 @@ class Geometry:
     rho: int        # LR down-scale factor, rho = H / h ([UG-note] 关键设计 2); 0 = no LR
     T: int          # text tokens
     lr_radius: int = -1   # -1: HR sees all LR (R3); r >= 0: only the window's region grown by r
+    halo_copy: bool = False   # K/V carry a compact halo block per window (R18)
 
     @property
     def nWh(self) -> int:
@@ -129,6 +136,27 @@ class Geometry:
     @property
     def N_raster(self) -> int:
         return self.T + self.N_hr + self.N_lr
+
+    @property
+    def n_windows(self) -> int:
+        return self.nWh * self.nWw
+
+    @property
+    def G(self) -> int:
+        """Slots of one window's halo block in the K/V layout (R18): the largest halo, padded
+        to a multiple of 128; 0 without halo blocks."""
+        if not self.halo_copy:
+            return 0
+        return pad128(max(len(halo_tokens(self, w)) for w in range(self.n_windows)))
+
+    @property
+    def off_halo(self) -> int:
+        return self.N_tot
+
+    @property
+    def N_kv(self) -> int:
+        """K/V slots: the permuted layout plus one halo block per window (R18)."""
+        return self.N_tot + self.n_windows * self.G
 
 
 # --------------------------------------------------------------------------------------
@@ -224,6 +252,77 @@ def unpermute(xp: np.ndarray, g: Geometry) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------------------
+# Compact halo blocks of K/V (R18)
+# --------------------------------------------------------------------------------------
+
+HALO = 3   # segment of a K/V slot in a window's halo block
+
+
+@functools.lru_cache(maxsize=4096)
+def halo_tokens(g: Geometry, w: int) -> tuple:
+    """Raster indices of window w's halo: the HR tokens of its box grown by b (clipped to the
+    image, R2) that lie outside the window itself, in raster order of the grown box (R18)."""
+    wr, wc = divmod(w, g.nWw)
+    r0, r1 = max(0, wr * g.l - g.b), min(g.H, (wr + 1) * g.l + g.b)
+    c0, c1 = max(0, wc * g.l - g.b), min(g.W, (wc + 1) * g.l + g.b)
+    out = []
+    for i in range(r0, r1):
+        for j in range(c0, c1):
+            if i // g.l == wr and j // g.l == wc:
+                continue
+            out.append(g.T + i * g.W + j)
+    return tuple(out)
+
+
+@functools.lru_cache(maxsize=8)
+def kv_perm_map(g: Geometry) -> np.ndarray:
+    """K/V slot -> raster index (-1 pad): the permuted layout, then window w's halo block at
+    off_halo + w * G holding halo_tokens(w) in order (R18)."""
+    kv = np.full(g.N_kv, -1, np.int64)
+    kv[:g.N_tot] = perm_map(g)
+    if g.halo_copy:
+        for w in range(g.n_windows):
+            toks = halo_tokens(g, w)
+            kv[g.off_halo + w * g.G:g.off_halo + w * g.G + len(toks)] = toks
+    return kv
+
+
+@functools.lru_cache(maxsize=8)
+def kv_slot_info(g: Geometry):
+    """Per K/V slot: segment (HALO for halo-block slots, PAD for pad), the token's coordinates,
+    and the owning window (HR window-segment and halo-block slots; -1 otherwise)."""
+    seg_r, ca_r, cb_r = raster_tokens(g)
+    kv = kv_perm_map(g)
+    real = kv >= 0
+    seg = np.full(g.N_kv, PAD, np.int64)
+    ca = np.zeros(g.N_kv, np.int64)
+    cb = np.zeros(g.N_kv, np.int64)
+    seg[real] = seg_r[kv[real]]
+    ca[real] = ca_r[kv[real]]
+    cb[real] = cb_r[kv[real]]
+    owner = np.full(g.N_kv, -1, np.int64)
+    s = np.arange(g.N_kv)
+    win_seg = (s >= g.off_hr) & (s < g.off_hr + g.N_hrp)
+    owner[win_seg] = (s[win_seg] - g.off_hr) // (g.l * g.l)
+    if g.halo_copy:
+        halo = s >= g.off_halo
+        owner[halo] = (s[halo] - g.off_halo) // g.G
+        seg[halo & real] = HALO
+    return seg, ca, cb, owner
+
+
+def permute_kv(x: np.ndarray, g: Geometry) -> np.ndarray:
+    """Raster [B, N_raster, Hh, D] -> K/V layout [B, Hh, N_kv, D]; pad slots are zero."""
+    B, N, Hh, D = x.shape
+    assert N == g.N_raster
+    kv = kv_perm_map(g)
+    out = np.zeros((B, Hh, g.N_kv, D), x.dtype)
+    real = kv >= 0
+    out[:, :, real, :] = np.transpose(x, (0, 2, 1, 3))[:, :, kv[real], :]
+    return out
+
+
+# --------------------------------------------------------------------------------------
 # Positions and 2D RoPE
 # --------------------------------------------------------------------------------------
 
@@ -283,16 +382,20 @@ def window_box(g: Geometry, i: np.ndarray, j: np.ndarray):
 
 
 def visible_rows(g: Geometry, q_slots: np.ndarray) -> np.ndarray:
-    """Explicit boolean mask rows M[q, :] over all N_tot key slots (R2-R5, R15).
+    """Explicit boolean mask rows M[q, :] over all N_kv key slots (R2-R5, R15, R18).
 
     text q -> text and HR keys;  HR q -> text, LR, and HR keys in its window's halo box;
     LR q -> LR and text keys;  pad q -> nothing.  Pad keys are never visible.
+    With halo blocks (R18) an HR query takes its own window's keys from the window segment and
+    every other key of its halo box from its window's halo block; halo-block keys are visible
+    to nothing else, so every query sees the same tokens as without them.
     """
     seg, ca, cb = slot_info(g)
+    kseg_a, ki_a, kj_a, kown_a = kv_slot_info(g)
     q_slots = np.asarray(q_slots, np.int64)
     qs = seg[q_slots]
-    kseg = seg[None, :]
-    vis = np.zeros((len(q_slots), g.N_tot), bool)
+    kseg = kseg_a[None, :]
+    vis = np.zeros((len(q_slots), g.N_kv), bool)
 
     t = qs == TEXT
     vis[t] = ((kseg == TEXT) | (kseg == HR))[0]
@@ -303,10 +406,14 @@ def visible_rows(g: Geometry, q_slots: np.ndarray) -> np.ndarray:
     hr = np.nonzero(qs == HR)[0]
     if len(hr):
         qi, qj = ca[q_slots[hr]], cb[q_slots[hr]]
-        r0, r1, c0, c1 = window_box(g, qi, qj)
-        ki, kj = ca[None, :], cb[None, :]
-        in_box = ((kseg == HR) & (ki >= r0[:, None]) & (ki < r1[:, None])
-                  & (kj >= c0[:, None]) & (kj < c1[:, None]))
+        ki, kj = ki_a[None, :], kj_a[None, :]
+        if g.halo_copy:
+            qw = (q_slots[hr] - g.off_hr) // (g.l * g.l)
+            in_box = ((kseg == HR) | (kseg == HALO)) & (kown_a[None, :] == qw[:, None])
+        else:
+            r0, r1, c0, c1 = window_box(g, qi, qj)
+            in_box = ((kseg == HR) & (ki >= r0[:, None]) & (ki < r1[:, None])
+                      & (kj >= c0[:, None]) & (kj < c1[:, None]))
         if g.lr_radius < 0:
             lr_vis = kseg == LR
         else:
@@ -330,7 +437,8 @@ def attention_rows(qp: np.ndarray, kp: np.ndarray, vp: np.ndarray, g: Geometry,
                    rows: np.ndarray, heads=None, chunk: int = 256) -> np.ndarray:
     """Dense fp64 masked softmax attention for selected permuted query rows.
 
-    qp, kp, vp: [B, Hh, N_tot, D] (already RoPE'd and permuted).  Returns [B, Hh', len(rows), D]
+    qp: [B, Hh, N_tot, D], kp, vp: [B, Hh, N_kv, D] (already RoPE'd and permuted; N_kv = N_tot
+    without halo blocks).  Returns [B, Hh', len(rows), D]
     with heads' = ``heads`` (all by default).  Pad rows give 0.
     """
     B, Hh, N, D = qp.shape
@@ -371,7 +479,7 @@ def forward(q: np.ndarray, k: np.ndarray, v: np.ndarray, g: Geometry, axes,
     pos = positions(g)
     qr = rope(q, pos, axes, theta)
     kr = rope(k, pos, axes, theta)
-    qp, kp, vp = permute(qr, g), permute(kr, g), permute(np.asarray(v, np.float64), g)
+    qp, kp, vp = permute(qr, g), permute_kv(kr, g), permute_kv(np.asarray(v, np.float64), g)
     rows = np.arange(g.N_tot) if rows is None else np.asarray(rows, np.int64)
     return attention_rows(qp, kp, vp, g, rows, heads=heads), rows
 
@@ -388,8 +496,8 @@ def qtile_entries(g: Geometry, t: int):
     perm = perm_map(g)
     slots = np.arange(t * TILE, (t + 1) * TILE)
     real = perm[slots] >= 0
-    nk = g.N_tot // TILE
-    vis = np.zeros((TILE, g.N_tot), bool)
+    nk = g.N_kv // TILE
+    vis = np.zeros((TILE, g.N_kv), bool)
     if real.any():
         vis[real] = visible_rows(g, slots[real])
     blocks = vis.reshape(TILE, nk, TILE)

@@ -481,3 +481,53 @@ def test_region_radius_covering_the_image_is_all_lr():
     wide = O.Geometry(20, 24, 8, 2, 4, 7, 64)
     rows = np.arange(base.N_tot)
     np.testing.assert_array_equal(O.visible_rows(base, rows), O.visible_rows(wide, rows))
+
+
+# ------------------------------------------------------------------ compact halo blocks (R18)
+HALO_GEOMS = [(32, 32, 8, 2, 4, 16), (37, 29, 12, 5, 3, 70), (20, 18, 4, 3, 5, 9),
+              (5, 7, 16, 3, 8, 3), (24, 24, 8, 8, 2, 4)]
+
+
+@pytest.mark.parametrize("geo", HALO_GEOMS)
+def test_halo_tokens_by_whole_image_scan(geo):
+    """Each window's halo list equals a scan of the whole image in raster order, keeping the
+    tokens within Chebyshev distance b of the window box (per axis) that are not in it."""
+    g = O.Geometry(*geo, halo_copy=True)
+    for w in range(g.n_windows):
+        wr, wc = divmod(w, g.nWw)
+        exp = []
+        for i in range(g.H):
+            for j in range(g.W):
+                di = max(wr * g.l - i, i - ((wr + 1) * g.l - 1), 0)
+                dj = max(wc * g.l - j, j - ((wc + 1) * g.l - 1), 0)
+                if max(di, dj) == 0:
+                    continue            # inside the window itself
+                if di <= g.b and dj <= g.b:
+                    exp.append(g.T + i * g.W + j)
+        assert list(O.halo_tokens(g, w)) == exp
+    assert g.G % 128 == 0 and g.G >= max(len(O.halo_tokens(g, w)) for w in range(g.n_windows))
+
+
+@pytest.mark.parametrize("geo", HALO_GEOMS)
+def test_halo_blocks_leave_every_query_seeing_the_same_tokens(geo):
+    g0, g1 = O.Geometry(*geo), O.Geometry(*geo, halo_copy=True)
+    rows = np.arange(g0.N_tot)
+    v0, v1 = O.visible_rows(g0, rows), O.visible_rows(g1, rows)
+    kv0, kv1 = O.kv_perm_map(g0), O.kv_perm_map(g1)
+    for r in range(len(rows)):
+        t0 = np.sort(kv0[np.nonzero(v0[r])[0]])
+        t1 = np.sort(kv1[np.nonzero(v1[r])[0]])
+        np.testing.assert_array_equal(t0, t1)      # same tokens, none twice
+    assert (kv1 >= 0).sum() == (kv0 >= 0).sum() + sum(len(O.halo_tokens(g1, w)) for w in range(g1.n_windows))
+
+
+@pytest.mark.parametrize("geo,lr_radius", [((32, 32, 8, 2, 4, 16), -1), ((20, 18, 4, 3, 5, 9), 2),
+                                           ((37, 29, 12, 5, 3, 70), -1)])
+def test_halo_blocks_give_the_same_attention(geo, lr_radius):
+    rng = np.random.default_rng(7)
+    g0 = O.Geometry(*geo, lr_radius=lr_radius)
+    g1 = O.Geometry(*geo, lr_radius=lr_radius, halo_copy=True)
+    q, k, v = (rng.standard_normal((1, g0.N_raster, 2, 64)) for _ in range(3))
+    o0, _ = O.forward(q, k, v, g0, (16, 24, 24))
+    o1, _ = O.forward(q, k, v, g1, (16, 24, 24))
+    np.testing.assert_allclose(o1, o0, rtol=0, atol=1e-12)
