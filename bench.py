@@ -49,6 +49,8 @@ def parse():
                     help="override the workload's head count (smaller profiling captures)")
     ap.add_argument("--lr-radius", type=int, default=-1,
                     help="HR->LR scope: -1 all LR tokens (default); r >= 0 the window's anchors grown by r")
+    ap.add_argument("--halo", type=int, default=-1, choices=[-1, 0, 1],
+                    help="compact halo blocks in the K/V layout: -1 automatic (default), 0 off, 1 on")
     ap.add_argument("--impl", default="ultragen", choices=["ultragen", "reference"])
     ap.add_argument("--unfused", action="store_true",
                     help="run unpermute as its own pass instead of in the attention epilogue")
@@ -413,6 +415,8 @@ def main():
     plan = ug.plan_for(wl)
     if args.lr_radius != -1:
         plan.set_lr_scope(args.lr_radius)
+    if args.halo != -1:
+        plan.set_halo(args.halo)
     info = plan.info
     q, k, v = ug.make_qkv(wl)
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
@@ -477,7 +481,11 @@ def main():
     pk, src = peaks()
     attn_tflops = flops / (ms_attn * 1e-3) / 1e12
     elem = wl.batch * wl.heads * info["N_tot"] * wl.D
-    perm_bytes = 3 * (wl.batch * info["N_raster"] * wl.heads * wl.D * (2 if wl.dtype == "bf16" else 4)) + 3 * elem * 2
+    kv_elem = wl.batch * wl.heads * info["N_kv"] * wl.D
+    in_size = 2 if wl.dtype == "bf16" else 4
+    # permute_rope: every raster row of Q, K, V read once (halo copies are written from the
+    # same read), Q written over N_tot slots and K, V over N_kv slots (pad slots as zeros)
+    perm_bytes = 3 * wl.batch * info["N_raster"] * wl.heads * wl.D * in_size + (elem + 2 * kv_elem) * 2
     unperm_bytes = elem * 2 + wl.batch * info["N_raster"] * wl.heads * wl.D * 2
     traffic = profiled_traffic(wl.name)
 
@@ -513,10 +521,9 @@ def main():
         cpu = cpu_baseline(wl, q, k, v)
 
     # roofline denominator: the burst bf16 figure while the SM clock held its maximum during
-    # the timed steps, the sustained (power-capped) one once the power cap throttled it
-    capped = "sw_power_cap" in clocks.get("reasons", []) or (
-        clocks.get("sm_mhz") and clocks.get("sm_max_mhz")
-        and clocks["sm_mhz"] < 0.97 * clocks["sm_max_mhz"])
+    # the timed steps, the sustained (power-capped) one once the clock dropped under the cap
+    capped = bool(clocks.get("sm_mhz") and clocks.get("sm_max_mhz")
+                  and clocks["sm_mhz"] < 0.97 * clocks["sm_max_mhz"])
     if capped:
         peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
         peak_note = f"{src} bf16 dense, sustained (the power cap held the SM clock at {clocks.get('sm_mhz')} MHz)"
@@ -533,7 +540,9 @@ def main():
                        "H": wl.H, "W": wl.W, "l": wl.l, "b": wl.b,
                        "rho": wl.rho, "text_len": wl.T, "lr_radius": args.lr_radius, "heads": wl.heads, "head_dim": wl.D,
                        "batch": wl.batch, "N_tot": info["N_tot"], "useful_pairs_per_head": info["useful_pairs"],
-                       "l2": "inputs larger than L2 (Q, K, V permuted: 3 x %.0f MB); no flush" % (elem * 2 / 1e6),
+                       "halo_blocks": bool(info["halo_copy"]), "N_kv": info["N_kv"],
+                       "l2": "inputs larger than L2 (permuted Q %.0f MB, K and V %.0f MB each); no flush"
+                             % (elem * 2 / 1e6, kv_elem * 2 / 1e6),
                        "parallelism": f"independent layer per rank x{world}"},
             "ms_per_kernel": {"permute_rope": ms_perm, "hla_forward": ms_attn,
                               "unpermute": ms_unperm if args.unfused else "in hla_forward's epilogue"},

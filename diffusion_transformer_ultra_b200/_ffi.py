@@ -31,7 +31,7 @@ SYMBOLS = (
     "ultragen_hla_forward_noalloc", "ultragen_plan_set_diagnostics", "ultragen_plan_set_lr_scope",
     "ultragen_hla_forward_raster", "ultragen_warm_start", "ultragen_host_runner_create",
     "ultragen_host_runner_forward", "ultragen_host_runner_last_launch_count",
-    "ultragen_host_runner_destroy",
+    "ultragen_host_runner_destroy", "ultragen_plan_set_halo", "ultragen_plan_export_kv",
 )
 
 
@@ -47,7 +47,9 @@ class PlanInfo(ctypes.Structure):
         ("rope_axes", ctypes.c_int32 * 3), ("rope_theta", ctypes.c_double),
         ("split_chunk", ctypes.c_int32), ("n_split_groups", ctypes.c_int32),
         ("n_split_items", ctypes.c_int32), ("workspace_bytes_per_head", ctypes.c_int64),
-        ("lr_radius", ctypes.c_int32),
+        ("lr_radius", ctypes.c_int32), ("halo_copy", ctypes.c_int32),
+        ("halo_slots_per_window", ctypes.c_int32), ("N_kv", ctypes.c_int64),
+        ("off_halo", ctypes.c_int64),
     ]
 
     def as_dict(self):
@@ -81,6 +83,8 @@ def lib() -> ctypes.CDLL:
     L.ultragen_plan_set_rope.argtypes = [vp, cint, cint, cint, ctypes.c_double]
     L.ultragen_plan_set_split.argtypes = [vp, cint]
     L.ultragen_plan_set_lr_scope.argtypes = [vp, cint]
+    L.ultragen_plan_set_halo.argtypes = [vp, cint]
+    L.ultragen_plan_export_kv.argtypes = [vp, vp]
     L.ultragen_plan_info.argtypes = [vp, ctypes.POINTER(PlanInfo)]
     L.ultragen_plan_export.argtypes = [vp, vp, vp, vp]
     L.ultragen_plan_export_rowmasks.argtypes = [vp, cint, vp]
@@ -140,6 +144,16 @@ class Plan:
     def set_lr_scope(self, radius: int):
         _check("ultragen_plan_set_lr_scope", lib().ultragen_plan_set_lr_scope(self._h, int(radius)))
         self._refresh()
+
+    def set_halo(self, mode: int):
+        """Compact halo blocks in the K/V layout: 1 on, 0 off, -1 automatic (the default)."""
+        _check("ultragen_plan_set_halo", lib().ultragen_plan_set_halo(self._h, int(mode)))
+        self._refresh()
+
+    def export_kv(self):
+        kv = np.empty(self.info["N_kv"], np.int32)
+        _check("ultragen_plan_export_kv", lib().ultragen_plan_export_kv(self._h, kv.ctypes.data))
+        return kv
 
     def export(self):
         i = self.info
@@ -203,13 +217,15 @@ def permute_rope(q, k, v, qp, kp, vp, plan: Plan, stream=None):
     i = plan.info
     B = q.shape[0]
     raster = (B, i["N_raster"], i["heads"], i["head_dim"])
-    perm_shape = (B, i["heads"], i["N_tot"], i["head_dim"])
+    q_shape = (B, i["heads"], i["N_tot"], i["head_dim"])
+    kv_shape = (B, i["heads"], i["N_kv"], i["head_dim"])
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, raster, (torch.bfloat16, torch.float32), n)
     if not (q.dtype == k.dtype == v.dtype):
         raise ValueError("q, k, v must share a dtype")
-    for t, n in ((qp, "qp"), (kp, "kp"), (vp, "vp")):
-        _need(t, perm_shape, (torch.bfloat16,), n)
+    _need(qp, q_shape, (torch.bfloat16,), "qp")
+    for t, n in ((kp, "kp"), (vp, "vp")):
+        _need(t, kv_shape, (torch.bfloat16,), n)
     dt = BF16 if q.dtype == torch.bfloat16 else F32
     _check("ultragen_permute_rope", lib().ultragen_permute_rope(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), dt, qp.data_ptr(), kp.data_ptr(), vp.data_ptr(),
@@ -222,8 +238,11 @@ def hla_forward(qp, kp, vp, op, plan: Plan, stream=None):
     i = plan.info
     B = qp.shape[0]
     shape = (B, i["heads"], i["N_tot"], i["head_dim"])
-    for t, n in ((qp, "qp"), (kp, "kp"), (vp, "vp"), (op, "op")):
+    kv_shape = (B, i["heads"], i["N_kv"], i["head_dim"])
+    for t, n in ((qp, "qp"), (op, "op")):
         _need(t, shape, (torch.bfloat16,), n)
+    for t, n in ((kp, "kp"), (vp, "vp")):
+        _need(t, kv_shape, (torch.bfloat16,), n)
     _check("ultragen_hla_forward", lib().ultragen_hla_forward(
         qp.data_ptr(), kp.data_ptr(), vp.data_ptr(), op.data_ptr(), plan.handle, B,
         _stream_ptr(stream)))
@@ -234,9 +253,9 @@ def hla_forward_raster(qp, kp, vp, o, plan: Plan, stream=None):
     import torch
     i = plan.info
     B = qp.shape[0]
-    shape = (B, i["heads"], i["N_tot"], i["head_dim"])
-    for t, n in ((qp, "qp"), (kp, "kp"), (vp, "vp")):
-        _need(t, shape, (torch.bfloat16,), n)
+    _need(qp, (B, i["heads"], i["N_tot"], i["head_dim"]), (torch.bfloat16,), "qp")
+    for t, n in ((kp, "kp"), (vp, "vp")):
+        _need(t, (B, i["heads"], i["N_kv"], i["head_dim"]), (torch.bfloat16,), n)
     _need(o, (B, i["N_raster"], i["heads"], i["head_dim"]), (torch.bfloat16,), "o")
     _check("ultragen_hla_forward_raster", lib().ultragen_hla_forward_raster(
         qp.data_ptr(), kp.data_ptr(), vp.data_ptr(), o.data_ptr(), plan.handle, B,
@@ -251,8 +270,11 @@ def hla_forward_noalloc(qp, kp, vp, op, plan: Plan, stream=None):
     i = plan.info
     B = qp.shape[0]
     shape = (B, i["heads"], i["N_tot"], i["head_dim"])
-    for t, n in ((qp, "qp"), (kp, "kp"), (vp, "vp"), (op, "op")):
+    kv_shape = (B, i["heads"], i["N_kv"], i["head_dim"])
+    for t, n in ((qp, "qp"), (op, "op")):
         _need(t, shape, (torch.bfloat16,), n)
+    for t, n in ((kp, "kp"), (vp, "vp")):
+        _need(t, kv_shape, (torch.bfloat16,), n)
     _check("ultragen_hla_forward_noalloc", lib().ultragen_hla_forward_noalloc(
         qp.data_ptr(), kp.data_ptr(), vp.data_ptr(), op.data_ptr(), plan.handle, B,
         _stream_ptr(stream)))
@@ -339,8 +361,9 @@ class Layer:
         i = plan.info
         self.plan = plan
         shape = (batch, i["heads"], i["N_tot"], i["head_dim"])
-        self.qp, self.kp, self.vp, self.op = (torch.empty(shape, dtype=torch.bfloat16, device=device)
-                                              for _ in range(4))
+        kv_shape = (batch, i["heads"], i["N_kv"], i["head_dim"])
+        self.qp, self.op = (torch.empty(shape, dtype=torch.bfloat16, device=device) for _ in range(2))
+        self.kp, self.vp = (torch.empty(kv_shape, dtype=torch.bfloat16, device=device) for _ in range(2))
 
     def __call__(self, q, k, v, o, stream=None, fused=None):
         """o: raster [B, N_raster, H, D].  With a bf16 o the unpermute runs inside the

@@ -30,7 +30,7 @@ int upload(T** dst, const std::vector<T>& src) {
 void free_device(ultragen_plan_t* p) {
   DeviceTables& d = p->dev;
   void* ptrs[] = {d.items, d.entries, d.mask_off, d.mask_pool, d.perm, d.inv_perm,
-                  d.slot_pos, d.rope, d.combine, d.error, d.ws};
+                  d.slot_pos, d.halo_ptr, d.halo_dst, d.rope, d.combine, d.error, d.ws};
   for (void* q : ptrs)
     if (q) cudaFree(q);
   d = DeviceTables();
@@ -74,7 +74,8 @@ int ensure_device(ultragen_plan_t* p) {
   if ((st = upload(&d.items, items)) || (st = upload(&d.entries, p->entries)) ||
       (st = upload(&d.mask_off, p->mask_off)) || (st = upload(&d.mask_pool, p->mask_pool)) ||
       (st = upload(&d.perm, p->perm)) || (st = upload(&d.inv_perm, p->inv_perm)) ||
-      (st = upload(&d.slot_pos, p->slot_pos)) || (st = upload(&d.rope, rope)) ||
+      (st = upload(&d.slot_pos, p->slot_pos)) || (st = upload(&d.halo_ptr, p->halo_ptr)) ||
+      (st = upload(&d.halo_dst, p->halo_dst)) || (st = upload(&d.rope, rope)) ||
       (st = upload(&d.combine, comb)) || (st = upload(&d.error, std::vector<int>(1, 0)))) {
     free_device(p);
     return st;
@@ -153,12 +154,12 @@ size_t split_workspace_bytes(const ultragen_plan_t* p, int64_t units) {
 int launch_attention(const ultragen_plan_t* p, const void* qp, const void* kp, const void* vp,
                      void* op, int units, int heads, int raster, float* ws, cudaStream_t s,
                      int* launches) {
-  const int64_t rows = (int64_t)units * p->N_tot;
+  const int64_t rows = (int64_t)units * p->N_tot, kv_rows = (int64_t)units * p->N_kv;
   const int64_t items = (int64_t)units * (int64_t)p->items.size();
   alignas(64) CUtensorMap tq, tk, tv;
   int st;
-  if ((st = make_tmap(&tq, qp, rows, p->D)) || (st = make_tmap(&tk, kp, rows, p->D)) ||
-      (st = make_tmap(&tv, vp, rows, p->D)))
+  if ((st = make_tmap(&tq, qp, rows, p->D)) || (st = make_tmap(&tk, kp, kv_rows, p->D)) ||
+      (st = make_tmap(&tv, vp, kv_rows, p->D)))
     return st;
   FwdParams f;
   f.items = p->dev.items;
@@ -172,6 +173,7 @@ int launch_attention(const ultragen_plan_t* p, const void* qp, const void* kp, c
   f.n_items_head = (int)p->items.size();
   f.total_items = (int)items;
   f.N_tot = (int)p->N_tot;
+  f.N_kv = (int)p->N_kv;
   f.off_hr = (int)p->off_hr;
   f.l2 = p->l * p->l;
   f.n_ws_head = p->n_split_items;
@@ -221,14 +223,19 @@ int launch_permute(const ultragen_plan_t* p, const void* q, const void* k, const
   a.perm = p->dev.perm;
   a.slot_pos = p->dev.slot_pos;
   a.rope = p->dev.rope;
-  a.rows_total = (int64_t)batch * heads * p->N_tot;
+  a.rows_total = (int64_t)batch * heads * p->N_kv;
   a.N_tot = (int)p->N_tot;
+  a.N_kv = (int)p->N_kv;
   a.N_raster = (int)p->N_raster;
   a.heads = heads;
   a.div_heads = FastDiv((uint32_t)heads);
-  a.div_ntot = FastDiv((uint32_t)p->N_tot);
+  a.div_nkv = FastDiv((uint32_t)p->N_kv);
   a.pair_a0 = p->axes[0] / 2;
   a.pair_a01 = (p->axes[0] + p->axes[1]) / 2;
+  a.halo_ptr = p->halo_copy ? p->dev.halo_ptr : nullptr;
+  a.halo_dst = p->dev.halo_dst;
+  a.off_hr = (int)p->off_hr;
+  a.N_hrp = (int)p->N_hrp;
   const int rows_per_block = 256 / (p->D / 8);
   return cuda_status(launch_permute_rope(a, in_dtype, p->D, grid_for(a.rows_total, rows_per_block), s));
 }
@@ -255,7 +262,7 @@ int ultragen_permute_rope(const void* q, const void* k, const void* v, int in_dt
   const void* ptrs[] = {q, k, v, qp, kp, vp};
   for (const void* x : ptrs)
     if (!aligned16(x)) return ULTRAGEN_ERR_INVALID_ARG;
-  if ((int64_t)batch * p->heads * p->N_tot >= ((int64_t)1 << 31) ||
+  if ((int64_t)batch * p->heads * p->N_kv >= ((int64_t)1 << 31) ||
       (int64_t)batch * p->heads * p->N_raster >= ((int64_t)1 << 31))
     return ULTRAGEN_ERR_UNSUPPORTED;
   int st = ensure_device(p);
@@ -274,7 +281,7 @@ static int hla_forward_impl(const void* qp, const void* kp, const void* vp, void
   const void* ptrs[] = {qp, kp, vp, op};
   for (const void* x : ptrs)
     if (!aligned16(x)) return ULTRAGEN_ERR_INVALID_ARG;
-  const int64_t rows = (int64_t)batch * p->heads * p->N_tot;
+  const int64_t rows = (int64_t)batch * p->heads * p->N_kv;
   const int64_t items = (int64_t)batch * p->heads * (int64_t)p->items.size();
   if (rows >= ((int64_t)1 << 31) || items >= ((int64_t)1 << 31)) return ULTRAGEN_ERR_UNSUPPORTED;
   int st = ensure_device(p);

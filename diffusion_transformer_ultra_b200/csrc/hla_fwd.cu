@@ -128,7 +128,7 @@ __device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
     }
     ++qi;
     for (int e = e0; e < e1 && ok; ++e) {
-      const int y = bh * p.N_tot + (__ldg(p.entries + e) & 0x7fffffff) * 128;
+      const int y = bh * p.N_kv + (__ldg(p.entries + e) & 0x7fffffff) * 128;
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
         const uint32_t s = ld % C::NS, ph = (ld / C::NS) & 1;

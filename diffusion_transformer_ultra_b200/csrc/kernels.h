@@ -27,13 +27,19 @@ struct FastDiv {
 
 struct PermuteArgs {
   const void* in[3];               // q, k, v raster [B, N_raster, heads, D]
-  __nv_bfloat16* out[3];           // qp, kp, vp window-first [B, heads, N_tot, D]
-  const int32_t* perm;             // slot -> raster, -1 pad
-  const uint32_t* slot_pos;        // (row_pos << 16) | col_pos
+  __nv_bfloat16* out[3];           // qp [B, heads, N_tot, D]; kp, vp [B, heads, N_kv, D]
+  const int32_t* perm;             // K/V slot -> raster, -1 pad (first N_tot: the Q slots)
+  const uint32_t* slot_pos;        // (row_pos << 16) | col_pos per K/V slot
   const float* rope;               // [max(H,W)][D/2][2] (cos, sin)
-  int64_t rows_total;              // B * heads * N_tot
-  int N_tot, N_raster, heads;
-  FastDiv div_heads, div_ntot;
+  int64_t rows_total;              // B * heads * N_kv
+  int N_tot, N_kv, N_raster, heads;
+  FastDiv div_heads, div_nkv;
+  // halo blocks (null when the plan has none): the halo-block copies of window-segment slot
+  // off_hr + k are halo_dst[halo_ptr[k] .. halo_ptr[k+1]); the kernel writes them from the same
+  // read, and writes only the pad slots of the halo region itself
+  const int32_t* halo_ptr;
+  const int32_t* halo_dst;
+  int off_hr, N_hrp;
   int pair_a0, pair_a01;           // pairs [0,a0) axis 0, [a0,a01) axis 1, rest axis 2
 };
 
@@ -67,7 +73,8 @@ struct FwdParams {
   int* err;                        // device error word
   int n_items_head;
   int total_items;
-  int N_tot;
+  int N_tot;                       // Q / O rows per (batch, head)
+  int N_kv;                        // K / V rows per (batch, head)
   int off_hr;
   int l2;                          // l * l
   int n_ws_head;

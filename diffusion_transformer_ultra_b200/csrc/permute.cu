@@ -63,20 +63,24 @@ __global__ void __launch_bounds__(256) permute_rope_kernel(PermuteArgs a) {
   for (int row0 = blockIdx.x * ROWS * U; row0 < rows_total; row0 += step) {
     float xq[U][8], xk[U][8], xv[U][8];
     int pos_r[U], pos_c[U];
-    int dst[U];                                       // output row, -1 when out of range
+    int dst[U];                                       // K/V output row, -1 when out of range
+    int dq[U];                                        // Q output row, -1 for halo-block slots
     bool real[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int row = row0 + u * ROWS + rsub;         // (b, slot, h)
+      const int row = row0 + u * ROWS + rsub;         // (b, K/V slot, h)
       dst[u] = -1;
+      dq[u] = -1;
       real[u] = false;
       if (row >= rows_total) continue;
       const int bs = (int)a.div_heads.div((uint32_t)row);
       const int h = row - bs * a.heads;
-      const int b = (int)a.div_ntot.div((uint32_t)bs);
-      const int slot = bs - b * a.N_tot;
-      dst[u] = (b * a.heads + h) * a.N_tot + slot;
+      const int b = (int)a.div_nkv.div((uint32_t)bs);
+      const int slot = bs - b * a.N_kv;
       const int r = __ldg(a.perm + slot);
+      if (slot >= a.N_tot && r >= 0) continue;          // a halo copy: written with its source
+      dst[u] = (b * a.heads + h) * a.N_kv + slot;
+      if (slot < a.N_tot) dq[u] = (b * a.heads + h) * a.N_tot + slot;
       if (r < 0) continue;
       real[u] = true;
       const uint32_t sp = __ldg(a.slot_pos + slot);
@@ -114,9 +118,23 @@ __global__ void __launch_bounds__(256) permute_rope_kernel(PermuteArgs a) {
                         pack_bf16(xv[u][4], xv[u][5]), pack_bf16(xv[u][6], xv[u][7]));
       }
       const int64_t o = (int64_t)dst[u] * D + c * 8;
-      *reinterpret_cast<uint4*>(a.out[0] + o) = oq;
+      if (dq[u] >= 0) *reinterpret_cast<uint4*>(a.out[0] + (int64_t)dq[u] * D + c * 8) = oq;
       *reinterpret_cast<uint4*>(a.out[1] + o) = ok;
       *reinterpret_cast<uint4*>(a.out[2] + o) = ov;
+      if (a.halo_ptr && real[u]) {
+        // copies into the halo blocks of the neighbouring windows
+        const int slot = dst[u] - (dst[u] / a.N_kv) * a.N_kv;
+        const int k = slot - a.off_hr;
+        if (k >= 0 && k < a.N_hrp) {
+          const int base = dst[u] - slot;
+          const int e1 = __ldg(a.halo_ptr + k + 1);
+          for (int e = __ldg(a.halo_ptr + k); e < e1; ++e) {
+            const int64_t oh = (int64_t)(base + __ldg(a.halo_dst + e)) * D + c * 8;
+            *reinterpret_cast<uint4*>(a.out[1] + oh) = ok;
+            *reinterpret_cast<uint4*>(a.out[2] + oh) = ov;
+          }
+        }
+      }
     }
   }
 }

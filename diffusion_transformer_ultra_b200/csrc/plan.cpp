@@ -30,6 +30,7 @@ struct ClassDesc {
   int kind;              // SEG_TEXT, SEG_HR, SEG_LR
   int r0, r1, c0, c1;    // HR halo box [r0, r1) x [c0, c1)
   int lr0, lr1, lc0, lc1;  // scaled LR positions visible to the window (lr_radius >= 0)
+  int wid;               // the window (HR classes)
 };
 
 inline bool visible(const ultragen_plan_t* p, const ClassDesc& c, int64_t s) {
@@ -46,6 +47,8 @@ inline bool visible(const ultragen_plan_t* p, const ClassDesc& c, int64_t s) {
         const int pm = p->rho * p->ci[s], pn = p->rho * p->cj[s];
         return pm >= c.lr0 && pm < c.lr1 && pn >= c.lc0 && pn < c.lc1;
       }
+      // with halo blocks, the window's own segment and its own halo block (R18)
+      if (p->halo_copy) return (sg == SEG_HR || sg == SEG_HALO) && p->owner[s] == c.wid;
       if (sg != SEG_HR) return false;
       return p->ci[s] >= c.r0 && p->ci[s] < c.r1 && p->cj[s] >= c.c0 && p->cj[s] < c.c1;
   }
@@ -55,6 +58,7 @@ ClassDesc window_class(const ultragen_plan_t* p, int wid) {
   const int wr = wid / p->nWw, wc = wid % p->nWw;
   ClassDesc c;
   c.kind = SEG_HR;
+  c.wid = wid;
   c.r0 = std::max(0, wr * p->l - p->b);
   c.r1 = std::min(p->H, (wr + 1) * p->l + p->b);
   c.c0 = std::max(0, wc * p->l - p->b);
@@ -72,9 +76,62 @@ void add_range(std::vector<int>& v, int64_t s_begin, int64_t s_end) {
   for (int64_t t = s_begin / kTile; t <= (s_end - 1) / kTile; ++t) v.push_back((int)t);
 }
 
+// Window w's halo (R18): the HR tokens of its grown box outside the window, raster order.
+template <typename F>
+void for_each_halo_token(const ultragen_plan_t* p, int w, F&& f) {
+  const int wr = w / p->nWw, wc = w % p->nWw;
+  const int r0 = std::max(0, wr * p->l - p->b), r1 = std::min(p->H, (wr + 1) * p->l + p->b);
+  const int c0 = std::max(0, wc * p->l - p->b), c1 = std::min(p->W, (wc + 1) * p->l + p->b);
+  for (int i = r0; i < r1; ++i)
+    for (int j = c0; j < c1; ++j)
+      if (i / p->l != wr || j / p->l != wc) f(i, j);
+}
+
+int build_tables_mode(ultragen_plan_t* p, int halo);
+
 }  // namespace
 
+// Builds the tables with compact halo blocks on or off; "auto" takes them when the tile-list
+// entries they save (one entry = one 128 x 128 tile step of one query tile) outweigh the extra
+// permute traffic of the copies (about 3.3 entries per copied 128-row K/V tile: written once
+// and read again by the attention).
 int build_tables(ultragen_plan_t* p) {
+  if (p->halo_req == 0 || p->b == 0) return build_tables_mode(p, 0);
+  if (p->halo_req == 1) return build_tables_mode(p, 1);
+  int st = build_tables_mode(p, 0);
+  if (st) return st;
+  // entries the halo blocks would replace: each HR query tile's neighbour-window tiles give way
+  // to its windows' halo tiles
+  const int64_t l2 = (int64_t)p->l * p->l;
+  std::vector<int> halo_tiles(p->nWh * p->nWw);
+  int64_t g_max = 0;
+  for (int w = 0; w < p->nWh * p->nWw; ++w) {
+    int64_t n = 0;
+    for_each_halo_token(p, w, [&](int, int) { ++n; });
+    halo_tiles[w] = (int)((n + kTile - 1) / kTile);
+    g_max = std::max(g_max, n);
+  }
+  const int64_t G = (g_max + kTile - 1) / kTile * kTile;
+  int64_t saved = 0;
+  for (int t = (int)(p->off_hr / kTile); t < (int)(p->off_lr / kTile); ++t) {
+    if (p->qt_wfirst[t] < 0) continue;
+    const int wf = p->qt_wfirst[t], C = p->qt_classes[t];
+    for (int e = p->row_ptr[t]; e < p->row_ptr[t + 1]; ++e) {
+      const int64_t k0 = (int64_t)(p->entries[e] & 0x7fffffff) * kTile;
+      if (k0 < p->off_hr || k0 >= p->off_lr) continue;
+      const int64_t kw = (k0 - p->off_hr) / l2;
+      if (kw < wf || kw >= wf + C) ++saved;                    // another window's tile
+    }
+    for (int c = 0; c < C; ++c) saved -= halo_tiles[wf + c];
+  }
+  const double copy_tiles = (double)p->nWh * p->nWw * (G / kTile);
+  if ((double)saved > 3.3 * copy_tiles) return build_tables_mode(p, 1);
+  return ULTRAGEN_OK;
+}
+
+namespace {
+
+int build_tables_mode(ultragen_plan_t* p, int halo) {
   p->nWh = cdiv(p->H, p->l);
   p->nWw = cdiv(p->W, p->l);
   p->h = p->rho > 0 ? cdiv(p->H, p->rho) : 0;
@@ -88,13 +145,29 @@ int build_tables(ultragen_plan_t* p) {
   p->N_raster = p->T + p->N_hr + p->N_lr;
   if (p->N_tot > (int64_t)1 << 30) return ULTRAGEN_ERR_UNSUPPORTED;
   p->n_qtiles = (int)(p->N_tot / kTile);
+  const int nW = p->nWh * p->nWw;
+  p->halo_copy = halo;
+  p->G = 0;
+  if (halo) {
+    int64_t g_max = 0;
+    for (int w = 0; w < nW; ++w) {
+      int64_t n = 0;
+      for_each_halo_token(p, w, [&](int, int) { ++n; });
+      g_max = std::max(g_max, n);
+    }
+    p->G = (g_max + kTile - 1) / kTile * kTile;
+  }
+  p->off_halo = p->N_tot;
+  p->N_kv = p->N_tot + (int64_t)nW * p->G;
+  if (p->N_kv > (int64_t)1 << 30) return ULTRAGEN_ERR_UNSUPPORTED;
 
-  const int64_t N = p->N_tot;
+  const int64_t N = p->N_kv;
   p->perm.assign(N, -1);
   p->inv_perm.assign(p->N_raster, -1);
   p->seg.assign(N, SEG_PAD);
   p->ci.assign(N, 0);
   p->cj.assign(N, 0);
+  p->owner.assign(N, -1);
   p->slot_pos.assign(N, 0u);
 
   // window-first permutation ([UG-note] 关键设计 1)
@@ -115,7 +188,41 @@ int build_tables(ultragen_plan_t* p) {
       p->seg[s] = SEG_HR;
       p->ci[s] = i;
       p->cj[s] = j;
+      p->owner[s] = (int32_t)win;
       p->slot_pos[s] = ((uint32_t)i << 16) | (uint32_t)j;
+    }
+  }
+  // compact halo blocks of K/V (R18): window w's halo tokens at off_halo + w * G, and for the
+  // permute, each window-segment slot's list of halo-block copies (CSR)
+  p->halo_ptr.clear();
+  p->halo_dst.clear();
+  if (halo) {
+    std::vector<int32_t> count(p->N_hrp + 1, 0);
+    for (int w = 0; w < nW; ++w) {
+      int64_t s = p->off_halo + (int64_t)w * p->G;
+      for_each_halo_token(p, w, [&](int i, int j) {
+        const int64_t r = p->T + (int64_t)i * p->W + j;
+        p->perm[s] = (int32_t)r;
+        p->seg[s] = SEG_HALO;
+        p->ci[s] = i;
+        p->cj[s] = j;
+        p->owner[s] = w;
+        p->slot_pos[s] = ((uint32_t)i << 16) | (uint32_t)j;
+        ++count[p->inv_perm[r] - p->off_hr + 1];
+        ++s;
+      });
+    }
+    for (int64_t k = 0; k < p->N_hrp; ++k) count[k + 1] += count[k];
+    p->halo_ptr = count;
+    p->halo_dst.assign(count[p->N_hrp], -1);
+    std::vector<int32_t> fill(count.begin(), count.end() - 1);
+    for (int w = 0; w < nW; ++w) {
+      int64_t s = p->off_halo + (int64_t)w * p->G;
+      for_each_halo_token(p, w, [&](int i, int j) {
+        const int64_t r = p->T + (int64_t)i * p->W + j;
+        p->halo_dst[fill[p->inv_perm[r] - p->off_hr]++] = (int32_t)s;
+        ++s;
+      });
     }
   }
   // LR tokens at positions (rho m, rho n) ([UG-note] 关键设计 2)
@@ -160,7 +267,7 @@ int build_tables(ultragen_plan_t* p) {
       const int wlast = (int)((std::min<int64_t>(s0 + kTile, hr_end) - 1 - p->off_hr) / l2);
       for (int wid = wfirst; wid <= wlast; ++wid) classes.push_back(window_class(p, wid));
     } else {
-      ClassDesc c{kind, 0, 0, 0, 0, 0, 0, 0, 0};
+      ClassDesc c{kind, 0, 0, 0, 0, 0, 0, 0, 0, -1};
       classes.push_back(c);
       if (kind == SEG_HR) wfirst = -1;   // pad-only tile between HR and LR segments
     }
@@ -205,6 +312,13 @@ int build_tables(ultragen_plan_t* p) {
       for (int c = 0; c < C; ++c) {
         if (class_real[c] == 0) continue;
         const ClassDesc& cd = classes[c];
+        if (p->halo_copy) {   // the window itself and its halo block (R18)
+          const int64_t ws = p->off_hr + (int64_t)cd.wid * l2;
+          add_range(cand, ws, ws + l2);
+          const int64_t hb = p->off_halo + (int64_t)cd.wid * p->G;
+          add_range(cand, hb, hb + p->G);
+          continue;
+        }
         if (cd.r1 <= cd.r0 || cd.c1 <= cd.c0) continue;
         for (int wr = cd.r0 / p->l; wr <= (cd.r1 - 1) / p->l; ++wr)
           for (int wc = cd.c0 / p->l; wc <= (cd.c1 - 1) / p->l; ++wc) {
@@ -252,6 +366,8 @@ int build_tables(ultragen_plan_t* p) {
   build_schedule(p);
   return ULTRAGEN_OK;
 }
+
+}  // namespace
 
 static bool same_list(const ultragen_plan_t* p, int a, int b) {
   const int na = p->row_ptr[a + 1] - p->row_ptr[a];
@@ -454,6 +570,25 @@ int ultragen_plan_set_lr_scope(ultragen_plan_t* p, int radius) {
   return ULTRAGEN_OK;
 }
 
+int ultragen_plan_set_halo(ultragen_plan_t* p, int mode) {
+  if (!p || mode < -1 || mode > 1) return ULTRAGEN_ERR_INVALID_ARG;
+  const int old = p->halo_req;
+  p->halo_req = mode;
+  int st;
+  try {
+    st = ug::build_tables(p);
+  } catch (const std::bad_alloc&) {
+    st = ULTRAGEN_ERR_OOM;
+  }
+  if (st != ULTRAGEN_OK) {
+    p->halo_req = old;
+    ug::build_tables(p);
+    return st;
+  }
+  p->dirty = true;
+  return ULTRAGEN_OK;
+}
+
 int ultragen_plan_info(const ultragen_plan_t* p, ultragen_plan_info_t* o) {
   if (!p || !o) return ULTRAGEN_ERR_INVALID_ARG;
   std::memset(o, 0, sizeof(*o));
@@ -474,15 +609,25 @@ int ultragen_plan_info(const ultragen_plan_t* p, ultragen_plan_info_t* o) {
   o->n_split_items = p->n_split_items;
   o->workspace_bytes_per_head = (int64_t)p->n_split_items * 2 * ug::kTile * (p->D + 1) * 4;
   o->lr_radius = p->lr_radius;
+  o->halo_copy = p->halo_copy;
+  o->halo_slots_per_window = (int32_t)p->G;
+  o->N_kv = p->N_kv;
+  o->off_halo = p->off_halo;
   return ULTRAGEN_OK;
 }
 
 int ultragen_plan_export(const ultragen_plan_t* p, int32_t* perm, int32_t* row_ptr,
                          int32_t* entries) {
   if (!p) return ULTRAGEN_ERR_INVALID_ARG;
-  if (perm) std::memcpy(perm, p->perm.data(), p->perm.size() * sizeof(int32_t));
+  if (perm) std::memcpy(perm, p->perm.data(), (size_t)p->N_tot * sizeof(int32_t));
   if (row_ptr) std::memcpy(row_ptr, p->row_ptr.data(), p->row_ptr.size() * sizeof(int32_t));
   if (entries) std::memcpy(entries, p->entries.data(), p->entries.size() * sizeof(int32_t));
+  return ULTRAGEN_OK;
+}
+
+int ultragen_plan_export_kv(const ultragen_plan_t* p, int32_t* kv_perm) {
+  if (!p || !kv_perm) return ULTRAGEN_ERR_INVALID_ARG;
+  std::memcpy(kv_perm, p->perm.data(), (size_t)p->N_kv * sizeof(int32_t));
   return ULTRAGEN_OK;
 }
 

@@ -11,7 +11,8 @@ namespace ug {
 constexpr int kTile = 128;          // query and key tile edge (rows / columns)
 constexpr int kItemInts = 8;        // int32 fields per work item
 
-enum Seg : int8_t { SEG_PAD = -1, SEG_TEXT = 0, SEG_HR = 1, SEG_LR = 2 };
+// SEG_HALO: a K/V slot of a window's compact halo block
+enum Seg : int8_t { SEG_PAD = -1, SEG_TEXT = 0, SEG_HR = 1, SEG_LR = 2, SEG_HALO = 3 };
 
 // One unit of kernel work for one (batch, head): one or two query tiles that share the same
 // key-tile list and masks, over a contiguous range of that list.
@@ -34,9 +35,11 @@ struct DeviceTables {
   int32_t* entries = nullptr;
   int32_t* mask_off = nullptr;
   uint32_t* mask_pool = nullptr;
-  int32_t* perm = nullptr;
+  int32_t* perm = nullptr;         // K/V slot -> raster over N_kv (its first N_tot: Q slots)
   int32_t* inv_perm = nullptr;
-  uint32_t* slot_pos = nullptr;    // (pos_row << 16) | pos_col per slot; 0 for text/pad
+  uint32_t* slot_pos = nullptr;    // (pos_row << 16) | pos_col per K/V slot; 0 for text/pad
+  int32_t* halo_ptr = nullptr;     // halo-block copies of each window-segment slot (CSR)
+  int32_t* halo_dst = nullptr;
   float* rope = nullptr;           // [max(H,W)][head_dim/2][2] (cos, sin)
   int32_t* combine = nullptr;      // CombineGroup[]
   int* error = nullptr;            // device error word
@@ -61,16 +64,25 @@ struct ultragen_plan {
   int split_chunk = 0;
   // HR -> LR scope: -1 all LR tokens; r >= 0 the anchors within r of the query's window
   int lr_radius = -1;
+  // compact halo blocks in the K/V layout: requested (-1 auto, 0 off, 1 on) and in effect;
+  // G K/V slots per window, N_kv = N_tot + nWh * nWw * G
+  int halo_req = -1;
+  int halo_copy = 0;
+  int64_t G = 0, N_kv = 0, off_halo = 0;
   // diagnostics: device wait limit and injected fault (ultragen_plan_set_diagnostics)
   unsigned long long wait_limit_ns = 2000ull * 1000 * 1000;
   int fault = 0;
 
   // host tables
-  std::vector<int32_t> perm;       // slot -> raster (-1 pad)
-  std::vector<int32_t> inv_perm;   // raster -> slot
-  std::vector<int8_t> seg;         // per slot
-  std::vector<int32_t> ci, cj;     // per slot coordinates (HR: i,j; LR: m,n; text: t,0)
-  std::vector<uint32_t> slot_pos;  // per slot packed RoPE positions
+  std::vector<int32_t> perm;       // K/V slot -> raster (-1 pad), N_kv long; Q slots are its
+                                   // first N_tot entries
+  std::vector<int32_t> inv_perm;   // raster -> slot (the window segment copy)
+  std::vector<int8_t> seg;         // per K/V slot
+  std::vector<int32_t> ci, cj;     // per K/V slot coordinates (HR: i,j; LR: m,n; text: t,0)
+  std::vector<int32_t> owner;      // per K/V slot: window of an HR or halo slot, else -1
+  std::vector<uint32_t> slot_pos;  // per K/V slot packed RoPE positions
+  std::vector<int32_t> halo_ptr;   // halo blocks: CSR over window-segment slots (N_hrp + 1) of
+  std::vector<int32_t> halo_dst;   //   the halo-block slots that copy the slot's token
   std::vector<int32_t> row_ptr;    // CSR over query tiles
   std::vector<int32_t> entries;    // key tile | partial << 31
   std::vector<int32_t> mask_off;   // per entry: offset into mask_pool, -1 when full

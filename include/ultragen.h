@@ -24,6 +24,9 @@
  *   slots [0, T) text | pad to a multiple of 128 | HR tokens window-first (windows row-major,
  *   l*l slots each, raster order inside; partial edge windows padded) | pad to 128 |
  *   LR tokens raster | pad to 128.   N_tot = number of slots, a multiple of 128.
+ *   K/V layout: the same N_tot slots, then, when the plan uses compact halo blocks
+ *   (ultragen_plan_set_halo), one block of G slots per window holding that window's halo
+ *   tokens; N_kv = N_tot + nWh * nWw * G (N_kv = N_tot without blocks).  Q and O use N_tot.
  *   Raster layout: tokens ordered text, HR raster (row i, column j), LR raster.
  */
 #ifndef ULTRAGEN_H
@@ -73,6 +76,10 @@ typedef struct {
   int32_t n_split_items;      /* items that write split partials (per head)             */
   int64_t workspace_bytes_per_head; /* split partial storage per (batch, head)          */
   int32_t lr_radius;          /* HR -> LR scope (ultragen_plan_set_lr_scope)            */
+  int32_t halo_copy;          /* 1: K/V carry compact halo blocks (ultragen_plan_set_halo) */
+  int32_t halo_slots_per_window; /* G: slots of one window's halo block (0 without)      */
+  int64_t N_kv;               /* K/V slots: N_tot + nWh * nWw * G                        */
+  int64_t off_halo;           /* first halo-block slot (= N_tot)                         */
 } ultragen_plan_info_t;
 
 /* Human-readable name of a status code.  Never NULL. */
@@ -115,6 +122,18 @@ int ultragen_plan_set_split(ultragen_plan_t* plan, int chunk);
  * tile lists; rope and split settings are kept.  INVALID_ARG for radius < -1. */
 int ultragen_plan_set_lr_scope(ultragen_plan_t* plan, int radius);
 
+/* Compact halo blocks in the K/V layout (no counterpart in the pages; the attention is the
+ * same function).  Window w's halo -- the HR tokens of its box grown by b ([UG-note] 关键设计 1/2,
+ * "adjacent boundary tokens"), clipped to the image, outside the window itself -- is copied
+ * by ultragen_permute_rope, in raster order of the box, into K/V slots
+ * [off_halo + w*G, off_halo + (w+1)*G), G = the largest halo padded to 128.  An HR query of
+ * window w then reads its neighbours' tokens from that one dense block instead of partial
+ * tiles of up to 8 neighbouring windows; nothing else sees the blocks.  mode = 1 on, 0 off,
+ * -1 automatic (the default: on when the tile steps saved outweigh the copies, e.g. b = 4 with
+ * l = 16; off when b = 0 or when the neighbours' tiles are all fully visible, e.g. b = l).
+ * Rebuilds the tile lists; changes N_kv.  INVALID_ARG for another mode. */
+int ultragen_plan_set_halo(ultragen_plan_t* plan, int mode);
+
 int ultragen_plan_info(const ultragen_plan_t* plan, ultragen_plan_info_t* out);
 
 /*
@@ -128,6 +147,11 @@ int ultragen_plan_info(const ultragen_plan_t* plan, ultragen_plan_info_t* out);
 int ultragen_plan_export(const ultragen_plan_t* plan, int32_t* perm, int32_t* row_ptr,
                          int32_t* entries);
 
+/* Host copy of the K/V slot map: kv_perm [N_kv], raster index of each K/V slot (its first
+ * N_tot entries equal perm; halo-block slots follow), -1 for pad slots.  Entries of the tile
+ * lists index K/V tiles of this layout. */
+int ultragen_plan_export_kv(const ultragen_plan_t* plan, int32_t* kv_perm);
+
 /* Per-row visibility of query tile `qtile`: out[e][r][w] (uint32) for each of the tile's
  * entries e, rows r in [0,128), words w in [0,4); bit c%32 of word c/32 = key column c of
  * the entry's key tile visible to row r.  Rows of pad slots are 0.  `out` holds
@@ -140,7 +164,9 @@ int ultragen_plan_destroy(ultragen_plan_t* plan);
  * ultragen_permute_rope -- raster -> window-first gather of Q, K, V fused with axial 2D
  * RoPE on Q and K ([UG-note] 关键设计 1 window-first order; 关键设计 2 position scaling).
  *   q, k, v     [batch, N_raster, heads, head_dim], in_dtype BF16 or F32 (device)
- *   qp, kp, vp  [batch, heads, N_tot, head_dim] BF16 (device); pad slots written as 0
+ *   qp          [batch, heads, N_tot, head_dim] BF16 (device); pad slots written as 0
+ *   kp, vp      [batch, heads, N_kv, head_dim] BF16 (device): the N_tot slots, then the
+ *               halo blocks (each halo token's row again, with its own RoPE position)
  * RoPE is computed in fp32 from fp32 tables and rounded to bf16 (nearest even); V and
  * text tokens are copied (F32 input: rounded to bf16).
  */
@@ -152,7 +178,8 @@ int ultragen_permute_rope(const void* q, const void* k, const void* v, int in_dt
  * ultragen_hla_forward -- masked joint attention softmax(Q K^T / sqrt(d) + M) V
  * ([UG-note] 关键设计 3, the MMA equation; M additive -inf on masked pairs) over the
  * permuted layout, visiting only the key tiles of each query tile's list.
- *   qp, kp, vp, op  [batch, heads, N_tot, head_dim] BF16 (device); op rows of pad slots = 0
+ *   qp, op  [batch, heads, N_tot, head_dim] BF16 (device); op rows of pad slots = 0
+ *   kp, vp  [batch, heads, N_kv, head_dim] BF16 (device), as ultragen_permute_rope writes them
  * bf16 tensor-core products with fp32 accumulation and fp32 online softmax.  Uses the
  * plan's split workspace (device memory the plan allocates and keeps) when the plan
  * splits groups; a call that needs more than the plan holds grows it with stream-ordered
@@ -165,7 +192,8 @@ int ultragen_hla_forward(const void* qp, const void* kp, const void* vp, void* o
 /*
  * ultragen_hla_forward_raster -- ultragen_hla_forward with the unpermute folded into its
  * epilogue: each output row goes straight to its raster place.
- *   qp, kp, vp  [batch, heads, N_tot, head_dim] BF16 (device, permuted)
+ *   qp          [batch, heads, N_tot, head_dim] BF16 (device, permuted)
+ *   kp, vp      [batch, heads, N_kv, head_dim] BF16 (device, K/V layout)
  *   o           [batch, N_raster, heads, head_dim] BF16 (device, raster); pad slots write nothing
  * Same arithmetic as ultragen_hla_forward + ultragen_unpermute (bit for bit), one pass less
  * over HBM.  Errors as ultragen_hla_forward.
@@ -244,8 +272,8 @@ int ultragen_last_launch_count(const ultragen_plan_t* plan);
  *   Asynchronous: the work is ordered after what `stream` holds at the call, and `stream`
  *   waits for all of it, so o is complete once `stream` is synchronised.  Calls on one runner
  *   must not overlap (one call at a time per runner).  PLAN_MISMATCH when called on another
- *   device than the one the runner was created on, or when the plan's split schedule now needs
- *   more partial storage than was allocated.  Device-side wait timeouts are reported by
+ *   device than the one the runner was created on, or when the plan's split schedule or halo
+ *   blocks now need more storage than was allocated.  Device-side wait timeouts are reported by
  *   ultragen_sync_status(plan, stream).
  * ultragen_host_runner_last_launch_count(runner): kernels the last forward launched.
  * ultragen_host_runner_destroy(runner): waits for the runner's streams, frees everything.

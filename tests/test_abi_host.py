@@ -155,14 +155,18 @@ def sample_qtiles(g, n_hr=40, seed=0):
     return sorted(set(text + lr[:3] + lr[-3:] + pick))
 
 
-def compare_plan(ffi, geom, qtiles=None):
-    g = O.Geometry(*geom)
+def compare_plan(ffi, geom, qtiles=None, halo=None):
     p = ffi.Plan(*geom, 2, 64)
+    if halo is not None:
+        p.set_halo(halo)
     info = p.info
+    g = O.Geometry(*geom, halo_copy=bool(info["halo_copy"]))
     assert info["N_tot"] == g.N_tot and info["N_raster"] == g.N_raster
     assert info["off_hr"] == g.off_hr and info["off_lr"] == g.off_lr
+    assert info["N_kv"] == g.N_kv and info["halo_slots_per_window"] == g.G
     perm, row_ptr, entries = p.export()
     np.testing.assert_array_equal(perm, O.perm_map(g))
+    np.testing.assert_array_equal(p.export_kv(), O.kv_perm_map(g))
     qtiles = range(g.N_tot // 128) if qtiles is None else qtiles
     for t in qtiles:
         e_ref, m_ref = O.qtile_entries(g, t)
@@ -172,11 +176,32 @@ def compare_plan(ffi, geom, qtiles=None):
     return g, p
 
 
+@pytest.mark.parametrize("halo", [None, 0, 1])
 @pytest.mark.parametrize("name", ["tiny", "1k", "odd", "small_l", "no_lr_text", "win32_rho2",
                                   "single", "win_exceeds", "rho_exceeds", "thin"])
-def test_plan_bit_exact_full(ffi, name):
-    g, p = compare_plan(ffi, GEOMS[name])
+def test_plan_bit_exact_full(ffi, name, halo):
+    g, p = compare_plan(ffi, GEOMS[name], halo=halo)
     assert p.info["useful_pairs"] == O.visible_pair_count(g)
+
+
+def test_halo_mode_argument_checks_and_auto_choice(ffi):
+    p = ffi.Plan(64, 64, 16, 4, 4, 512, 2, 64)
+    assert ffi.lib().ultragen_plan_set_halo(p.handle, 2) == 1
+    assert ffi.lib().ultragen_plan_set_halo(p.handle, -2) == 1
+    useful = p.info["useful_pairs"]
+    for mode in (0, 1, -1):
+        p.set_halo(mode)
+        assert p.info["useful_pairs"] == useful            # the same attention either way
+    p.set_halo(1)
+    assert p.info["halo_copy"] == 1 and p.info["N_kv"] > p.info["N_tot"]
+    p.set_halo(0)
+    assert p.info["halo_copy"] == 0 and p.info["N_kv"] == p.info["N_tot"]
+    # b = l: every neighbour tile is fully visible, so the automatic choice keeps them
+    q = ffi.Plan(256, 135, 16, 16, 4, 256, 2, 64)
+    assert q.info["halo_copy"] == 0
+    # b = 0: no halo at all
+    r = ffi.Plan(64, 64, 16, 0, 4, 16, 2, 64)
+    assert r.info["halo_copy"] == 0
 
 
 @pytest.mark.parametrize("name", ["ragged"])
@@ -201,7 +226,10 @@ def test_plan_4k_8k_sampled_and_pair_counts(ffi):
 def test_split_policy(ffi):
     p = ffi.Plan(256, 256, 16, 4, 4, 512, 24, 128)
     i = p.info
-    assert i["split_chunk"] == 48 and i["n_split_groups"] == 2
+    # automatic chunk: the longest HR / LR query-tile list, applied to the text groups only
+    _, row_ptr, _ = p.export()
+    longest = int(np.diff(row_ptr)[i["off_hr"] // 128:].max())
+    assert i["split_chunk"] == max(longest, 8) and i["n_split_groups"] == 2
     p.set_split(0)
     assert p.info["n_split_groups"] == 0 and p.info["workspace_bytes_per_head"] == 0
     p.set_split(7)
@@ -220,12 +248,13 @@ def test_diagnostics_validation(ffi):
 
 
 def compare_region_plan(ffi, geom, r, qtiles=None):
-    g = O.Geometry(*geom, lr_radius=r)
     p = ffi.Plan(*geom, 2, 64)
     p.set_lr_scope(r)
     assert p.info["lr_radius"] == r
+    g = O.Geometry(*geom, lr_radius=r, halo_copy=bool(p.info["halo_copy"]))
     perm, row_ptr, entries = p.export()
     np.testing.assert_array_equal(perm, O.perm_map(g))
+    np.testing.assert_array_equal(p.export_kv(), O.kv_perm_map(g))
     for t in (range(g.N_tot // 128) if qtiles is None else qtiles):
         e_ref, m_ref = O.qtile_entries(g, t)
         np.testing.assert_array_equal(entries[row_ptr[t]:row_ptr[t + 1]].view(np.uint32), e_ref,

@@ -29,11 +29,13 @@ def _wl(name, **kw):
     return dataclasses.replace(WORKLOADS[name], **kw) if kw else WORKLOADS[name]
 
 
-def run_layer(ug, wl, split=None, poison=True, lr_radius=-1):
+def run_layer(ug, wl, split=None, poison=True, lr_radius=-1, halo=None):
     import torch
     plan = ug.plan_for(wl)
     if lr_radius != -1:
         plan.set_lr_scope(lr_radius)
+    if halo is not None:
+        plan.set_halo(halo)
     if split is not None:
         plan.set_split(split)
     q, k, v = ug.make_qkv(wl)
@@ -75,22 +77,24 @@ def custom(name):
     return dataclasses.replace(WORKLOADS["1k"], **CUSTOM[name])
 
 
-def expected_qkv_perm(wl, q, k, v, b, h):
-    """Oracle RoPE'd, permuted Q, K (rounded to bf16), V, and the per-element pair magnitude
-    |x_2k| + |x_2k+1| of the unrotated inputs."""
-    g = geometry(wl)
+def expected_qkv_perm(wl, q, k, v, b, h, halo=False):
+    """Oracle RoPE'd, permuted Q, K (rounded to bf16), V -- K and V in the K/V layout, with the
+    halo blocks when the plan has them -- and the per-element pair magnitude |x_2k| + |x_2k+1|
+    of the unrotated inputs in the same layouts."""
+    g = dataclasses.replace(geometry(wl), halo_copy=halo)
     pos = O.positions(g)
     qh, kh, vh = (to_np64(x[b:b + 1, :, h:h + 1, :]) for x in (q, k, v))
     qp = O.permute(O.rope(qh, pos, wl.axes), g)[0, 0]
-    kp = O.permute(O.rope(kh, pos, wl.axes), g)[0, 0]
-    vp = O.permute(vh, g)[0, 0]
+    kp = O.permute_kv(O.rope(kh, pos, wl.axes), g)[0, 0]
+    vp = O.permute_kv(vh, g)[0, 0]
 
-    def pair_mag(x):
-        xp = np.abs(O.permute(x, g)[0, 0])
+    def pair_mag(x, perm):
+        xp = np.abs(perm(x, g)[0, 0])
         s = xp[:, 0::2] + xp[:, 1::2]
         return np.repeat(s, 2, axis=1)
 
-    return (O.round_bf16(qp), O.round_bf16(kp), O.round_bf16(vp), pair_mag(qh), pair_mag(kh))
+    return (O.round_bf16(qp), O.round_bf16(kp), O.round_bf16(vp), pair_mag(qh, O.permute),
+            pair_mag(kh, O.permute_kv))
 
 
 # RoPE is evaluated in fp32 from fp32 cos/sin tables, then rounded to bf16 (nearest even).
@@ -108,15 +112,17 @@ def ulp_bf16(x):
     return np.where(a > 0, 2.0 ** (np.maximum(e, -126) - 7), 2.0 ** -133)
 
 
-@pytest.mark.parametrize("name", ["tiny", "1k", "ragged", "odd", "small_l", "text_only_pad", "single",
-                                  "win_exceeds", "thin"])
-def test_permute_rope_parity(ug, name):
+@pytest.mark.parametrize("name,halo", [("tiny", None), ("1k", None), ("ragged", None), ("odd", None),
+                                       ("small_l", None), ("text_only_pad", None), ("single", None),
+                                       ("win_exceeds", None), ("thin", None), ("1k", 1), ("odd", 1),
+                                       ("thin", 1)])
+def test_permute_rope_parity(ug, name, halo):
     wl = _wl(name) if name in ("tiny", "1k", "ragged") else custom(name)
-    plan, (q, k, v), lay, _ = run_layer(ug, wl)
+    plan, (q, k, v), lay, _ = run_layer(ug, wl, halo=halo)
     heads = range(wl.heads) if wl.heads <= 3 else (0, wl.heads // 2, wl.heads - 1)
     for b in range(wl.batch):
         for h in heads:
-            eq, ek, ev, mq, mk = expected_qkv_perm(wl, q, k, v, b, h)
+            eq, ek, ev, mq, mk = expected_qkv_perm(wl, q, k, v, b, h, bool(plan.info["halo_copy"]))
             gq, gk, gv = (to_np64(t[b, h]) for t in (lay.qp, lay.kp, lay.vp))
             np.testing.assert_array_equal(gv, ev, err_msg="V gather must be bit-exact")
             for got, exp, mag, nm in ((gq, eq, mq, "Q"), (gk, ek, mk, "K")):
@@ -138,24 +144,31 @@ def test_unpermute_inverts_permute_bitwise(ug, name):
     wl = _wl(name)
     plan, (q, k, v), lay, _ = run_layer(ug, wl)
     vd = v.cuda()
+    vq = lay.vp[:, :, :plan.info["N_tot"]].contiguous()   # the window segment (Q layout)
     back = torch.empty_like(vd)
-    ug.unpermute(lay.vp, back, plan)
+    ug.unpermute(vq, back, plan)
     back32 = torch.empty(vd.shape, dtype=torch.float32, device="cuda")
-    ug.unpermute(lay.vp, back32, plan)
+    ug.unpermute(vq, back32, plan)
     torch.cuda.synchronize()
     assert torch.equal(back.view(torch.int16), vd.view(torch.int16))
     assert torch.equal(back32, vd.float())
 
 
 # ------------------------------------------------------------------ attention
-@pytest.mark.parametrize("name,split", [("tiny", None), ("tiny", 0), ("tiny", 2), ("1k", None),
-                                        ("1k", 0), ("1k", 5), ("odd", None), ("odd", 3),
-                                        ("small_l", None), ("no_lr_text", None), ("win32_rho2", None),
-                                        ("text_only_pad", 1), ("single", None), ("win_exceeds", None),
-                                        ("rho_exceeds", None), ("thin", None), ("thin", 1)])
-def test_attention_full_parity(ug, name, split):
+@pytest.mark.parametrize("name,split,halo", [
+    ("tiny", None, None), ("tiny", 0, None), ("tiny", 2, None), ("1k", None, None), ("1k", 0, None),
+    ("1k", 5, None), ("odd", None, None), ("odd", 3, None), ("small_l", None, None),
+    ("no_lr_text", None, None), ("win32_rho2", None, None), ("text_only_pad", 1, None),
+    ("single", None, None), ("win_exceeds", None, None), ("rho_exceeds", None, None),
+    ("thin", None, None), ("thin", 1, None),
+    # compact halo blocks forced on (R18): the same attention
+    ("tiny", None, 1), ("1k", None, 1), ("1k", 5, 1), ("odd", 3, 1), ("small_l", None, 1),
+    ("win32_rho2", None, 1), ("win_exceeds", None, 1), ("thin", 1, 1),
+    # and forced off where the automatic choice takes them
+    ("win32_rho2", None, 0)])
+def test_attention_full_parity(ug, name, split, halo):
     wl = _wl(name) if name in ("tiny", "1k") else custom(name)
-    plan, (q, k, v), lay, o = run_layer(ug, wl, split=split)
+    plan, (q, k, v), lay, o = run_layer(ug, wl, split=split, halo=halo)
     g = geometry(wl)
     perm = O.perm_map(g)
     rows = np.arange(g.N_tot)
