@@ -54,6 +54,14 @@ Readings taken where the pages are silent or garbled (each is listed in DESIGN.m
       w then takes the other windows' tokens of its box from w's block instead of their
       window segments; halo blocks are visible to nothing else.  Every query sees the same
       tokens as without them, so the attention output is the same function.
+  R19 Optional 8-bit Q K^T (qk_format = "e4m3"; the pages only place the permuted layout next
+      to SageAttention's tiling, [UG-note] 关键设计 1): after RoPE, every element x of Q (of K)
+      is stored as the e4m3 value nearest to x * 2^-q_exp (x * 2^-k_exp), ties to even, values
+      beyond the largest finite e4m3 magnitude 448 clamped to +-448; the logits are formed from
+      those stored values times 2^(q_exp + k_exp).  The exponents are per tensor and chosen by
+      the caller (default 0); a power of two makes the scaling itself exact.  V, the softmax
+      and P V keep their precision.  e4m3 is the OCP 8-bit float with 4 exponent bits
+      (bias 7) and 3 mantissa bits, subnormals, no infinities, one NaN pattern per sign.
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py`` (brute force
 on tiny grids, closed forms, textbook special cases, invariants).  The pages print no
@@ -470,15 +478,21 @@ def attention_rows(qp: np.ndarray, kp: np.ndarray, vp: np.ndarray, g: Geometry,
 
 
 def forward(q: np.ndarray, k: np.ndarray, v: np.ndarray, g: Geometry, axes,
-            theta: float = 1.0e4, rows=None, heads=None):
+            theta: float = 1.0e4, rows=None, heads=None, qk_format: str = "bf16",
+            q_exp: int = 0, k_exp: int = 0):
     """Whole path on raster inputs [B, N_raster, Hh, D]: RoPE -> permute -> attention.
 
-    Returns (O_rows [B, Hh', n, D] for the permuted ``rows`` (all slots by default),
-    rows).  Unpermute the full result with ``unpermute``.
+    qk_format "e4m3" stores the RoPE'd Q and K as scaled e4m3 values first (R19); "bf16"
+    keeps them exact.  Returns (O_rows [B, Hh', n, D] for the permuted ``rows`` (all slots by
+    default), rows).  Unpermute the full result with ``unpermute``.
     """
     pos = positions(g)
     qr = rope(q, pos, axes, theta)
     kr = rope(k, pos, axes, theta)
+    if qk_format == "e4m3":
+        qr, kr = quantize_e4m3(qr, q_exp), quantize_e4m3(kr, k_exp)
+    elif qk_format != "bf16":
+        raise ValueError(f"unknown qk_format {qk_format!r}")
     qp, kp, vp = permute(qr, g), permute_kv(kr, g), permute_kv(np.asarray(v, np.float64), g)
     rows = np.arange(g.N_tot) if rows is None else np.asarray(rows, np.int64)
     return attention_rows(qp, kp, vp, g, rows, heads=heads), rows
@@ -550,3 +564,55 @@ def round_bf16(x: np.ndarray) -> np.ndarray:
     ulp = 2.0 ** (e - 7)
     out[nz] = np.round(xv / ulp) * ulp        # np.round: ties to even
     return out
+
+
+# --------------------------------------------------------------------------------------
+# 8-bit Q K^T (R19)
+# --------------------------------------------------------------------------------------
+
+E4M3_MAX = 448.0             # largest finite e4m3 magnitude: 2^8 * (1 + 6/8)
+E4M3_MIN_NORMAL_EXP = -6     # 1 - bias 7; below 2^-6 the spacing stays 2^-9 (subnormals)
+
+
+def round_e4m3(x: np.ndarray) -> np.ndarray:
+    """Nearest e4m3 value (ties to even), clamped to +-448; returns fp64 (R19).
+
+    A finite x with 2^e <= |x| < 2^(e+1) has spacing 2^(e-3) between its e4m3 neighbours
+    (3 mantissa bits); below the smallest normal 2^-6 the spacing stays 2^-9.  Rounding x
+    to a multiple of that spacing, ties to even, is exact in fp64.  Finite inputs only.
+    """
+    x = np.asarray(x, np.float64)
+    out = np.zeros_like(x)
+    nz = x != 0
+    xv = x[nz]
+    e = np.floor(np.log2(np.abs(xv)))
+    e = np.where(np.abs(xv) < 2.0 ** e, e - 1, e)          # log2 rounding at powers of two
+    e = np.where(np.abs(xv) >= 2.0 ** (e + 1), e + 1, e)
+    e = np.maximum(e, float(E4M3_MIN_NORMAL_EXP))
+    ulp = 2.0 ** (e - 3)
+    out[nz] = np.clip(np.round(xv / ulp) * ulp, -E4M3_MAX, E4M3_MAX)   # np.round: ties to even
+    return out
+
+
+def quantize_e4m3(x: np.ndarray, exp: int) -> np.ndarray:
+    """The value an e4m3-stored tensor with scale 2^exp represents: round(x 2^-exp) 2^exp."""
+    return round_e4m3(np.asarray(x, np.float64) * 2.0 ** -exp) * 2.0 ** exp
+
+
+def e4m3_codes(x: np.ndarray, exp: int) -> np.ndarray:
+    """The stored bytes of round_e4m3(x 2^-exp) (R19): sign bit 7, exponent bits 6..3
+    (bias 7, field 0 for zero and subnormals), mantissa bits 2..0."""
+    y = round_e4m3(np.asarray(x, np.float64) * 2.0 ** -exp)
+    sign = (y < 0) | ((y == 0) & np.signbit(y))
+    a = np.abs(y)
+    code = np.zeros(y.shape, np.int64)
+    nz = a > 0
+    av = a[nz]
+    e = np.floor(np.log2(av))
+    e = np.where(av < 2.0 ** e, e - 1, e)
+    e = np.where(av >= 2.0 ** (e + 1), e + 1, e)
+    sub = e < E4M3_MIN_NORMAL_EXP
+    field = np.where(sub, 0, e + 7).astype(np.int64)
+    mant = np.where(sub, av / 2.0 ** -9, (av / 2.0 ** e - 1.0) * 8.0)
+    code[nz] = (field << 3) | np.rint(mant).astype(np.int64)
+    return (code | (sign.astype(np.int64) << 7)).astype(np.uint8)

@@ -112,14 +112,19 @@ def bf_rope_vec(x, pos, axes, theta=1e4):
     return y
 
 
-def bf_forward(q, k, v, H, W, l, b, rho, T, axes, lr_radius=-1):
-    """Pure-Python HLA on raster inputs [B, N, Hh, D]; returns raster output."""
+def bf_forward(q, k, v, H, W, l, b, rho, T, axes, lr_radius=-1, quant_q=None, quant_k=None):
+    """Pure-Python HLA on raster inputs [B, N, Hh, D]; returns raster output.  quant_q /
+    quant_k, when given, map each RoPE'd element of Q / K to its stored value."""
     toks = bf_tokens(H, W, rho, T)
     B, N, Hh, D = q.shape
     out = np.zeros((B, N, Hh, D))
     for bi, hh in itertools.product(range(B), range(Hh)):
         qr = [bf_rope_vec(q[bi, t, hh].tolist(), bf_position(tok, rho), axes) for t, tok in enumerate(toks)]
         kr = [bf_rope_vec(k[bi, t, hh].tolist(), bf_position(tok, rho), axes) for t, tok in enumerate(toks)]
+        if quant_q is not None:
+            qr = [[quant_q(x) for x in row] for row in qr]
+        if quant_k is not None:
+            kr = [[quant_k(x) for x in row] for row in kr]
         for t, tok in enumerate(toks):
             logits = []
             for u, utok in enumerate(toks):
