@@ -51,6 +51,10 @@ def parse():
                     help="HR->LR scope: -1 all LR tokens (default); r >= 0 the window's anchors grown by r")
     ap.add_argument("--halo", type=int, default=-1, choices=[-1, 0, 1],
                     help="compact halo blocks in the K/V layout: -1 automatic (default), 0 off, 1 on")
+    ap.add_argument("--qk", default="bf16", choices=["bf16", "e4m3"],
+                    help="storage of the permuted Q and K: bf16 (default) or scaled e4m3 with 8-bit Q K^T")
+    ap.add_argument("--q-exp", type=int, default=0, help="e4m3 Q stores x * 2^-q_exp")
+    ap.add_argument("--k-exp", type=int, default=0, help="e4m3 K stores x * 2^-k_exp")
     ap.add_argument("--impl", default="ultragen", choices=["ultragen", "reference"])
     ap.add_argument("--unfused", action="store_true",
                     help="run unpermute as its own pass instead of in the attention epilogue")
@@ -167,9 +171,10 @@ def profiled_traffic(workload: str):
     return ent.get("dram_bytes_per_launch")
 
 
-def cpu_baseline(wl, q, k, v, budget_s: float = 12.0):
+def cpu_baseline(wl, q, k, v, budget_s: float = 12.0, **fwd):
     """The oracle as it stands, timed on this host on a bounded sample: one head, rows of one
-    interior window plus text and LR rows, growing until about `budget_s` of CPU work."""
+    interior window plus text and LR rows, growing until about `budget_s` of CPU work
+    (``fwd``: the oracle forward's Q/K format options)."""
     import numpy as np
 
     from oracle import hla_oracle as O
@@ -186,7 +191,7 @@ def cpu_baseline(wl, q, k, v, budget_s: float = 12.0):
     t0 = time.perf_counter()
     reps = 0
     while True:
-        O.forward(qh, kh, vh, g, wl.axes, rows=rows)
+        O.forward(qh, kh, vh, g, wl.axes, rows=rows, **fwd)
         reps += 1
         if time.perf_counter() - t0 > budget_s:
             break
@@ -417,6 +422,9 @@ def main():
         plan.set_lr_scope(args.lr_radius)
     if args.halo != -1:
         plan.set_halo(args.halo)
+    e4m3 = args.qk == "e4m3"
+    if e4m3:
+        plan.set_qk_format("e4m3", args.q_exp, args.k_exp)
     info = plan.info
     q, k, v = ug.make_qkv(wl)
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
@@ -483,11 +491,13 @@ def main():
     elem = wl.batch * wl.heads * info["N_tot"] * wl.D
     kv_elem = wl.batch * wl.heads * info["N_kv"] * wl.D
     in_size = 2 if wl.dtype == "bf16" else 4
+    qk_size = 1 if e4m3 else 2
     # permute_rope: every raster row of Q, K, V read once (halo copies are written from the
     # same read), Q written over N_tot slots and K, V over N_kv slots (pad slots as zeros)
-    perm_bytes = 3 * wl.batch * info["N_raster"] * wl.heads * wl.D * in_size + (elem + 2 * kv_elem) * 2
+    perm_bytes = (3 * wl.batch * info["N_raster"] * wl.heads * wl.D * in_size
+                  + (elem + kv_elem) * qk_size + kv_elem * 2)
     unperm_bytes = elem * 2 + wl.batch * info["N_raster"] * wl.heads * wl.D * 2
-    traffic = profiled_traffic(wl.name)
+    traffic = profiled_traffic(wl.name + ("-e4m3" if e4m3 else ""))
 
     e2e = None
     if not args.no_e2e:
@@ -518,7 +528,8 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(wl, q, k, v)
+        cpu = cpu_baseline(wl, q, k, v, **({"qk_format": "e4m3", "q_exp": args.q_exp,
+                                            "k_exp": args.k_exp} if e4m3 else {}))
 
     # roofline denominator: the burst bf16 figure while the SM clock held its maximum during
     # the timed steps, the sustained (power-capped) one once the clock dropped under the cap
@@ -530,19 +541,27 @@ def main():
     else:
         peak = pk["bf16_tflops"]
         peak_note = f"{src} bf16 dense, burst (SM clock at its maximum during the timed steps)"
+    if e4m3:
+        # half the useful FLOPs (Q K^T) at the e4m3 rate, nominally twice the bf16 rate, half
+        # (P V) at the bf16 rate: the mixed peak is 1 / (0.5 / 2P + 0.5 / P) = 4P / 3
+        peak *= 4.0 / 3.0
+        peak_note += "; x 4/3 for the mixed e4m3 Q K^T (nominal 2x bf16) + bf16 P V contraction"
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "useful TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3 Q.K^T (fp32 acc) + bf16 P.V" if e4m3 else "bf16",
             "data": "synthetic (seeded N(0,1) + smooth 2D sinusoid Q/K/V; no weights needed)",
-            "config": {"workload": wl.name + ("" if args.lr_radius < 0 else f"-lr-region-r{args.lr_radius}"),
+            "config": {"workload": wl.name + ("" if args.lr_radius < 0 else f"-lr-region-r{args.lr_radius}")
+                                   + ("-e4m3-qk" if e4m3 else ""),
                        "H": wl.H, "W": wl.W, "l": wl.l, "b": wl.b,
                        "rho": wl.rho, "text_len": wl.T, "lr_radius": args.lr_radius, "heads": wl.heads, "head_dim": wl.D,
                        "batch": wl.batch, "N_tot": info["N_tot"], "useful_pairs_per_head": info["useful_pairs"],
                        "halo_blocks": bool(info["halo_copy"]), "N_kv": info["N_kv"],
-                       "l2": "inputs larger than L2 (permuted Q %.0f MB, K and V %.0f MB each); no flush"
-                             % (elem * 2 / 1e6, kv_elem * 2 / 1e6),
+                       "qk_format": args.qk, **({"q_exp": args.q_exp, "k_exp": args.k_exp} if e4m3 else {}),
+                       "l2": "inputs larger than L2 (permuted Q %.0f MB, K %.0f MB, V %.0f MB); no flush"
+                             % (elem * qk_size / 1e6, kv_elem * qk_size / 1e6, kv_elem * 2 / 1e6),
                        "parallelism": f"independent layer per rank x{world}"},
             "ms_per_kernel": {"permute_rope": ms_perm, "hla_forward": ms_attn,
                               "unpermute": ms_unperm if args.unfused else "in hla_forward's epilogue"},

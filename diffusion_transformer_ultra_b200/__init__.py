@@ -4,7 +4,8 @@ The compute lives in ``libultragen.so`` (hand-written CUDA behind a C ABI, see
 ``include/ultragen.h``); this package holds its ctypes binding, the in-tree build script and
 the seeded synthetic-input generator.
 """
-from ._ffi import (BF16, F32, HostRunner, Layer, Plan, UltragenError, hla_forward,  # noqa: F401
+from ._ffi import (BF16, F32, QK_BF16, QK_E4M3, HostRunner, Layer, Plan, UltragenError,  # noqa: F401
+                   hla_forward,
                    hla_forward_noalloc, hla_forward_raster, lib, permute_rope,
                    unpermute, warm_start)
 from .inputs import (WARM_WORKLOADS, WORKLOADS, WarmWorkload, Workload,  # noqa: F401

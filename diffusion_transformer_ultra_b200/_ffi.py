@@ -21,6 +21,7 @@ STATUS = {
     7: "no sm_100 device",
 }
 BF16, F32 = 0, 1
+QK_BF16, QK_E4M3 = 0, 1          # storage of the permuted Q and K (Plan.set_qk_format)
 
 # exported names of include/ultragen.h
 SYMBOLS = (
@@ -32,6 +33,7 @@ SYMBOLS = (
     "ultragen_hla_forward_raster", "ultragen_warm_start", "ultragen_host_runner_create",
     "ultragen_host_runner_forward", "ultragen_host_runner_last_launch_count",
     "ultragen_host_runner_destroy", "ultragen_plan_set_halo", "ultragen_plan_export_kv",
+    "ultragen_plan_set_qk_format",
 )
 
 
@@ -49,7 +51,8 @@ class PlanInfo(ctypes.Structure):
         ("n_split_items", ctypes.c_int32), ("workspace_bytes_per_head", ctypes.c_int64),
         ("lr_radius", ctypes.c_int32), ("halo_copy", ctypes.c_int32),
         ("halo_slots_per_window", ctypes.c_int32), ("N_kv", ctypes.c_int64),
-        ("off_halo", ctypes.c_int64),
+        ("off_halo", ctypes.c_int64), ("qk_format", ctypes.c_int32), ("q_exp", ctypes.c_int32),
+        ("k_exp", ctypes.c_int32),
     ]
 
     def as_dict(self):
@@ -85,6 +88,7 @@ def lib() -> ctypes.CDLL:
     L.ultragen_plan_set_lr_scope.argtypes = [vp, cint]
     L.ultragen_plan_set_halo.argtypes = [vp, cint]
     L.ultragen_plan_export_kv.argtypes = [vp, vp]
+    L.ultragen_plan_set_qk_format.argtypes = [vp, cint, cint, cint]
     L.ultragen_plan_info.argtypes = [vp, ctypes.POINTER(PlanInfo)]
     L.ultragen_plan_export.argtypes = [vp, vp, vp, vp]
     L.ultragen_plan_export_rowmasks.argtypes = [vp, cint, vp]
@@ -149,6 +153,21 @@ class Plan:
         """Compact halo blocks in the K/V layout: 1 on, 0 off, -1 automatic (the default)."""
         _check("ultragen_plan_set_halo", lib().ultragen_plan_set_halo(self._h, int(mode)))
         self._refresh()
+
+    def set_qk_format(self, fmt, q_exp: int = 0, k_exp: int = 0):
+        """Storage of the permuted Q and K: "bf16" (the default) or "e4m3" -- Q and K as e4m3
+        bytes of x * 2^-q_exp and x * 2^-k_exp, multiplied by 8-bit tensor-core products."""
+        code = {"bf16": QK_BF16, "e4m3": QK_E4M3}.get(fmt, fmt)
+        _check("ultragen_plan_set_qk_format",
+               lib().ultragen_plan_set_qk_format(self._h, int(code), int(q_exp), int(k_exp)))
+        self._refresh()
+
+    def qk_dtypes(self):
+        """Tensor dtypes accepted for the permuted Q and K under the plan's Q/K format."""
+        import torch
+        if self.info["qk_format"] == QK_E4M3:
+            return (torch.float8_e4m3fn, torch.uint8)
+        return (torch.bfloat16,)
 
     def export_kv(self):
         kv = np.empty(self.info["N_kv"], np.int32)
@@ -223,9 +242,9 @@ def permute_rope(q, k, v, qp, kp, vp, plan: Plan, stream=None):
         _need(t, raster, (torch.bfloat16, torch.float32), n)
     if not (q.dtype == k.dtype == v.dtype):
         raise ValueError("q, k, v must share a dtype")
-    _need(qp, q_shape, (torch.bfloat16,), "qp")
-    for t, n in ((kp, "kp"), (vp, "vp")):
-        _need(t, kv_shape, (torch.bfloat16,), n)
+    _need(qp, q_shape, plan.qk_dtypes(), "qp")
+    _need(kp, kv_shape, plan.qk_dtypes(), "kp")
+    _need(vp, kv_shape, (torch.bfloat16,), "vp")
     dt = BF16 if q.dtype == torch.bfloat16 else F32
     _check("ultragen_permute_rope", lib().ultragen_permute_rope(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), dt, qp.data_ptr(), kp.data_ptr(), vp.data_ptr(),
@@ -239,10 +258,10 @@ def hla_forward(qp, kp, vp, op, plan: Plan, stream=None):
     B = qp.shape[0]
     shape = (B, i["heads"], i["N_tot"], i["head_dim"])
     kv_shape = (B, i["heads"], i["N_kv"], i["head_dim"])
-    for t, n in ((qp, "qp"), (op, "op")):
-        _need(t, shape, (torch.bfloat16,), n)
-    for t, n in ((kp, "kp"), (vp, "vp")):
-        _need(t, kv_shape, (torch.bfloat16,), n)
+    _need(qp, shape, plan.qk_dtypes(), "qp")
+    _need(op, shape, (torch.bfloat16,), "op")
+    _need(kp, kv_shape, plan.qk_dtypes(), "kp")
+    _need(vp, kv_shape, (torch.bfloat16,), "vp")
     _check("ultragen_hla_forward", lib().ultragen_hla_forward(
         qp.data_ptr(), kp.data_ptr(), vp.data_ptr(), op.data_ptr(), plan.handle, B,
         _stream_ptr(stream)))
@@ -253,9 +272,9 @@ def hla_forward_raster(qp, kp, vp, o, plan: Plan, stream=None):
     import torch
     i = plan.info
     B = qp.shape[0]
-    _need(qp, (B, i["heads"], i["N_tot"], i["head_dim"]), (torch.bfloat16,), "qp")
-    for t, n in ((kp, "kp"), (vp, "vp")):
-        _need(t, (B, i["heads"], i["N_kv"], i["head_dim"]), (torch.bfloat16,), n)
+    _need(qp, (B, i["heads"], i["N_tot"], i["head_dim"]), plan.qk_dtypes(), "qp")
+    _need(kp, (B, i["heads"], i["N_kv"], i["head_dim"]), plan.qk_dtypes(), "kp")
+    _need(vp, (B, i["heads"], i["N_kv"], i["head_dim"]), (torch.bfloat16,), "vp")
     _need(o, (B, i["N_raster"], i["heads"], i["head_dim"]), (torch.bfloat16,), "o")
     _check("ultragen_hla_forward_raster", lib().ultragen_hla_forward_raster(
         qp.data_ptr(), kp.data_ptr(), vp.data_ptr(), o.data_ptr(), plan.handle, B,
@@ -271,10 +290,10 @@ def hla_forward_noalloc(qp, kp, vp, op, plan: Plan, stream=None):
     B = qp.shape[0]
     shape = (B, i["heads"], i["N_tot"], i["head_dim"])
     kv_shape = (B, i["heads"], i["N_kv"], i["head_dim"])
-    for t, n in ((qp, "qp"), (op, "op")):
-        _need(t, shape, (torch.bfloat16,), n)
-    for t, n in ((kp, "kp"), (vp, "vp")):
-        _need(t, kv_shape, (torch.bfloat16,), n)
+    _need(qp, shape, plan.qk_dtypes(), "qp")
+    _need(op, shape, (torch.bfloat16,), "op")
+    _need(kp, kv_shape, plan.qk_dtypes(), "kp")
+    _need(vp, kv_shape, (torch.bfloat16,), "vp")
     _check("ultragen_hla_forward_noalloc", lib().ultragen_hla_forward_noalloc(
         qp.data_ptr(), kp.data_ptr(), vp.data_ptr(), op.data_ptr(), plan.handle, B,
         _stream_ptr(stream)))
@@ -362,8 +381,11 @@ class Layer:
         self.plan = plan
         shape = (batch, i["heads"], i["N_tot"], i["head_dim"])
         kv_shape = (batch, i["heads"], i["N_kv"], i["head_dim"])
-        self.qp, self.op = (torch.empty(shape, dtype=torch.bfloat16, device=device) for _ in range(2))
-        self.kp, self.vp = (torch.empty(kv_shape, dtype=torch.bfloat16, device=device) for _ in range(2))
+        qk = plan.qk_dtypes()[0]
+        self.qp = torch.empty(shape, dtype=qk, device=device)
+        self.op = torch.empty(shape, dtype=torch.bfloat16, device=device)
+        self.kp = torch.empty(kv_shape, dtype=qk, device=device)
+        self.vp = torch.empty(kv_shape, dtype=torch.bfloat16, device=device)
 
     def __call__(self, q, k, v, o, stream=None, fused=None):
         """o: raster [B, N_raster, H, D].  With a bf16 o the unpermute runs inside the

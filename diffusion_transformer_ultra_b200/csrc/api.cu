@@ -133,6 +133,21 @@ int make_tmap(CUtensorMap* m, const void* base, uint64_t rows, int D) {
   return r == CUDA_SUCCESS ? ULTRAGEN_OK : ULTRAGEN_ERR_CUDA;
 }
 
+// 2D view [rows, D] of bytes (e4m3) with [128 x 128] boxes (128-byte rows) and the 128-byte
+// swizzle: the layout the 8-bit S = Q K^T products read (D = 128).
+int make_tmap_u8(CUtensorMap* m, const void* base, uint64_t rows, int D) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || D != 128) return ULTRAGEN_ERR_CUDA;
+  const cuuint64_t dims[2] = {(cuuint64_t)D, rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)D};
+  const cuuint32_t box[2] = {128, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ULTRAGEN_OK : ULTRAGEN_ERR_CUDA;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int sm_count() {
@@ -157,10 +172,16 @@ int launch_attention(const ultragen_plan_t* p, const void* qp, const void* kp, c
   const int64_t rows = (int64_t)units * p->N_tot, kv_rows = (int64_t)units * p->N_kv;
   const int64_t items = (int64_t)units * (int64_t)p->items.size();
   alignas(64) CUtensorMap tq, tk, tv;
+  const int qk8 = p->qk_format == ULTRAGEN_QK_E4M3;
+  if (qk8 && p->D != 128) return ULTRAGEN_ERR_UNSUPPORTED;
   int st;
-  if ((st = make_tmap(&tq, qp, rows, p->D)) || (st = make_tmap(&tk, kp, kv_rows, p->D)) ||
-      (st = make_tmap(&tv, vp, kv_rows, p->D)))
+  if (qk8) {
+    if ((st = make_tmap_u8(&tq, qp, rows, p->D)) || (st = make_tmap_u8(&tk, kp, kv_rows, p->D)))
+      return st;
+  } else if ((st = make_tmap(&tq, qp, rows, p->D)) || (st = make_tmap(&tk, kp, kv_rows, p->D))) {
     return st;
+  }
+  if ((st = make_tmap(&tv, vp, kv_rows, p->D))) return st;
   FwdParams f;
   f.items = p->dev.items;
   f.entries = p->dev.entries;
@@ -177,7 +198,9 @@ int launch_attention(const ultragen_plan_t* p, const void* qp, const void* kp, c
   f.off_hr = (int)p->off_hr;
   f.l2 = p->l * p->l;
   f.n_ws_head = p->n_split_items;
-  f.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)p->D));
+  // log2(e) / sqrt(D), times 2^(q_exp + k_exp) for the scaled e4m3 Q and K
+  f.scale_log2 = (float)(std::ldexp(1.4426950408889634, p->q_exp + p->k_exp) /
+                         std::sqrt((double)p->D));
   f.timeout_ns = p->wait_limit_ns;
   f.fault = p->fault;
   f.raster = raster;
@@ -186,7 +209,7 @@ int launch_attention(const ultragen_plan_t* p, const void* qp, const void* kp, c
   const int grid = (int)std::min<int64_t>(items, sm_count());
   *launches = 0;
   if (grid > 0) {
-    st = cuda_status(launch_hla_fwd(&tq, &tk, &tv, f, p->D, grid, s));
+    st = cuda_status(launch_hla_fwd(&tq, &tk, &tv, f, p->D, qk8, grid, s));
     if (st) return st;
     ++*launches;
   }
@@ -217,9 +240,13 @@ int launch_permute(const ultragen_plan_t* p, const void* q, const void* k, const
                    cudaStream_t s) {
   PermuteArgs a;
   a.in[0] = q; a.in[1] = k; a.in[2] = v;
-  a.out[0] = static_cast<__nv_bfloat16*>(qp);
-  a.out[1] = static_cast<__nv_bfloat16*>(kp);
-  a.out[2] = static_cast<__nv_bfloat16*>(vp);
+  a.out[0] = qp;
+  a.out[1] = kp;
+  a.out[2] = vp;
+  a.qk8 = p->qk_format == ULTRAGEN_QK_E4M3;
+  if (a.qk8 && p->D != 128) return ULTRAGEN_ERR_UNSUPPORTED;
+  a.qk_inv[0] = std::ldexp(1.0f, -p->q_exp);
+  a.qk_inv[1] = std::ldexp(1.0f, -p->k_exp);
   a.perm = p->dev.perm;
   a.slot_pos = p->dev.slot_pos;
   a.rope = p->dev.rope;

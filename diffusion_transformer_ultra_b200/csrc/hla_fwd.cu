@@ -24,6 +24,9 @@
 // P (bf16, packed in pairs) overwrites the first 64 columns of its S block.
 // Shared memory: Q0, Q1, and NS K/V slots, each [128 rows x D] bf16 stored as D/64 boxes of
 // [128 x 64] with the 128-byte swizzle (TMA writes it, the MMA descriptors read it).
+// With 8-bit Q K^T (QK8, D = 128) Q and K tiles are e4m3 bytes, one [128 x 128] box of 128-byte
+// rows at the start of their slot, and S = Q K^T takes 4 kind::f8f6f4 products of 32
+// K-elements instead of 8 kind::f16 products of 16; V, P and O are unchanged.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -99,11 +102,12 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // ------------------------------------------------------------------------ producer warp
-template <int D>
+template <int D, bool QK8>
 __device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
                               const CUtensorMap* tmV, const FwdParams& p, uint32_t sbase,
                               volatile int* abort_flag) {
   using C = FwdCfg<D>;
+  constexpr int QK_BYTES = QK8 ? 128 * D : C::TILE_BYTES;   // one Q or K tile
   const uint32_t sQ = sbase + C::Q_OFF, sKV = sbase + C::KV_OFF, bar = sbase + C::BAR_OFF;
   uint32_t ld = 0, qi = 0;
   bool ok = true;
@@ -118,13 +122,17 @@ __device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
       break;
     }
     const int ntile = qt1 >= 0 ? 2 : 1;
-    mbar_expect_tx(bar + 8 * C::B_QF, ntile * C::TILE_BYTES);
+    mbar_expect_tx(bar + 8 * C::B_QF, ntile * QK_BYTES);
     for (int t = 0; t < ntile; ++t) {
       const int y = bh * p.N_tot + (t ? qt1 : qt0) * 128;
+      if (QK8) {
+        tma_load_2d(sQ + t * C::TILE_BYTES, tmQ, 0, y, bar + 8 * C::B_QF);
+      } else {
 #pragma unroll
-      for (int bx = 0; bx < C::BOXES; ++bx)
-        tma_load_2d(sQ + t * C::TILE_BYTES + bx * C::BOX_BYTES, tmQ, bx * 64, y,
-                    bar + 8 * C::B_QF);
+        for (int bx = 0; bx < C::BOXES; ++bx)
+          tma_load_2d(sQ + t * C::TILE_BYTES + bx * C::BOX_BYTES, tmQ, bx * 64, y,
+                      bar + 8 * C::B_QF);
+      }
     }
     ++qi;
     for (int e = e0; e < e1 && ok; ++e) {
@@ -137,11 +145,16 @@ __device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
           ok = false;
           break;
         }
-        mbar_expect_tx(bar + 8 * (C::B_KVF + s), C::TILE_BYTES);
+        if (QK8 && !which) {
+          mbar_expect_tx(bar + 8 * (C::B_KVF + s), QK_BYTES);
+          tma_load_2d(sKV + s * C::TILE_BYTES, tmK, 0, y, bar + 8 * (C::B_KVF + s));
+        } else {
+          mbar_expect_tx(bar + 8 * (C::B_KVF + s), C::TILE_BYTES);
 #pragma unroll
-        for (int bx = 0; bx < C::BOXES; ++bx)
-          tma_load_2d(sKV + s * C::TILE_BYTES + bx * C::BOX_BYTES, which ? tmV : tmK, bx * 64, y,
-                      bar + 8 * (C::B_KVF + s));
+          for (int bx = 0; bx < C::BOXES; ++bx)
+            tma_load_2d(sKV + s * C::TILE_BYTES + bx * C::BOX_BYTES, which ? tmV : tmK, bx * 64,
+                        y, bar + 8 * (C::B_KVF + s));
+        }
         ++ld;
       }
     }
@@ -160,15 +173,24 @@ __device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
 }
 
 // ------------------------------------------------------------------------ MMA warp
-template <int D>
+template <int D, bool QK8>
 __device__ __forceinline__ void issue_s(uint32_t tmem_d, uint32_t sQt, uint32_t sK) {
   using C = FwdCfg<D>;
-  constexpr uint32_t idS = idesc_bf16(128, 128, 0);
+  if (QK8) {
+    // e4m3 rows of 128 bytes: each product takes the next 32 bytes (32 K-elements) of the row
+    constexpr uint32_t idS = idesc_e4m3(128, 128);
 #pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t off = (kk / 4) * C::BOX_BYTES + (kk % 4) * 32;
-    mma_ss(tmem_d, smem_desc_sw128(sQt + off, 16, 1024), smem_desc_sw128(sK + off, 16, 1024), idS,
-           kk > 0 ? 1u : 0u);
+    for (int kk = 0; kk < D / 32; ++kk)
+      mma_ss_f8(tmem_d, smem_desc_sw128(sQt + kk * 32, 16, 1024),
+                smem_desc_sw128(sK + kk * 32, 16, 1024), idS, kk > 0 ? 1u : 0u);
+  } else {
+    constexpr uint32_t idS = idesc_bf16(128, 128, 0);
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint32_t off = (kk / 4) * C::BOX_BYTES + (kk % 4) * 32;
+      mma_ss(tmem_d, smem_desc_sw128(sQt + off, 16, 1024), smem_desc_sw128(sK + off, 16, 1024),
+             idS, kk > 0 ? 1u : 0u);
+    }
   }
 }
 
@@ -184,7 +206,7 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem_d, uint32_t tmem_p, uint3
   }
 }
 
-template <int D>
+template <int D, bool QK8>
 __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t tbase,
                          volatile int* abort_flag) {
   using C = FwdCfg<D>;
@@ -208,7 +230,7 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t tbase,
       if (!wait(C::B_KVF + s, (ld / C::NS) & 1)) { ok = false; break; }
       tc_fence_after();
       for (int t = 0; t < ntile; ++t) {
-        issue_s<D>(tbase + 128 * t, sQ + t * C::TILE_BYTES, sKV + s * C::TILE_BYTES);
+        issue_s<D, QK8>(tbase + 128 * t, sQ + t * C::TILE_BYTES, sKV + s * C::TILE_BYTES);
         if (withhold && t == 0) {
           withhold = false;     // nothing completes this barrier: its waiters time out
         } else {
@@ -231,7 +253,7 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t tbase,
         ++pc;
         tc_fence_after();
         issue_pv<D>(tbase + C::O_COL + D * t, tbase + 128 * t, sKV + sv * C::TILE_BYTES, j > 1);
-        issue_s<D>(tbase + 128 * t, sQ + t * C::TILE_BYTES, sKV + sk * C::TILE_BYTES);
+        issue_s<D, QK8>(tbase + 128 * t, sQ + t * C::TILE_BYTES, sKV + sk * C::TILE_BYTES);
         mma_commit(bar + 8 * (C::B_SF + t));
       }
       if (!ok) break;
@@ -440,7 +462,7 @@ __device__ void softmax_role(const FwdParams& p, uint32_t sbase, uint32_t tbase,
 }
 
 // ------------------------------------------------------------------------ kernel
-template <int D>
+template <int D, bool QK8>
 __global__ void __launch_bounds__(kThreads, 1)
     hla_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -487,9 +509,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp >= 8) {
     regs_shrink<kRegsControl>();
     if (warp == kWarpProducer) {
-      if (lane == 0) producer_role<D>(&tmQ, &tmK, &tmV, p, sbase, abort_flag);
+      if (lane == 0) producer_role<D, QK8>(&tmQ, &tmK, &tmV, p, sbase, abort_flag);
     } else if (warp == kWarpMma) {
-      if (lane == 0) mma_role<D>(p, sbase, tbase, abort_flag);
+      if (lane == 0) mma_role<D, QK8>(p, sbase, tbase, abort_flag);
     }
   } else {
     regs_grow<kRegsSoftmax>();
@@ -505,7 +527,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D>
+template <int D, bool QK8>
 static cudaError_t launch_d(const void* tmQ, const void* tmK, const void* tmV, const FwdParams& p,
                             int grid, cudaStream_t st) {
   static bool attr_set = false;
@@ -514,23 +536,28 @@ static cudaError_t launch_d(const void* tmQ, const void* tmK, const void* tmV, c
     // The register split above is only sound if the kernel really launches with
     // kRegsLaunch registers per thread; refuse to launch otherwise.
     cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, hla_fwd_kernel<D>);
+    cudaError_t e = cudaFuncGetAttributes(&fa, hla_fwd_kernel<D, QK8>);
     if (e != cudaSuccess) return e;
     if (fa.numRegs != kRegsLaunch) return cudaErrorInvalidConfiguration;
-    e = cudaFuncSetAttribute(hla_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    e = cudaFuncSetAttribute(hla_fwd_kernel<D, QK8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  hla_fwd_kernel<D><<<grid, kThreads, smem, st>>>(*static_cast<const CUtensorMap*>(tmQ),
-                                                   *static_cast<const CUtensorMap*>(tmK),
-                                                   *static_cast<const CUtensorMap*>(tmV), p);
+  hla_fwd_kernel<D, QK8><<<grid, kThreads, smem, st>>>(*static_cast<const CUtensorMap*>(tmQ),
+                                                        *static_cast<const CUtensorMap*>(tmK),
+                                                        *static_cast<const CUtensorMap*>(tmV), p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_hla_fwd(const void* tmQ, const void* tmK, const void* tmV, const FwdParams& p,
-                           int D, int grid, cudaStream_t st) {
-  return D == 128 ? launch_d<128>(tmQ, tmK, tmV, p, grid, st)
-                  : launch_d<64>(tmQ, tmK, tmV, p, grid, st);
+                           int D, int qk8, int grid, cudaStream_t st) {
+  if (qk8) {
+    if (D != 128) return cudaErrorInvalidValue;
+    return launch_d<128, true>(tmQ, tmK, tmV, p, grid, st);
+  }
+  return D == 128 ? launch_d<128, false>(tmQ, tmK, tmV, p, grid, st)
+                  : launch_d<64, false>(tmQ, tmK, tmV, p, grid, st);
 }
 
 }  // namespace ug

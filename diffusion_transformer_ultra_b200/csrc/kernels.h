@@ -27,7 +27,10 @@ struct FastDiv {
 
 struct PermuteArgs {
   const void* in[3];               // q, k, v raster [B, N_raster, heads, D]
-  __nv_bfloat16* out[3];           // qp [B, heads, N_tot, D]; kp, vp [B, heads, N_kv, D]
+  void* out[3];                    // qp [B, heads, N_tot, D]; kp, vp [B, heads, N_kv, D]:
+                                   // bf16, or e4m3 bytes for qp and kp when qk8 is set
+  int qk8;                         // 1: Q and K stored as e4m3 of x * qk_inv[0 / 1]
+  float qk_inv[2];                 // 2^-q_exp, 2^-k_exp
   const int32_t* perm;             // K/V slot -> raster, -1 pad (first N_tot: the Q slots)
   const uint32_t* slot_pos;        // (row_pos << 16) | col_pos per K/V slot
   const float* rope;               // [max(H,W)][D/2][2] (cos, sin)
@@ -103,11 +106,14 @@ cudaError_t launch_unpermute(const UnpermuteArgs& a, int out_dtype, int D, int g
 cudaError_t launch_combine(const CombineArgs& a, int D, cudaStream_t st);
 // 2D bf16 tensor map [rows, D] with [128 x 64] boxes and the 128-byte swizzle (api.cu).
 int make_tmap(CUtensorMap* m, const void* base, uint64_t rows, int D);
+// 2D byte tensor map [rows, D] with [128 x 128] boxes and the 128-byte swizzle (api.cu).
+int make_tmap_u8(CUtensorMap* m, const void* base, uint64_t rows, int D);
 // Streaming multiprocessors of the current device (api.cu).
 int sm_count();
 cudaError_t launch_warm_start(const WarmArgs& a, cudaStream_t st);
 // Launches the block-sparse attention kernel; tensor maps are built by the caller.
+// qk8 = 1: tmQ and tmK are byte maps of e4m3 Q and K (D = 128 only).
 cudaError_t launch_hla_fwd(const void* tmQ, const void* tmK, const void* tmV,
-                           const FwdParams& p, int D, int grid, cudaStream_t st);
+                           const FwdParams& p, int D, int qk8, int grid, cudaStream_t st);
 
 }  // namespace ug

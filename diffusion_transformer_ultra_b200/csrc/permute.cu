@@ -1,11 +1,13 @@
 // HBM-bound passes around the attention:
 //   permute_rope   raster [B, N_raster, H, D] -> window-first [B, H, N_tot, D] bf16, with axial
 //                  2D RoPE on Q and K ("UltraGen ..." papernotes note, 关键设计 1 window-first
-//                  order; 关键设计 2 LR positions (rho m, rho n)).
+//                  order; 关键设计 2 LR positions (rho m, rho n)); optionally Q and K as scaled
+//                  e4m3 bytes (the 8-bit Q K^T format).
 //   unpermute      window-first [B, H, N_tot, D] bf16 -> raster [B, N_raster, H, D].
 //   split combine  log-sum-exp merge of the partial outputs of split query groups.
 // Every thread moves 16-byte chunks (8 bf16) so loads and stores are full-sector.
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -38,6 +40,17 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
+// Eight values times a power of two as e4m3 bytes (nearest even, saturating at +-448), element
+// i in byte i.
+__device__ __forceinline__ uint2 pack_e4m3x8(const float (&x)[8], float s) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    w[i] = __nv_cvt_float2_to_fp8x2(make_float2(x[2 * i] * s, x[2 * i + 1] * s), __NV_SATFINITE,
+                                    __NV_E4M3);
+  return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
+}
+
 }  // namespace
 
 // One thread = one 16-byte chunk of one output row, for Q, K and V together: the row's index
@@ -45,8 +58,8 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 // three loads per row are in flight at once.  Rows are visited in (batch, slot, head) order,
 // so the heads of one token -- contiguous in the raster input -- are read together while
 // each output row is written whole.  (4K layer on B200: 5.9 TB/s with one row per thread,
-// 4.9 TB/s with two, 2.5 TB/s with four.)
-template <typename Tin, int D>
+// 4.9 TB/s with two, 2.5 TB/s with four.)  QK8: Q and K leave as 8 e4m3 bytes per thread.
+template <typename Tin, int D, bool QK8>
 __global__ void __launch_bounds__(256) permute_rope_kernel(PermuteArgs a) {
   constexpr int CH = D / 8;
   constexpr int ROWS = 256 / CH;
@@ -95,6 +108,7 @@ __global__ void __launch_bounds__(256) permute_rope_kernel(PermuteArgs a) {
     for (int u = 0; u < U; ++u) {
       if (dst[u] < 0) continue;
       uint4 oq = make_uint4(0u, 0u, 0u, 0u), ok = oq, ov = oq;
+      uint2 oq8 = make_uint2(0u, 0u), ok8 = oq8;
       if (real[u]) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -110,17 +124,32 @@ __global__ void __launch_bounds__(256) permute_rope_kernel(PermuteArgs a) {
             xk[u][2 * k + 1] = k0 * cs.y + k1 * cs.x;
           }
         }
-        oq = make_uint4(pack_bf16(xq[u][0], xq[u][1]), pack_bf16(xq[u][2], xq[u][3]),
-                        pack_bf16(xq[u][4], xq[u][5]), pack_bf16(xq[u][6], xq[u][7]));
-        ok = make_uint4(pack_bf16(xk[u][0], xk[u][1]), pack_bf16(xk[u][2], xk[u][3]),
-                        pack_bf16(xk[u][4], xk[u][5]), pack_bf16(xk[u][6], xk[u][7]));
+        if (QK8) {
+          oq8 = pack_e4m3x8(xq[u], a.qk_inv[0]);
+          ok8 = pack_e4m3x8(xk[u], a.qk_inv[1]);
+        } else {
+          oq = make_uint4(pack_bf16(xq[u][0], xq[u][1]), pack_bf16(xq[u][2], xq[u][3]),
+                          pack_bf16(xq[u][4], xq[u][5]), pack_bf16(xq[u][6], xq[u][7]));
+          ok = make_uint4(pack_bf16(xk[u][0], xk[u][1]), pack_bf16(xk[u][2], xk[u][3]),
+                          pack_bf16(xk[u][4], xk[u][5]), pack_bf16(xk[u][6], xk[u][7]));
+        }
         ov = make_uint4(pack_bf16(xv[u][0], xv[u][1]), pack_bf16(xv[u][2], xv[u][3]),
                         pack_bf16(xv[u][4], xv[u][5]), pack_bf16(xv[u][6], xv[u][7]));
       }
-      const int64_t o = (int64_t)dst[u] * D + c * 8;
-      if (dq[u] >= 0) *reinterpret_cast<uint4*>(a.out[0] + (int64_t)dq[u] * D + c * 8) = oq;
-      *reinterpret_cast<uint4*>(a.out[1] + o) = ok;
-      *reinterpret_cast<uint4*>(a.out[2] + o) = ov;
+      const int64_t o = (int64_t)dst[u] * D + c * 8;   // element offset of the chunk
+      __nv_bfloat16* const vout = static_cast<__nv_bfloat16*>(a.out[2]);
+      if (QK8) {
+        uint8_t* const qout = static_cast<uint8_t*>(a.out[0]);
+        uint8_t* const kout = static_cast<uint8_t*>(a.out[1]);
+        if (dq[u] >= 0) *reinterpret_cast<uint2*>(qout + (int64_t)dq[u] * D + c * 8) = oq8;
+        *reinterpret_cast<uint2*>(kout + o) = ok8;
+      } else {
+        __nv_bfloat16* const qout = static_cast<__nv_bfloat16*>(a.out[0]);
+        __nv_bfloat16* const kout = static_cast<__nv_bfloat16*>(a.out[1]);
+        if (dq[u] >= 0) *reinterpret_cast<uint4*>(qout + (int64_t)dq[u] * D + c * 8) = oq;
+        *reinterpret_cast<uint4*>(kout + o) = ok;
+      }
+      *reinterpret_cast<uint4*>(vout + o) = ov;
       if (a.halo_ptr && real[u]) {
         // copies into the halo blocks of the neighbouring windows
         const int slot = dst[u] - (dst[u] / a.N_kv) * a.N_kv;
@@ -130,8 +159,11 @@ __global__ void __launch_bounds__(256) permute_rope_kernel(PermuteArgs a) {
           const int e1 = __ldg(a.halo_ptr + k + 1);
           for (int e = __ldg(a.halo_ptr + k); e < e1; ++e) {
             const int64_t oh = (int64_t)(base + __ldg(a.halo_dst + e)) * D + c * 8;
-            *reinterpret_cast<uint4*>(a.out[1] + oh) = ok;
-            *reinterpret_cast<uint4*>(a.out[2] + oh) = ov;
+            if (QK8)
+              *reinterpret_cast<uint2*>(static_cast<uint8_t*>(a.out[1]) + oh) = ok8;
+            else
+              *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out[1]) + oh) = ok;
+            *reinterpret_cast<uint4*>(vout + oh) = ov;
           }
         }
       }
@@ -242,12 +274,16 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
 cudaError_t launch_permute_rope(const PermuteArgs& a, int in_dtype, int D, int grid_x,
                                 cudaStream_t st) {
   dim3 grid(grid_x, 1);
-  if (D == 128) {
-    if (in_dtype == 0) permute_rope_kernel<__nv_bfloat16, 128><<<grid, 256, 0, st>>>(a);
-    else permute_rope_kernel<float, 128><<<grid, 256, 0, st>>>(a);
+  if (a.qk8) {
+    if (D != 128) return cudaErrorInvalidValue;
+    if (in_dtype == 0) permute_rope_kernel<__nv_bfloat16, 128, true><<<grid, 256, 0, st>>>(a);
+    else permute_rope_kernel<float, 128, true><<<grid, 256, 0, st>>>(a);
+  } else if (D == 128) {
+    if (in_dtype == 0) permute_rope_kernel<__nv_bfloat16, 128, false><<<grid, 256, 0, st>>>(a);
+    else permute_rope_kernel<float, 128, false><<<grid, 256, 0, st>>>(a);
   } else {
-    if (in_dtype == 0) permute_rope_kernel<__nv_bfloat16, 64><<<grid, 256, 0, st>>>(a);
-    else permute_rope_kernel<float, 64><<<grid, 256, 0, st>>>(a);
+    if (in_dtype == 0) permute_rope_kernel<__nv_bfloat16, 64, false><<<grid, 256, 0, st>>>(a);
+    else permute_rope_kernel<float, 64, false><<<grid, 256, 0, st>>>(a);
   }
   return cudaGetLastError();
 }

@@ -589,6 +589,18 @@ int ultragen_plan_set_halo(ultragen_plan_t* p, int mode) {
   return ULTRAGEN_OK;
 }
 
+int ultragen_plan_set_qk_format(ultragen_plan_t* p, int format, int q_exp, int k_exp) {
+  if (!p || (format != ULTRAGEN_QK_BF16 && format != ULTRAGEN_QK_E4M3) ||
+      q_exp < -ULTRAGEN_QK_EXP_MAX || q_exp > ULTRAGEN_QK_EXP_MAX ||
+      k_exp < -ULTRAGEN_QK_EXP_MAX || k_exp > ULTRAGEN_QK_EXP_MAX)
+    return ULTRAGEN_ERR_INVALID_ARG;
+  if (format == ULTRAGEN_QK_E4M3 && p->D != 128) return ULTRAGEN_ERR_UNSUPPORTED;
+  p->qk_format = format;
+  p->q_exp = format == ULTRAGEN_QK_E4M3 ? q_exp : 0;
+  p->k_exp = format == ULTRAGEN_QK_E4M3 ? k_exp : 0;
+  return ULTRAGEN_OK;
+}
+
 int ultragen_plan_info(const ultragen_plan_t* p, ultragen_plan_info_t* o) {
   if (!p || !o) return ULTRAGEN_ERR_INVALID_ARG;
   std::memset(o, 0, sizeof(*o));
@@ -613,6 +625,9 @@ int ultragen_plan_info(const ultragen_plan_t* p, ultragen_plan_info_t* o) {
   o->halo_slots_per_window = (int32_t)p->G;
   o->N_kv = p->N_kv;
   o->off_halo = p->off_halo;
+  o->qk_format = p->qk_format;
+  o->q_exp = p->q_exp;
+  o->k_exp = p->k_exp;
   return ULTRAGEN_OK;
 }
 

@@ -69,6 +69,10 @@ struct ultragen_plan {
   int halo_req = -1;
   int halo_copy = 0;
   int64_t G = 0, N_kv = 0, off_halo = 0;
+  // format of the permuted Q and K: ULTRAGEN_QK_BF16, or ULTRAGEN_QK_E4M3 with the stored
+  // values x * 2^-q_exp (Q) and x * 2^-k_exp (K)
+  int qk_format = 0;
+  int q_exp = 0, k_exp = 0;
   // diagnostics: device wait limit and injected fault (ultragen_plan_set_diagnostics)
   unsigned long long wait_limit_ns = 2000ull * 1000 * 1000;
   int fault = 0;

@@ -55,6 +55,10 @@ enum ultragen_status {
 
 enum ultragen_dtype { ULTRAGEN_BF16 = 0, ULTRAGEN_F32 = 1 };
 
+/* Storage of the permuted Q and K (ultragen_plan_set_qk_format). */
+enum ultragen_qk_format { ULTRAGEN_QK_BF16 = 0, ULTRAGEN_QK_E4M3 = 1 };
+#define ULTRAGEN_QK_EXP_MAX 32   /* |q_exp|, |k_exp| <= this */
+
 typedef struct ultragen_plan ultragen_plan_t;   /* opaque, owned by the library */
 
 typedef struct {
@@ -80,6 +84,8 @@ typedef struct {
   int32_t halo_slots_per_window; /* G: slots of one window's halo block (0 without)      */
   int64_t N_kv;               /* K/V slots: N_tot + nWh * nWw * G                        */
   int64_t off_halo;           /* first halo-block slot (= N_tot)                         */
+  int32_t qk_format;          /* ULTRAGEN_QK_BF16 or ULTRAGEN_QK_E4M3                    */
+  int32_t q_exp, k_exp;       /* e4m3 scale exponents (0 for bf16)                       */
 } ultragen_plan_info_t;
 
 /* Human-readable name of a status code.  Never NULL. */
@@ -134,6 +140,21 @@ int ultragen_plan_set_lr_scope(ultragen_plan_t* plan, int radius);
  * Rebuilds the tile lists; changes N_kv.  INVALID_ARG for another mode. */
 int ultragen_plan_set_halo(ultragen_plan_t* plan, int mode);
 
+/* Storage format of the permuted Q and K, and so the precision of the logits Q K^T (no
+ * counterpart in the pages, which only place the permuted layout next to SageAttention's
+ * tiling, [UG-note] 关键设计 1).
+ *   format ULTRAGEN_QK_BF16 (the default): bf16 Q and K, bf16 tensor-core products.
+ *   format ULTRAGEN_QK_E4M3: ultragen_permute_rope stores each RoPE'd element x of Q as the
+ *     e4m3 byte nearest to x * 2^-q_exp (of K: x * 2^-k_exp), ties to even, saturating at
+ *     +-448 (cvt.rn.satfinite); the attention forms Q K^T from those bytes with 8-bit
+ *     tensor-core products (tcgen05 kind::f8f6f4, fp32 accumulation) and multiplies the logits
+ *     by 2^(q_exp + k_exp) / sqrt(head_dim).  V, the softmax and P V keep bf16 / fp32.  Choose
+ *     the exponents so that |x| * 2^-exp stays below 448 (0 suits RMS-normalised activations).
+ * The permuted Q and K buffers then hold one byte per element ([batch, heads, N_tot, D] and
+ * [batch, heads, N_kv, D] bytes).  The tile lists do not change.  INVALID_ARG for another
+ * format or |exp| > ULTRAGEN_QK_EXP_MAX; UNSUPPORTED for E4M3 with head_dim 64. */
+int ultragen_plan_set_qk_format(ultragen_plan_t* plan, int format, int q_exp, int k_exp);
+
 int ultragen_plan_info(const ultragen_plan_t* plan, ultragen_plan_info_t* out);
 
 /*
@@ -168,7 +189,9 @@ int ultragen_plan_destroy(ultragen_plan_t* plan);
  *   kp, vp      [batch, heads, N_kv, head_dim] BF16 (device): the N_tot slots, then the
  *               halo blocks (each halo token's row again, with its own RoPE position)
  * RoPE is computed in fp32 from fp32 tables and rounded to bf16 (nearest even); V and
- * text tokens are copied (F32 input: rounded to bf16).
+ * text tokens are copied (F32 input: rounded to bf16).  With the plan's Q/K format set to
+ * ULTRAGEN_QK_E4M3, qp and kp receive e4m3 bytes instead: the fp32 RoPE result times
+ * 2^-q_exp (2^-k_exp), rounded to nearest even and saturated at +-448; vp stays BF16.
  */
 int ultragen_permute_rope(const void* q, const void* k, const void* v, int in_dtype,
                           void* qp, void* kp, void* vp, int batch,
@@ -180,7 +203,9 @@ int ultragen_permute_rope(const void* q, const void* k, const void* v, int in_dt
  * permuted layout, visiting only the key tiles of each query tile's list.
  *   qp, op  [batch, heads, N_tot, head_dim] BF16 (device); op rows of pad slots = 0
  *   kp, vp  [batch, heads, N_kv, head_dim] BF16 (device), as ultragen_permute_rope writes them
- * bf16 tensor-core products with fp32 accumulation and fp32 online softmax.  Uses the
+ * bf16 tensor-core products with fp32 accumulation and fp32 online softmax (with the
+ * plan's Q/K format ULTRAGEN_QK_E4M3: qp and kp are e4m3 bytes and Q K^T uses 8-bit
+ * products, see ultragen_plan_set_qk_format).  Uses the
  * plan's split workspace (device memory the plan allocates and keeps) when the plan
  * splits groups; a call that needs more than the plan holds grows it with stream-ordered
  * allocation on `stream` (cudaFreeAsync / cudaMallocAsync from the device's default pool),
@@ -192,8 +217,9 @@ int ultragen_hla_forward(const void* qp, const void* kp, const void* vp, void* o
 /*
  * ultragen_hla_forward_raster -- ultragen_hla_forward with the unpermute folded into its
  * epilogue: each output row goes straight to its raster place.
- *   qp          [batch, heads, N_tot, head_dim] BF16 (device, permuted)
- *   kp, vp      [batch, heads, N_kv, head_dim] BF16 (device, K/V layout)
+ *   qp          [batch, heads, N_tot, head_dim] BF16, or e4m3 bytes (device, permuted)
+ *   kp, vp      [batch, heads, N_kv, head_dim] BF16 (kp: e4m3 bytes with the E4M3 Q/K
+ *               format) (device, K/V layout)
  *   o           [batch, N_raster, heads, head_dim] BF16 (device, raster); pad slots write nothing
  * Same arithmetic as ultragen_hla_forward + ultragen_unpermute (bit for bit), one pass less
  * over HBM.  Errors as ultragen_hla_forward.

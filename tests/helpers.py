@@ -25,15 +25,16 @@ def check_attention(got, ref, what=""):
     return max_abs, mean_rel
 
 
-def oracle_rows(q, k, v, wl, b, heads, rows, lr_radius=-1):
-    """Oracle output [len(heads), len(rows), D] for batch b, the given heads and permuted rows."""
+def oracle_rows(q, k, v, wl, b, heads, rows, lr_radius=-1, **fwd):
+    """Oracle output [len(heads), len(rows), D] for batch b, the given heads and permuted rows
+    (``fwd``: further options of the oracle's forward, e.g. the Q/K format)."""
     g = geometry(wl, lr_radius)
     out = []
     for h in heads:
         qh = to_np64(q[b:b + 1, :, h:h + 1, :])
         kh = to_np64(k[b:b + 1, :, h:h + 1, :])
         vh = to_np64(v[b:b + 1, :, h:h + 1, :])
-        o, _ = O.forward(qh, kh, vh, g, wl.axes, rows=rows)
+        o, _ = O.forward(qh, kh, vh, g, wl.axes, rows=rows, **fwd)
         out.append(o[0, 0])
     return np.stack(out)
 

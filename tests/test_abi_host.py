@@ -184,6 +184,32 @@ def test_plan_bit_exact_full(ffi, name, halo):
     assert p.info["useful_pairs"] == O.visible_pair_count(g)
 
 
+def test_qk_format_argument_checks(ffi):
+    """The Q/K storage format: validated on the host, kept across plan rebuilds, and the
+    bf16 format carries no exponents."""
+    L = ffi.lib()
+    p = ffi.Plan(64, 64, 16, 4, 4, 512, 2, 128)
+    assert p.info["qk_format"] == ffi.QK_BF16 and p.info["q_exp"] == p.info["k_exp"] == 0
+    assert L.ultragen_plan_set_qk_format(None, 1, 0, 0) == 1
+    assert L.ultragen_plan_set_qk_format(p.handle, 2, 0, 0) == 1
+    assert L.ultragen_plan_set_qk_format(p.handle, -1, 0, 0) == 1
+    assert L.ultragen_plan_set_qk_format(p.handle, 1, 33, 0) == 1
+    assert L.ultragen_plan_set_qk_format(p.handle, 1, 0, -33) == 1
+    p.set_qk_format("e4m3", -32, 32)
+    assert (p.info["qk_format"], p.info["q_exp"], p.info["k_exp"]) == (ffi.QK_E4M3, -32, 32)
+    entries = p.info["n_entries"]
+    p.set_halo(1)
+    p.set_split(3)
+    assert p.info["n_entries"] < entries                # the halo blocks rebuilt the lists
+    assert (p.info["qk_format"], p.info["q_exp"], p.info["k_exp"]) == (ffi.QK_E4M3, -32, 32)
+    p.set_qk_format("bf16", 5, 5)
+    assert (p.info["qk_format"], p.info["q_exp"], p.info["k_exp"]) == (ffi.QK_BF16, 0, 0)
+    # e4m3 products read 128-byte rows: head_dim 64 is not supported
+    q = ffi.Plan(64, 64, 16, 4, 4, 512, 2, 64)
+    assert L.ultragen_plan_set_qk_format(q.handle, 1, 0, 0) == 2
+    q.set_qk_format("bf16")
+
+
 def test_halo_mode_argument_checks_and_auto_choice(ffi):
     p = ffi.Plan(64, 64, 16, 4, 4, 512, 2, 64)
     assert ffi.lib().ultragen_plan_set_halo(p.handle, 2) == 1
