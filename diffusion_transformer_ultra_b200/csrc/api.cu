@@ -30,7 +30,8 @@ int upload(T** dst, const std::vector<T>& src) {
 void free_device(ultragen_plan_t* p) {
   DeviceTables& d = p->dev;
   void* ptrs[] = {d.items, d.entries, d.mask_off, d.mask_pool, d.perm, d.inv_perm,
-                  d.slot_pos, d.halo_ptr, d.halo_dst, d.rope, d.combine, d.error, d.ws};
+                  d.slot_pos, d.halo_ptr, d.halo_dst, d.halo_pad, d.rope, d.combine, d.error,
+                  d.ws};
   for (void* q : ptrs)
     if (q) cudaFree(q);
   d = DeviceTables();
@@ -75,7 +76,8 @@ int ensure_device(ultragen_plan_t* p) {
       (st = upload(&d.mask_off, p->mask_off)) || (st = upload(&d.mask_pool, p->mask_pool)) ||
       (st = upload(&d.perm, p->perm)) || (st = upload(&d.inv_perm, p->inv_perm)) ||
       (st = upload(&d.slot_pos, p->slot_pos)) || (st = upload(&d.halo_ptr, p->halo_ptr)) ||
-      (st = upload(&d.halo_dst, p->halo_dst)) || (st = upload(&d.rope, rope)) ||
+      (st = upload(&d.halo_dst, p->halo_dst)) || (st = upload(&d.halo_pad, p->halo_pad)) ||
+      (st = upload(&d.rope, rope)) ||
       (st = upload(&d.combine, comb)) || (st = upload(&d.error, std::vector<int>(1, 0)))) {
     free_device(p);
     return st;
@@ -250,13 +252,17 @@ int launch_permute(const ultragen_plan_t* p, const void* q, const void* k, const
   a.perm = p->dev.perm;
   a.slot_pos = p->dev.slot_pos;
   a.rope = p->dev.rope;
-  a.rows_total = (int64_t)batch * heads * p->N_kv;
+  // rows: every Q slot, then the pad slots of the halo blocks (their token slots are written
+  // with their source rows)
+  const int64_t n_pad = p->halo_copy ? (int64_t)p->halo_pad.size() : 0;
+  a.rows_total = (int64_t)batch * heads * (p->N_tot + n_pad);
   a.N_tot = (int)p->N_tot;
   a.N_kv = (int)p->N_kv;
+  a.halo_pad = p->dev.halo_pad;
+  a.div_rows = FastDiv((uint32_t)(p->N_tot + n_pad));
   a.N_raster = (int)p->N_raster;
   a.heads = heads;
   a.div_heads = FastDiv((uint32_t)heads);
-  a.div_nkv = FastDiv((uint32_t)p->N_kv);
   a.pair_a0 = p->axes[0] / 2;
   a.pair_a01 = (p->axes[0] + p->axes[1]) / 2;
   a.halo_ptr = p->halo_copy ? p->dev.halo_ptr : nullptr;

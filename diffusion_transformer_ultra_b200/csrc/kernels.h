@@ -34,9 +34,10 @@ struct PermuteArgs {
   const int32_t* perm;             // K/V slot -> raster, -1 pad (first N_tot: the Q slots)
   const uint32_t* slot_pos;        // (row_pos << 16) | col_pos per K/V slot
   const float* rope;               // [max(H,W)][D/2][2] (cos, sin)
-  int64_t rows_total;              // B * heads * N_kv
+  int64_t rows_total;              // B * heads * (N_tot + number of halo pad slots)
   int N_tot, N_kv, N_raster, heads;
-  FastDiv div_heads, div_nkv;
+  FastDiv div_heads, div_rows;     // by heads, by N_tot + number of halo pad slots
+  const int32_t* halo_pad;         // halo-block pad slots (rows past N_tot of each (b, h))
   // halo blocks (null when the plan has none): the halo-block copies of window-segment slot
   // off_hr + k are halo_dst[halo_ptr[k] .. halo_ptr[k+1]); the kernel writes them from the same
   // read, and writes only the pad slots of the halo region itself

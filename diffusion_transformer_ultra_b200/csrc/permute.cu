@@ -57,7 +57,9 @@ __device__ __forceinline__ uint2 pack_e4m3x8(const float (&x)[8], float s) {
 // decode and its cos/sin values (the same for Q and K) are shared by the three tensors, and
 // three loads per row are in flight at once.  Rows are visited in (batch, slot, head) order,
 // so the heads of one token -- contiguous in the raster input -- are read together while
-// each output row is written whole.  (4K layer on B200: 5.9 TB/s with one row per thread,
+// each output row is written whole.  The walk covers the N_tot Q slots and then only the pad
+// slots of the halo blocks: a halo block's token slots are written from the source token's
+// row, whose halo-copy list (CSR bounds and first target) is loaded together with the row.  (4K layer on B200: 5.9 TB/s with one row per thread,
 // 4.9 TB/s with two, 2.5 TB/s with four.)  QK8: Q and K leave as 8 e4m3 bytes per thread.
 template <typename Tin, int D, bool QK8>
 __global__ void __launch_bounds__(256) permute_rope_kernel(PermuteArgs a) {
@@ -77,23 +79,29 @@ __global__ void __launch_bounds__(256) permute_rope_kernel(PermuteArgs a) {
     float xq[U][8], xk[U][8], xv[U][8];
     int pos_r[U], pos_c[U];
     int dst[U];                                       // K/V output row, -1 when out of range
-    int dq[U];                                        // Q output row, -1 for halo-block slots
+    int dq[U];                                        // Q output row, -1 for halo-block pads
+    int hb[U], he[U], h0[U];                          // halo copies: CSR range, first target
+    int kvb[U];                                       // first K/V row of this (b, h)
     bool real[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int row = row0 + u * ROWS + rsub;         // (b, K/V slot, h)
+      const int row = row0 + u * ROWS + rsub;         // (b, slot index, h)
       dst[u] = -1;
       dq[u] = -1;
       real[u] = false;
+      hb[u] = he[u] = h0[u] = kvb[u] = 0;
       if (row >= rows_total) continue;
       const int bs = (int)a.div_heads.div((uint32_t)row);
       const int h = row - bs * a.heads;
-      const int b = (int)a.div_nkv.div((uint32_t)bs);
-      const int slot = bs - b * a.N_kv;
+      const int b = (int)a.div_rows.div((uint32_t)bs);
+      const int idx = bs - b * (int)a.div_rows.d;
+      // indices past N_tot are the halo blocks' pad slots; their token slots are written with
+      // the source token's row below
+      const int slot = idx < a.N_tot ? idx : __ldg(a.halo_pad + (idx - a.N_tot));
       const int r = __ldg(a.perm + slot);
-      if (slot >= a.N_tot && r >= 0) continue;          // a halo copy: written with its source
-      dst[u] = (b * a.heads + h) * a.N_kv + slot;
-      if (slot < a.N_tot) dq[u] = (b * a.heads + h) * a.N_tot + slot;
+      kvb[u] = (b * a.heads + h) * a.N_kv;
+      dst[u] = kvb[u] + slot;
+      if (idx < a.N_tot) dq[u] = (b * a.heads + h) * a.N_tot + slot;
       if (r < 0) continue;
       real[u] = true;
       const uint32_t sp = __ldg(a.slot_pos + slot);
@@ -103,6 +111,12 @@ __global__ void __launch_bounds__(256) permute_rope_kernel(PermuteArgs a) {
       load8(qin + src, xq[u]);
       load8(kin + src, xk[u]);
       load8(vin + src, xv[u]);
+      const int k = slot - a.off_hr;
+      if (a.halo_ptr && k >= 0 && k < a.N_hrp) {
+        hb[u] = __ldg(a.halo_ptr + k);
+        he[u] = __ldg(a.halo_ptr + k + 1);
+        if (he[u] > hb[u]) h0[u] = __ldg(a.halo_dst + hb[u]);
+      }
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
@@ -150,21 +164,17 @@ __global__ void __launch_bounds__(256) permute_rope_kernel(PermuteArgs a) {
         *reinterpret_cast<uint4*>(kout + o) = ok;
       }
       *reinterpret_cast<uint4*>(vout + o) = ov;
-      if (a.halo_ptr && real[u]) {
-        // copies into the halo blocks of the neighbouring windows
-        const int slot = dst[u] - (dst[u] / a.N_kv) * a.N_kv;
-        const int k = slot - a.off_hr;
-        if (k >= 0 && k < a.N_hrp) {
-          const int base = dst[u] - slot;
-          const int e1 = __ldg(a.halo_ptr + k + 1);
-          for (int e = __ldg(a.halo_ptr + k); e < e1; ++e) {
-            const int64_t oh = (int64_t)(base + __ldg(a.halo_dst + e)) * D + c * 8;
-            if (QK8)
-              *reinterpret_cast<uint2*>(static_cast<uint8_t*>(a.out[1]) + oh) = ok8;
-            else
-              *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out[1]) + oh) = ok;
-            *reinterpret_cast<uint4*>(vout + oh) = ov;
-          }
+      if (he[u] > hb[u]) {
+        // copies into the halo blocks of the neighbouring windows (the first target was loaded
+        // with the row)
+        for (int e = hb[u]; e < he[u]; ++e) {
+          const int tgt = e == hb[u] ? h0[u] : __ldg(a.halo_dst + e);
+          const int64_t oh = (int64_t)(kvb[u] + tgt) * D + c * 8;
+          if (QK8)
+            *reinterpret_cast<uint2*>(static_cast<uint8_t*>(a.out[1]) + oh) = ok8;
+          else
+            *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out[1]) + oh) = ok;
+          *reinterpret_cast<uint4*>(vout + oh) = ov;
         }
       }
     }

@@ -196,6 +196,7 @@ int build_tables_mode(ultragen_plan_t* p, int halo) {
   // permute, each window-segment slot's list of halo-block copies (CSR)
   p->halo_ptr.clear();
   p->halo_dst.clear();
+  p->halo_pad.clear();
   if (halo) {
     std::vector<int32_t> count(p->N_hrp + 1, 0);
     for (int w = 0; w < nW; ++w) {
@@ -211,6 +212,7 @@ int build_tables_mode(ultragen_plan_t* p, int halo) {
         ++count[p->inv_perm[r] - p->off_hr + 1];
         ++s;
       });
+      for (; s < p->off_halo + (int64_t)(w + 1) * p->G; ++s) p->halo_pad.push_back((int32_t)s);
     }
     for (int64_t k = 0; k < p->N_hrp; ++k) count[k + 1] += count[k];
     p->halo_ptr = count;

@@ -40,6 +40,7 @@ struct DeviceTables {
   uint32_t* slot_pos = nullptr;    // (pos_row << 16) | pos_col per K/V slot; 0 for text/pad
   int32_t* halo_ptr = nullptr;     // halo-block copies of each window-segment slot (CSR)
   int32_t* halo_dst = nullptr;
+  int32_t* halo_pad = nullptr;     // pad slots of the halo blocks
   float* rope = nullptr;           // [max(H,W)][head_dim/2][2] (cos, sin)
   int32_t* combine = nullptr;      // CombineGroup[]
   int* error = nullptr;            // device error word
@@ -87,6 +88,7 @@ struct ultragen_plan {
   std::vector<uint32_t> slot_pos;  // per K/V slot packed RoPE positions
   std::vector<int32_t> halo_ptr;   // halo blocks: CSR over window-segment slots (N_hrp + 1) of
   std::vector<int32_t> halo_dst;   //   the halo-block slots that copy the slot's token
+  std::vector<int32_t> halo_pad;   // halo-block slots that hold no token (written as zeros)
   std::vector<int32_t> row_ptr;    // CSR over query tiles
   std::vector<int32_t> entries;    // key tile | partial << 31
   std::vector<int32_t> mask_off;   // per entry: offset into mask_pool, -1 when full
