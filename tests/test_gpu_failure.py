@@ -16,11 +16,13 @@ def ug(gpu_required):
     return pkg
 
 
-def test_withheld_signal_times_out_and_context_survives(ug):
+@pytest.mark.parametrize("qk", ["bf16", "e4m3"])
+def test_withheld_signal_times_out_and_context_survives(ug, qk):
     import torch
     wl = ug.WORKLOADS["1k"]
     q, k, v = (t.cuda() for t in ug.make_qkv(wl))
     plan = ug.plan_for(wl)
+    plan.set_qk_format(qk)
     lay = ug.Layer(plan, wl.batch)
     ug.permute_rope(q, k, v, lay.qp, lay.kp, lay.vp, plan)
     assert plan.sync_status() == 0
@@ -34,6 +36,7 @@ def test_withheld_signal_times_out_and_context_survives(ug):
     ug.hla_forward(lay.qp, lay.kp, lay.vp, lay.op, plan)
     assert plan.sync_status() == 0
     fresh = ug.plan_for(wl)
+    fresh.set_qk_format(qk)
     lay2 = ug.Layer(fresh, wl.batch)
     ug.permute_rope(q, k, v, lay2.qp, lay2.kp, lay2.vp, fresh)
     ug.hla_forward(lay2.qp, lay2.kp, lay2.vp, lay2.op, fresh)
