@@ -30,8 +30,8 @@ int upload(T** dst, const std::vector<T>& src) {
 void free_device(ultragen_plan_t* p) {
   DeviceTables& d = p->dev;
   void* ptrs[] = {d.items, d.entries, d.mask_off, d.mask_pool, d.perm, d.inv_perm,
-                  d.slot_pos, d.halo_ptr, d.halo_dst, d.halo_pad, d.rope, d.combine, d.error,
-                  d.ws};
+                  d.slot_pos, d.halo_ptr, d.halo_dst, d.halo_pad, d.item_order, d.rope,
+                  d.combine, d.error, d.ws};
   for (void* q : ptrs)
     if (q) cudaFree(q);
   d = DeviceTables();
@@ -77,6 +77,7 @@ int ensure_device(ultragen_plan_t* p) {
       (st = upload(&d.perm, p->perm)) || (st = upload(&d.inv_perm, p->inv_perm)) ||
       (st = upload(&d.slot_pos, p->slot_pos)) || (st = upload(&d.halo_ptr, p->halo_ptr)) ||
       (st = upload(&d.halo_dst, p->halo_dst)) || (st = upload(&d.halo_pad, p->halo_pad)) ||
+      (st = upload(&d.item_order, p->item_order)) ||
       (st = upload(&d.rope, rope)) ||
       (st = upload(&d.combine, comb)) || (st = upload(&d.error, std::vector<int>(1, 0)))) {
     free_device(p);
@@ -209,6 +210,12 @@ int launch_attention(const ultragen_plan_t* p, const void* qp, const void* kp, c
   f.N_raster = (int)p->N_raster;
   f.heads = heads;
   const int grid = (int)std::min<int64_t>(items, sm_count());
+  // few items per CTA: hand them out item-major, longest first, so that the last round holds
+  // the short ones; otherwise head-major keeps one head's shared key tiles (its LR segment)
+  // hot in L2 while many CTAs work on it
+  f.item_major = items < 8 * (int64_t)grid ? 1 : 0;
+  f.units = units;
+  f.item_order = p->dev.item_order;
   *launches = 0;
   if (grid > 0) {
     st = cuda_status(launch_hla_fwd(&tq, &tk, &tv, f, p->D, qk8, grid, s));

@@ -101,6 +101,17 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
+// The i-th work item of the launch: its 8-int record and its (batch, head) index.
+__device__ __forceinline__ const int32_t* item_at(const FwdParams& p, int it, int& bh) {
+  if (p.item_major) {
+    const int k = it / p.units;
+    bh = it - k * p.units;
+    return p.items + __ldg(p.item_order + k) * 8;
+  }
+  bh = it / p.n_items_head;
+  return p.items + (it - bh * p.n_items_head) * 8;
+}
+
 // ------------------------------------------------------------------------ producer warp
 template <int D, bool QK8>
 __device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
@@ -112,8 +123,8 @@ __device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
   uint32_t ld = 0, qi = 0;
   bool ok = true;
   for (int it = blockIdx.x; it < p.total_items && ok; it += gridDim.x) {
-    const int32_t* I = p.items + (it % p.n_items_head) * 8;
-    const int bh = it / p.n_items_head;
+    int bh;
+    const int32_t* I = item_at(p, it, bh);
     const int qt0 = I[0], qt1 = I[1], e0 = I[2], e1 = I[3];
     if (e1 == e0) continue;
     if (!mbar_wait(bar + 8 * C::B_QE, (qi & 1) ^ 1, abort_flag, p.err, DEV_TIMEOUT_PRODUCER,
@@ -218,7 +229,9 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t tbase,
   };
   bool ok = true;
   for (int it = blockIdx.x; it < p.total_items && ok; it += gridDim.x) {
-    const int32_t* I = p.items + (it % p.n_items_head) * 8;
+    int bh;
+    const int32_t* I = item_at(p, it, bh);
+    (void)bh;
     const int qt1 = I[1], n = I[3] - I[2];
     if (n == 0) continue;
     const int ntile = qt1 >= 0 ? 2 : 1;
@@ -301,8 +314,8 @@ __device__ void softmax_role(const FwdParams& p, uint32_t sbase, uint32_t tbase,
   uint32_t sc = 0, oc = 0;
 
   for (int it = blockIdx.x; it < p.total_items; it += gridDim.x) {
-    const int32_t* I = p.items + (it % p.n_items_head) * 8;
-    const int bh = it / p.n_items_head;
+    int bh;
+    const int32_t* I = item_at(p, it, bh);
     const int qt = t ? I[1] : I[0];
     if (qt < 0) continue;
     const int e0 = I[2], n = I[3] - I[2], ws_slot = I[4], ncls = I[5], wfirst = I[6];

@@ -76,6 +76,12 @@ struct FwdParams {
   float* ws;                       // split partials [B*heads][n_ws_head][2][128][D+1]
   int* err;                        // device error word
   int n_items_head;
+  // work order: 0 head-major (item i of the layer is item i % n_items_head of (batch, head)
+  // i / n_items_head); 1 item-major over item_order, longest first (item i is item
+  // item_order[i / units] of (batch, head) i % units), used when a layer has few items per CTA
+  int item_major = 0;
+  int units = 1;                   // batch * heads of the launch
+  const int32_t* item_order = nullptr;
   int total_items;
   int N_tot;                       // Q / O rows per (batch, head)
   int N_kv;                        // K / V rows per (batch, head)

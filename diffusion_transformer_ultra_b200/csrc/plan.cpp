@@ -451,6 +451,12 @@ void build_schedule(ultragen_plan_t* p) {
     }
   }
   p->items.insert(p->items.end(), rest.begin(), rest.end());
+  // longest items first, for the item-major order small layers use (ties keep the list order)
+  p->item_order.resize(p->items.size());
+  for (size_t i = 0; i < p->items.size(); ++i) p->item_order[i] = (int32_t)i;
+  std::stable_sort(p->item_order.begin(), p->item_order.end(), [&](int32_t a, int32_t b) {
+    return p->items[a].v[3] - p->items[a].v[2] > p->items[b].v[3] - p->items[b].v[2];
+  });
   p->dirty = true;
 }
 

@@ -41,6 +41,7 @@ struct DeviceTables {
   int32_t* halo_ptr = nullptr;     // halo-block copies of each window-segment slot (CSR)
   int32_t* halo_dst = nullptr;
   int32_t* halo_pad = nullptr;     // pad slots of the halo blocks
+  int32_t* item_order = nullptr;   // items by decreasing key-tile count
   float* rope = nullptr;           // [max(H,W)][head_dim/2][2] (cos, sin)
   int32_t* combine = nullptr;      // CombineGroup[]
   int* error = nullptr;            // device error word
@@ -89,6 +90,7 @@ struct ultragen_plan {
   std::vector<int32_t> halo_ptr;   // halo blocks: CSR over window-segment slots (N_hrp + 1) of
   std::vector<int32_t> halo_dst;   //   the halo-block slots that copy the slot's token
   std::vector<int32_t> halo_pad;   // halo-block slots that hold no token (written as zeros)
+  std::vector<int32_t> item_order; // item indices by decreasing key-tile count (stable)
   std::vector<int32_t> row_ptr;    // CSR over query tiles
   std::vector<int32_t> entries;    // key tile | partial << 31
   std::vector<int32_t> mask_off;   // per entry: offset into mask_pool, -1 when full
