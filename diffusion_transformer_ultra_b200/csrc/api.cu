@@ -8,6 +8,7 @@
 #include <mutex>
 
 #include "kernels.h"
+#include "warm_fused.h"
 #include "plan_internal.h"
 
 namespace ug {
@@ -87,6 +88,68 @@ int ensure_device(ultragen_plan_t* p) {
   d.valid = true;
   p->dirty = false;
   return ULTRAGEN_OK;
+}
+
+// Weights of output phase p of an axis with integer ratio rho (half-pixel centres): output
+// rho k + p interpolates its cell's rows k + o, o in {-1, 0, 1}, as w[o + 1].  The source
+// coordinate relative to row k is (p + 1/2) / rho - 1/2, in (-1/2, 1/2).
+void phase_weights(int rho, int p, double (&w)[3]) {
+  w[0] = w[1] = w[2] = 0.0;
+  const double src = (p + 0.5) / rho - 0.5;
+  const double f0 = std::floor(src);
+  const double f = src - f0;
+  const int o = (int)f0;                   // -1 or 0
+  w[o + 1] += 1.0 - f;
+  w[o + 2] += f;
+}
+
+// Row (ra, rb) and column (ca, cb) weights of the fused warm start: bilinear weights a_p,
+// blurred ones b_p = (a_{p-1} + 2 a_p + a_{p+1}) / 4 (neighbouring phases of the adjacent
+// cells shifted by one row), and the column weights scaled by the sharpening and the blend.
+void warm_weights(WarmFused& a, int ry, float sharpen, float alpha) {
+  auto fill = [](int rho, int p, double (&aw)[3], double (&bw)[3]) {
+    double c[3], u[3], d[3];
+    phase_weights(rho, p, c);
+    // the row above: phase p - 1 of this cell, or phase rho - 1 of the cell above
+    if (p > 0) {
+      phase_weights(rho, p - 1, u);
+    } else {
+      double t[3];
+      phase_weights(rho, rho - 1, t);
+      u[0] = t[1]; u[1] = t[2]; u[2] = 0.0;
+      // t[0] would sit two rows up: phase rho - 1 starts at its own row, so t[0] == 0
+    }
+    if (p + 1 < rho) {
+      phase_weights(rho, p + 1, d);
+    } else {
+      double t[3];
+      phase_weights(rho, 0, t);
+      d[0] = 0.0; d[1] = t[0]; d[2] = t[1];
+      // t[2] would sit two rows down: phase 0 ends at its own row, so t[2] == 0
+    }
+    for (int i = 0; i < 3; ++i) {
+      aw[i] = c[i];
+      bw[i] = (u[i] + 2.0 * c[i] + d[i]) / 4.0;
+    }
+  };
+  a.ry = ry;
+  for (int p = 0; p < ry; ++p) {
+    double aw[3], bw[3];
+    fill(ry, p, aw, bw);
+    for (int i = 0; i < 3; ++i) {
+      a.ra[p][i] = (float)aw[i];
+      a.rb[p][i] = (float)bw[i];
+    }
+  }
+  const double s = sharpen, beta = 1.0 - (double)alpha;
+  for (int q = 0; q < 4; ++q) {
+    double aw[3], bw[3];
+    fill(4, q, aw, bw);
+    for (int j = 0; j < 3; ++j) {
+      a.ca[q][j] = (float)(beta * (1.0 + s) * aw[j]);
+      a.cb[q][j] = (float)(-beta * s * bw[j]);
+    }
+  }
 }
 
 int grid_for(int64_t rows, int rows_per_block) {
@@ -438,7 +501,13 @@ int ultragen_warm_start(const float* x_lr, const float* noise, float* x_hr, int 
   a.seed = seed;
   a.offset = offset;
   a.vec = (W % 4 == 0) && aligned16(x_hr) && (!noise || aligned16(noise));
-  return cuda_status(launch_warm_start(a, reinterpret_cast<cudaStream_t>(stream)));
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (a.vec && W == 4 * w && H % h == 0 && H / h <= 8) {
+    WarmFused f;
+    warm_weights(f, H / h, sharpen, alpha);
+    return cuda_status(launch_warm_start_fused(a, f, s));
+  }
+  return cuda_status(launch_warm_start(a, s));
 }
 
 int ultragen_plan_set_diagnostics(ultragen_plan_t* p, int fault, double wait_limit_s) {

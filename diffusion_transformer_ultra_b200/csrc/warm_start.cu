@@ -24,6 +24,7 @@
 #include <cstdint>
 
 #include "kernels.h"
+#include "warm_fused.h"
 
 namespace ug {
 namespace {
@@ -214,11 +215,79 @@ __global__ void __launch_bounds__(kWarmThreads) warm_start_kernel(const WarmArgs
   }
 }
 
+// Integer ratios (W = 4 w, H = ry h): upsampling, blur, sharpening and the blend are linear
+// and separable, so output (ry k + p, 4 l + q) is
+//   alpha X_T + sum_j ca[q][j] Ra[j] + sum_j cb[q][j] Rb[j],
+//   Ra[j] = sum_i ra[p][i] X(k + i - 1, l + j - 1),  Rb[j] = sum_i rb[p][i] X(k + i - 1, l + j - 1),
+// with X read at clamped indices.  Clamping reproduces both edge rules: a source coordinate
+// clamped at 0 (or a second tap clamped at the last row) reads one value with weights summing
+// to 1, and the blur's replicated edge row equals the upsampled edge row, which is that value.
+// One thread per low-resolution cell: its 3 x 3 neighbourhood, then ry rows of 4 outputs (one
+// 16-byte load of noise and one 16-byte store each); a warp covers 32 cells of one row, so
+// loads and stores are 512-byte runs.
+__global__ void __launch_bounds__(kWarmThreads) warm_start_fused_kernel(const WarmArgs a,
+                                                                        const WarmFused wf) {
+  const int plane = blockIdx.z;
+  const int l = blockIdx.x * 32 + (threadIdx.x & 31);
+  const int k = blockIdx.y * (kWarmThreads / 32) + (threadIdx.x >> 5);
+  if (l >= a.w || k >= a.h) return;
+  const int x = 4 * l;
+  const uint64_t row0 = static_cast<uint64_t>(plane) * a.H + static_cast<uint64_t>(k) * wf.ry;
+  // the noise of the cell's outputs first, so the loads are in flight during the arithmetic
+  float4 nz[8];
+  if (a.noise) {
+#pragma unroll
+    for (int p = 0; p < 8; ++p)
+      if (p < wf.ry)
+        nz[p] = __ldcs(reinterpret_cast<const float4*>(a.noise + (row0 + p) * a.W + x));
+  }
+  const float* L = a.lr + static_cast<size_t>(plane) * a.h * a.w;
+  float X[3][3];
+#pragma unroll
+  for (int i = 0; i < 3; ++i) {
+    const float* row = L + static_cast<size_t>(min(max(k + i - 1, 0), a.h - 1)) * a.w;
+#pragma unroll
+    for (int j = 0; j < 3; ++j) X[i][j] = __ldg(row + min(max(l + j - 1, 0), a.w - 1));
+  }
+  const float alpha = a.alpha;
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    if (p >= wf.ry) break;
+    float Ra[3], Rb[3];
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+      Ra[j] = fmaf(wf.ra[p][2], X[2][j], fmaf(wf.ra[p][1], X[1][j], wf.ra[p][0] * X[0][j]));
+      Rb[j] = fmaf(wf.rb[p][2], X[2][j], fmaf(wf.rb[p][1], X[1][j], wf.rb[p][0] * X[0][j]));
+    }
+    float r[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float acc = wf.ca[q][0] * Ra[0];
+      acc = fmaf(wf.ca[q][1], Ra[1], acc);
+      acc = fmaf(wf.ca[q][2], Ra[2], acc);
+      acc = fmaf(wf.cb[q][0], Rb[0], acc);
+      acc = fmaf(wf.cb[q][1], Rb[1], acc);
+      r[q] = fmaf(wf.cb[q][2], Rb[2], acc);
+    }
+    const uint64_t flat = (row0 + p) * a.W + x;
+    const float4 n = a.noise ? nz[p] : normals4(flat >> 2, a.seed, a.offset);
+    __stcs(reinterpret_cast<float4*>(a.out + flat),
+           make_float4(fmaf(alpha, n.x, r[0]), fmaf(alpha, n.y, r[1]), fmaf(alpha, n.z, r[2]),
+                       fmaf(alpha, n.w, r[3])));
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_warm_start(const WarmArgs& a, cudaStream_t st) {
   const dim3 grid((a.W + kTW - 1) / kTW, (a.H + kTH - 1) / kTH, a.planes);
   warm_start_kernel<<<grid, kWarmThreads, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_warm_start_fused(const WarmArgs& a, const WarmFused& f, cudaStream_t st) {
+  const dim3 grid((a.w + 31) / 32, (a.h + kWarmThreads / 32 - 1) / (kWarmThreads / 32), a.planes);
+  warm_start_fused_kernel<<<grid, kWarmThreads, 0, st>>>(a, f);
   return cudaGetLastError();
 }
 

@@ -137,3 +137,24 @@ def test_warm_start_drawn_noise_is_deterministic_and_seeded(ug):
     assert not torch.equal(a, c)
     z = a.double().numpy().reshape(-1)
     assert abs(z.mean()) < 5 / np.sqrt(z.size) and abs(z.var() - 1) < 5 * np.sqrt(2 / z.size)
+
+
+# integer ratios take the fused kernel (W = 4 w, H = ry h with ry <= 8); the last shape has
+# H % h != 0 and takes the tiled kernel
+FUSED_SHAPES = [(9, 7, 9, 28), (9, 7, 18, 28), (5, 6, 15, 24), (4, 5, 32, 20), (5, 6, 17, 24)]
+
+
+@pytest.mark.parametrize("shape", FUSED_SHAPES)
+@pytest.mark.parametrize("mode", ["given", "drawn"])
+def test_warm_start_integer_ratio_paths(ug, shape, mode):
+    import dataclasses
+    h, w, H, W = shape
+    wl = dataclasses.replace(ug.WARM_WORKLOADS["warm_tiny"], name="warm_ratio", cfg=24, batch=2,
+                             C=3, h=h, w=w, H=H, W=W, alpha=0.4, sharpen=0.8)
+    x_lr, noise, out, alpha, s = run(ug, wl, mode)
+    assert not np.isnan(out.numpy()).any()
+    planes = [(b, c) for b in range(wl.batch) for c in range(wl.C)]
+    ref, nz = oracle_planes(x_lr, H, W, alpha, s, planes,
+                            noise=noise if mode == "given" else None, seed=12345, offset=7)
+    got = np.stack([out[b, c].double().numpy() for b, c in planes])
+    check(got, ref, nz, x_lr, alpha, s, mode == "drawn", f"{shape} {mode}")
