@@ -81,57 +81,107 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    """SM clock, power and throttle reasons of this process's GPU during the timed region.
 
+    NVML (the device found by the CUDA device's UUID, so the reading is of the GPU the
+    kernels run on) is polled every ~5 ms from a thread between start() and stop(); without
+    NVML, nvidia-smi is polled every 20 ms.  start() is called right before the timed steps are
+    enqueued and stop() right after the closing synchronize, so the samples cover the steps."""
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, index: int):
         self.index = index
+        self.samples = []               # (sm_mhz, power_w, reasons)
+        self.smax = None
+        self.stop_evt = threading.Event()
+        self.thread = None
         self.proc = None
-        self.lines = []
+        self.source = None
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        uuid = str(torch.cuda.get_device_properties(self.index).uuid)
+        for cand in (uuid, "GPU-" + uuid):
+            try:
+                return pynvml, pynvml.nvmlDeviceGetHandleByUUID(cand)
+            except Exception:
+                pass
+        raise RuntimeError("no NVML device with the CUDA device's UUID")
 
     def start(self):
         try:
+            nv, h = self._nvml_handle()
+            self.smax = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            masks = [(name, getattr(nv, attr)) for name, attr in self.REASONS]
+
+            def poll():
+                while not self.stop_evt.is_set():
+                    try:
+                        sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                        pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                        bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        self.samples.append((sm, pw, {n for n, m in masks if bits & m}))
+                    except Exception:
+                        pass
+                    time.sleep(0.005)
+
+            self.source = "nvml"
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            pass
+        try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.source = "nvidia-smi"
+            self.thread = threading.Thread(target=self._read_smi, daemon=True)
             self.thread.start()
         except Exception:
             self.proc = None
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
-    def stop(self):
-        if not self.proc:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.thread.join(timeout=2)
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [x.strip() for x in ln.split(",")]
+    def _read_smi(self):
+        names = [n for n, _ in self.REASONS]
+        for ln in self.proc.stdout:
+            parts = [x.strip() for x in ln.strip().split(",")]
             if len(parts) < 9:
                 continue
             try:
-                sm.append(float(parts[1]))
-                smax = float(parts[2])
+                sm, self.smax, pw = float(parts[1]), float(parts[2]), float(parts[3])
             except ValueError:
                 continue
-            for nm, val in zip(names, parts[5:9]):
-                if val.lower() in ("active", "1", "0x1"):
-                    reasons.add(nm)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+            self.samples.append((sm, pw, {n for n, v in zip(names, parts[5:9])
+                                          if v.lower() in ("active", "1", "0x1")}))
+
+    def stop(self):
+        if self.source is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampling unavailable"]}
+        self.stop_evt.set()
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm = [x[0] for x in self.samples]
+        pw = [x[1] for x in self.samples]
+        reasons = set().union(*(x[2] for x in self.samples)) if self.samples else set()
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.smax,
+                "sm_mhz_min": min(sm) if sm else None, "power_w_max": max(pw) if pw else None,
+                "reasons": sorted(reasons), "samples": len(sm), "source": self.source}
 
 
 def max_over_ranks(x: float, world: int, device) -> float:
@@ -318,7 +368,6 @@ def main_warm(args, rank, world, local):
         dist.barrier()
     torch.cuda.synchronize()
     sampler.start()
-    time.sleep(0.3)
     launches = 0
     for i in range(args.steps):
         flush.zero_()
@@ -466,7 +515,6 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     sampler.start()
-    time.sleep(0.3)
     launches = 0
     start.record(stream)
     for i in range(args.steps):
