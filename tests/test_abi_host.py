@@ -326,3 +326,37 @@ def test_plan_at_16k_maximum_size(ffi):
     assert 24 * i["n_items"] < 2 ** 31
     g = O.Geometry(*geom)
     assert (i["N_tot"], i["N_raster"], i["off_hr"], i["off_lr"]) == (g.N_tot, g.N_raster, g.off_hr, g.off_lr)
+
+
+def test_plan_matches_oracle_on_random_geometries(ffi):
+    """60 seeded random small geometries (any H, W, l, b <= l, rho including 0, text length,
+    LR scope, halo mode): layout, K/V slot map, tile lists, partial flags and row masks are
+    bit-exact against the oracle's explicit mask."""
+    rng = np.random.default_rng(2026)
+    for case in range(60):
+        H, W = (int(x) for x in rng.integers(1, 49, 2))
+        l = int(rng.integers(1, 21))
+        b = int(rng.integers(0, l + 1))
+        rho = int(rng.integers(0, 7))
+        T = int(rng.choice([0, 1, 3, 127, 128, 129, 300]))
+        r = int(rng.choice([-1, -1, 0, 2, 5])) if rho else -1
+        halo = [None, 0, 1][case % 3]
+        p = ffi.Plan(H, W, l, b, rho, T, 2, 64)
+        if r >= 0:
+            p.set_lr_scope(r)
+        if halo is not None:
+            p.set_halo(halo)
+        info = p.info
+        g = O.Geometry(H, W, l, b, rho, T, r, halo_copy=bool(info["halo_copy"]))
+        what = f"case {case}: H={H} W={W} l={l} b={b} rho={rho} T={T} r={r} halo={halo}"
+        assert (info["N_tot"], info["N_kv"], info["off_lr"]) == (g.N_tot, g.N_kv, g.off_lr), what
+        perm, row_ptr, entries = p.export()
+        np.testing.assert_array_equal(perm, O.perm_map(g), err_msg=what)
+        np.testing.assert_array_equal(p.export_kv(), O.kv_perm_map(g), err_msg=what)
+        for t in range(g.N_tot // 128):
+            e_ref, m_ref = O.qtile_entries(g, t)
+            e_got = entries[row_ptr[t]:row_ptr[t + 1]].view(np.uint32)
+            np.testing.assert_array_equal(e_got, e_ref, err_msg=f"{what}, q-tile {t}")
+            np.testing.assert_array_equal(p.rowmasks(t, len(e_ref)), m_ref,
+                                          err_msg=f"{what}, q-tile {t} masks")
+        assert info["useful_pairs"] == O.visible_pair_count(g), what
