@@ -54,6 +54,12 @@ Readings taken where the pages are silent or garbled (each is listed in DESIGN.m
       w then takes the other windows' tokens of its box from w's block instead of their
       window segments; halo blocks are visible to nothing else.  Every query sees the same
       tokens as without them, so the attention output is the same function.
+  R20 Optional block order of the LR segment (lr_block; a layout choice for the LR-region
+      reading of R3): LR token (m, n) takes slot off_lr + ((m // 8) * nbw + n // 16) * 128 +
+      (m % 8) * 16 + n % 16, nbw = ceil(w / 16), so every 128-slot tile holds one 8 x 16 block
+      of the LR grid (partial blocks at the bottom and right edges keep their pad slots).  The
+      window-grown LR region of an HR window then falls into a few dense tiles instead of one
+      row per tile.  Every query sees the same tokens, so the attention is the same function.
   R19 Optional 8-bit Q K^T (qk_format = "e4m3"; the pages only place the permuted layout next
       to SageAttention's tiling, [UG-note] 关键设计 1): after RoPE, every element x of Q (of K)
       is stored as the e4m3 value nearest to x * 2^-q_exp (x * 2^-k_exp), ties to even, values
@@ -78,6 +84,7 @@ import numpy as np
 
 TEXT, HR, LR, PAD = 0, 1, 2, -1
 TILE = 128
+LR_BH, LR_BW = 8, 16      # LR block of one tile in the block order (R20)
 
 
 def pad128(n: int) -> int:
@@ -100,6 +107,7 @@ class Geometry:
     T: int          # text tokens
     lr_radius: int = -1   # -1: HR sees all LR (R3); r >= 0: only the window's region grown by r
     halo_copy: bool = False   # K/V carry a compact halo block per window (R18)
+    lr_block: bool = False    # LR segment in 8 x 16 blocks of the LR grid (R20)
 
     @property
     def nWh(self) -> int:
@@ -138,8 +146,15 @@ class Geometry:
         return self.off_hr + pad128(self.N_hrp)
 
     @property
+    def N_lrp(self) -> int:
+        """Slots of the LR segment: padded to 128, or whole 8 x 16 blocks (R20)."""
+        if self.lr_block:
+            return cdiv(self.h, LR_BH) * cdiv(self.w, LR_BW) * TILE
+        return pad128(self.N_lr)
+
+    @property
     def N_tot(self) -> int:
-        return self.off_lr + pad128(self.N_lr)
+        return self.off_lr + self.N_lrp
 
     @property
     def N_raster(self) -> int:
@@ -213,7 +228,13 @@ def slot_of_tokens(g: Geometry) -> np.ndarray:
     window = (i // g.l) * g.nWw + (j // g.l)
     slot[hr] = g.off_hr + window * g.l * g.l + (i % g.l) * g.l + (j % g.l)
     lr = seg == LR
-    slot[lr] = g.off_lr + ca[lr] * g.w + cb[lr]
+    m, n = ca[lr], cb[lr]
+    if g.lr_block:
+        nbw = cdiv(g.w, LR_BW)
+        slot[lr] = (g.off_lr + ((m // LR_BH) * nbw + n // LR_BW) * TILE
+                    + (m % LR_BH) * LR_BW + n % LR_BW)
+    else:
+        slot[lr] = g.off_lr + m * g.w + n
     return slot
 
 

@@ -36,10 +36,11 @@ def bf_tokens(H, W, rho, T):
     return toks
 
 
-def bf_slots(H, W, l, rho, T):
+def bf_slots(H, W, l, rho, T, lr_block=False):
     """Walk the permuted sequence slot by slot: text, pad to 128, windows row-major with
-    raster order inside, pad to 128, LR raster, pad to 128.  Returns list of token keys
-    (None for pad)."""
+    raster order inside, pad to 128, LR raster (or, with lr_block, LR blocks of 8 rows x 16
+    columns row-major, raster order inside, out-of-grid cells as pads), pad to 128.  Returns
+    list of token keys (None for pad)."""
     seq = [("text", t, 0) for t in range(T)]
     while len(seq) % 128:
         seq.append(None)
@@ -51,7 +52,15 @@ def bf_slots(H, W, l, rho, T):
                     seq.append(("hr", i, j) if (i < H and j < W) else None)
     while len(seq) % 128:
         seq.append(None)
-    if rho:
+    if rho and lr_block:
+        h, w = math.ceil(H / rho), math.ceil(W / rho)
+        for bm in range(math.ceil(h / 8)):
+            for bn in range(math.ceil(w / 16)):
+                for i in range(8):
+                    for j in range(16):
+                        m, n = 8 * bm + i, 16 * bn + j
+                        seq.append(("lr", m, n) if (m < h and n < w) else None)
+    elif rho:
         h, w = math.ceil(H / rho), math.ceil(W / rho)
         for m in range(h):
             for n in range(w):
@@ -486,6 +495,38 @@ def test_region_radius_covering_the_image_is_all_lr():
     wide = O.Geometry(20, 24, 8, 2, 4, 7, 64)
     rows = np.arange(base.N_tot)
     np.testing.assert_array_equal(O.visible_rows(base, rows), O.visible_rows(wide, rows))
+
+
+# ------------------------------------------------------------------ LR block order (R20)
+LR_BLOCK_GEOMS = [(40, 72, 8, 2, 2, 9, 3), (19, 23, 8, 3, 3, 9, 1), (64, 64, 16, 4, 4, 512, 4),
+                  (12, 200, 4, 1, 1, 0, 0)]
+
+
+@pytest.mark.parametrize("geom", LR_BLOCK_GEOMS)
+def test_lr_block_slots_match_walk_and_mask(geom):
+    H, W, l, b, rho, T, r = geom
+    g = O.Geometry(H, W, l, b, rho, T, r, lr_block=True)
+    seq = bf_slots(H, W, l, rho, T, lr_block=True)
+    toks = bf_tokens(H, W, rho, T)
+    index = {tok: i for i, tok in enumerate(toks)}
+    assert len(seq) == g.N_tot
+    np.testing.assert_array_equal(O.perm_map(g), [-1 if x is None else index[x] for x in seq])
+    if g.N_tot <= 2048:
+        expect = np.array([[bf_visible(qt, kt, l, b, rho, r) for kt in seq] for qt in seq])
+        np.testing.assert_array_equal(O.visible_rows(g, np.arange(g.N_tot)), expect)
+
+
+@pytest.mark.parametrize("geom", LR_BLOCK_GEOMS[:2])
+def test_lr_block_order_gives_the_same_attention(geom):
+    H, W, l, b, rho, T, r = geom
+    g0 = O.Geometry(H, W, l, b, rho, T, r)
+    g1 = O.Geometry(H, W, l, b, rho, T, r, lr_block=True)
+    assert O.visible_pair_count(g0) == O.visible_pair_count(g1)
+    rng = np.random.default_rng(5)
+    q, k, v = (rng.standard_normal((1, g0.N_raster, 2, 64)) for _ in range(3))
+    o0 = O.unpermute(O.forward(q, k, v, g0, (16, 24, 24))[0], g0)
+    o1 = O.unpermute(O.forward(q, k, v, g1, (16, 24, 24))[0], g1)
+    np.testing.assert_allclose(o1, o0, rtol=0, atol=1e-12)
 
 
 # ------------------------------------------------------------------ compact halo blocks (R18)
