@@ -49,6 +49,8 @@ def parse():
                     help="override the workload's head count (smaller profiling captures)")
     ap.add_argument("--lr-radius", type=int, default=-1,
                     help="HR->LR scope: -1 all LR tokens (default); r >= 0 the window's anchors grown by r")
+    ap.add_argument("--lr-order", type=int, default=-1, choices=[-1, 0, 1],
+                    help="LR segment order with an LR-region scope: -1 automatic (default), 0 raster, 1 8x16 blocks")
     ap.add_argument("--halo", type=int, default=-1, choices=[-1, 0, 1],
                     help="compact halo blocks in the K/V layout: -1 automatic (default), 0 off, 1 on")
     ap.add_argument("--qk", default="bf16", choices=["bf16", "e4m3"],
@@ -221,14 +223,15 @@ def profiled_traffic(workload: str):
     return ent.get("dram_bytes_per_launch")
 
 
-def cpu_baseline(wl, q, k, v, budget_s: float = 12.0, **fwd):
+def cpu_baseline(wl, q, k, v, budget_s: float = 12.0, lr_radius: int = -1, lr_block: bool = False,
+                 **fwd):
     """The oracle as it stands, timed on this host on a bounded sample: one head, rows of one
     interior window plus text and LR rows, growing until about `budget_s` of CPU work
     (``fwd``: the oracle forward's Q/K format options)."""
     import numpy as np
 
     from oracle import hla_oracle as O
-    g = O.Geometry(wl.H, wl.W, wl.l, wl.b, wl.rho, wl.T)
+    g = O.Geometry(wl.H, wl.W, wl.l, wl.b, wl.rho, wl.T, lr_radius, lr_block=lr_block)
     l2 = g.l * g.l
     win = (g.nWh // 2) * g.nWw + g.nWw // 2
     rows = list(range(g.off_hr + win * l2, g.off_hr + (win + 1) * l2))
@@ -469,6 +472,8 @@ def main():
     plan = ug.plan_for(wl)
     if args.lr_radius != -1:
         plan.set_lr_scope(args.lr_radius)
+    if args.lr_order != -1:
+        plan.set_lr_order(args.lr_order)
     if args.halo != -1:
         plan.set_halo(args.halo)
     e4m3 = args.qk == "e4m3"
@@ -576,8 +581,9 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(wl, q, k, v, **({"qk_format": "e4m3", "q_exp": args.q_exp,
-                                            "k_exp": args.k_exp} if e4m3 else {}))
+        cpu = cpu_baseline(wl, q, k, v, lr_radius=args.lr_radius, lr_block=bool(info["lr_block"]),
+                           **({"qk_format": "e4m3", "q_exp": args.q_exp, "k_exp": args.k_exp}
+                              if e4m3 else {}))
 
     # roofline denominator: the burst bf16 figure while the SM clock held its maximum during
     # the timed steps, the sustained (power-capped) one once the clock dropped under the cap
@@ -607,6 +613,7 @@ def main():
                        "rho": wl.rho, "text_len": wl.T, "lr_radius": args.lr_radius, "heads": wl.heads, "head_dim": wl.D,
                        "batch": wl.batch, "N_tot": info["N_tot"], "useful_pairs_per_head": info["useful_pairs"],
                        "halo_blocks": bool(info["halo_copy"]), "N_kv": info["N_kv"],
+                       "lr_blocks": bool(info["lr_block"]),
                        "qk_format": args.qk, **({"q_exp": args.q_exp, "k_exp": args.k_exp} if e4m3 else {}),
                        "l2": "inputs larger than L2 (permuted Q %.0f MB, K %.0f MB, V %.0f MB); no flush"
                              % (elem * qk_size / 1e6, kv_elem * qk_size / 1e6, kv_elem * 2 / 1e6),

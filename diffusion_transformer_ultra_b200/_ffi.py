@@ -33,7 +33,7 @@ SYMBOLS = (
     "ultragen_hla_forward_raster", "ultragen_warm_start", "ultragen_host_runner_create",
     "ultragen_host_runner_forward", "ultragen_host_runner_last_launch_count",
     "ultragen_host_runner_destroy", "ultragen_plan_set_halo", "ultragen_plan_export_kv",
-    "ultragen_plan_set_qk_format",
+    "ultragen_plan_set_qk_format", "ultragen_plan_set_lr_order",
 )
 
 
@@ -52,7 +52,7 @@ class PlanInfo(ctypes.Structure):
         ("lr_radius", ctypes.c_int32), ("halo_copy", ctypes.c_int32),
         ("halo_slots_per_window", ctypes.c_int32), ("N_kv", ctypes.c_int64),
         ("off_halo", ctypes.c_int64), ("qk_format", ctypes.c_int32), ("q_exp", ctypes.c_int32),
-        ("k_exp", ctypes.c_int32),
+        ("k_exp", ctypes.c_int32), ("lr_block", ctypes.c_int32),
     ]
 
     def as_dict(self):
@@ -89,6 +89,7 @@ def lib() -> ctypes.CDLL:
     L.ultragen_plan_set_halo.argtypes = [vp, cint]
     L.ultragen_plan_export_kv.argtypes = [vp, vp]
     L.ultragen_plan_set_qk_format.argtypes = [vp, cint, cint, cint]
+    L.ultragen_plan_set_lr_order.argtypes = [vp, cint]
     L.ultragen_plan_info.argtypes = [vp, ctypes.POINTER(PlanInfo)]
     L.ultragen_plan_export.argtypes = [vp, vp, vp, vp]
     L.ultragen_plan_export_rowmasks.argtypes = [vp, cint, vp]
@@ -147,6 +148,12 @@ class Plan:
 
     def set_lr_scope(self, radius: int):
         _check("ultragen_plan_set_lr_scope", lib().ultragen_plan_set_lr_scope(self._h, int(radius)))
+        self._refresh()
+
+    def set_lr_order(self, mode: int):
+        """LR segment order: 1 blocks of 8 x 16 LR tokens, 0 raster, -1 automatic (the
+        default; blocks only with an LR-region scope, when they give fewer tile entries)."""
+        _check("ultragen_plan_set_lr_order", lib().ultragen_plan_set_lr_order(self._h, int(mode)))
         self._refresh()
 
     def set_halo(self, mode: int):

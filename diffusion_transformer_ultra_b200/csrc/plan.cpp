@@ -71,6 +71,18 @@ ClassDesc window_class(const ultragen_plan_t* p, int wid) {
   return c;
 }
 
+// LR block of one tile in the block order of the LR segment (R20): 8 LR rows x 16 columns.
+constexpr int kLrBH = 8, kLrBW = 16;
+
+// Slot of LR token (m, n): raster order over the LR grid, or block order (blocks of
+// kLrBH x kLrBW row-major, raster order inside a block) when the plan takes it.
+int64_t lr_slot(const ultragen_plan_t* p, int m, int n) {
+  if (!p->lr_block) return p->off_lr + (int64_t)m * p->w + n;
+  const int nbw = cdiv(p->w, kLrBW);
+  return p->off_lr + ((int64_t)(m / kLrBH) * nbw + n / kLrBW) * kTile + (m % kLrBH) * kLrBW +
+         n % kLrBW;
+}
+
 void add_range(std::vector<int>& v, int64_t s_begin, int64_t s_end) {
   if (s_end <= s_begin) return;
   for (int64_t t = s_begin / kTile; t <= (s_end - 1) / kTile; ++t) v.push_back((int)t);
@@ -87,7 +99,7 @@ void for_each_halo_token(const ultragen_plan_t* p, int w, F&& f) {
       if (i / p->l != wr || j / p->l != wc) f(i, j);
 }
 
-int build_tables_mode(ultragen_plan_t* p, int halo);
+int build_tables_mode(ultragen_plan_t* p, int halo, int lr_block);
 
 }  // namespace
 
@@ -96,9 +108,24 @@ int build_tables_mode(ultragen_plan_t* p, int halo);
 // permute traffic of the copies (about 3.3 entries per copied 128-row K/V tile: written once
 // and read again by the attention).
 int build_tables(ultragen_plan_t* p) {
-  if (p->halo_req == 0 || p->b == 0) return build_tables_mode(p, 0);
-  if (p->halo_req == 1) return build_tables_mode(p, 1);
-  int st = build_tables_mode(p, 0);
+  // LR segment order (R20): blocks only serve the LR-region scope; "auto" takes them when they
+  // give fewer tile-list entries (they cost no extra traffic)
+  int lrb = 0;
+  if (p->lr_radius >= 0 && p->rho > 0 && p->lr_order_req != 0) {
+    if (p->lr_order_req == 1) {
+      lrb = 1;
+    } else {
+      int st = build_tables_mode(p, 0, 0);
+      if (st) return st;
+      const size_t n_raster_order = p->entries.size();
+      st = build_tables_mode(p, 0, 1);
+      if (st) return st;
+      lrb = p->entries.size() < n_raster_order ? 1 : 0;
+    }
+  }
+  if (p->halo_req == 0 || p->b == 0) return build_tables_mode(p, 0, lrb);
+  if (p->halo_req == 1) return build_tables_mode(p, 1, lrb);
+  int st = build_tables_mode(p, 0, lrb);
   if (st) return st;
   // entries the halo blocks would replace: each HR query tile's neighbour-window tiles give way
   // to its windows' halo tiles
@@ -125,13 +152,13 @@ int build_tables(ultragen_plan_t* p) {
     for (int c = 0; c < C; ++c) saved -= halo_tiles[wf + c];
   }
   const double copy_tiles = (double)p->nWh * p->nWw * (G / kTile);
-  if ((double)saved > 3.3 * copy_tiles) return build_tables_mode(p, 1);
+  if ((double)saved > 3.3 * copy_tiles) return build_tables_mode(p, 1, lrb);
   return ULTRAGEN_OK;
 }
 
 namespace {
 
-int build_tables_mode(ultragen_plan_t* p, int halo) {
+int build_tables_mode(ultragen_plan_t* p, int halo, int lr_block) {
   p->nWh = cdiv(p->H, p->l);
   p->nWw = cdiv(p->W, p->l);
   p->h = p->rho > 0 ? cdiv(p->H, p->rho) : 0;
@@ -141,7 +168,9 @@ int build_tables_mode(ultragen_plan_t* p, int halo) {
   p->N_hrp = (int64_t)p->nWh * p->nWw * p->l * p->l;
   p->off_hr = pad128(p->T);
   p->off_lr = p->off_hr + pad128(p->N_hrp);
-  p->N_tot = p->off_lr + pad128(p->N_lr);
+  p->lr_block = (lr_block && p->lr_radius >= 0 && p->rho > 0) ? 1 : 0;
+  const int nbw = cdiv(p->w, kLrBW);   // LR blocks per block row (R20)
+  p->N_tot = p->off_lr + (p->lr_block ? (int64_t)cdiv(p->h, kLrBH) * nbw * kTile : pad128(p->N_lr));
   p->N_raster = p->T + p->N_hr + p->N_lr;
   if (p->N_tot > (int64_t)1 << 30) return ULTRAGEN_ERR_UNSUPPORTED;
   p->n_qtiles = (int)(p->N_tot / kTile);
@@ -230,7 +259,7 @@ int build_tables_mode(ultragen_plan_t* p, int halo) {
   // LR tokens at positions (rho m, rho n) ([UG-note] 关键设计 2)
   for (int m = 0; m < p->h; ++m) {
     for (int n = 0; n < p->w; ++n) {
-      const int64_t s = p->off_lr + (int64_t)m * p->w + n;
+      const int64_t s = lr_slot(p, m, n);
       const int64_t r = p->T + p->N_hr + (int64_t)m * p->w + n;
       p->perm[s] = (int32_t)r;
       p->inv_perm[r] = (int32_t)s;
@@ -296,7 +325,7 @@ int build_tables_mode(ultragen_plan_t* p, int halo) {
     add_range(cand, 0, p->T);
     if (kind == SEG_TEXT) add_range(cand, p->off_hr, hr_end);
     if (kind == SEG_LR || (kind == SEG_HR && p->lr_radius < 0))
-      add_range(cand, p->off_lr, p->off_lr + p->N_lr);
+      add_range(cand, p->off_lr, p->N_tot);
     if (kind == SEG_HR && p->lr_radius >= 0 && p->rho > 0) {
       for (int c = 0; c < C; ++c) {
         if (class_real[c] == 0) continue;
@@ -306,8 +335,16 @@ int build_tables_mode(ultragen_plan_t* p, int halo) {
         const int m1 = std::min(p->h - 1, (cd.lr1 - 1) / p->rho);
         const int n0 = std::max(0, cd.lc0 > 0 ? cdiv(cd.lc0, p->rho) : 0);
         const int n1 = std::min(p->w - 1, (cd.lc1 - 1) / p->rho);
-        for (int m = m0; m <= m1 && n0 <= n1; ++m)
-          add_range(cand, p->off_lr + (int64_t)m * p->w + n0, p->off_lr + (int64_t)m * p->w + n1 + 1);
+        for (int m = m0; m <= m1 && n0 <= n1; ++m) {
+          if (!p->lr_block) {
+            add_range(cand, p->off_lr + (int64_t)m * p->w + n0, p->off_lr + (int64_t)m * p->w + n1 + 1);
+            continue;
+          }
+          for (int bn = n0 / kLrBW; bn <= n1 / kLrBW; ++bn) {   // the row's piece in each block
+            const int a = std::max(n0, bn * kLrBW), z = std::min(n1, bn * kLrBW + kLrBW - 1);
+            add_range(cand, lr_slot(p, m, a), lr_slot(p, m, z) + 1);
+          }
+        }
       }
     }
     if (kind == SEG_HR) {
@@ -597,6 +634,25 @@ int ultragen_plan_set_halo(ultragen_plan_t* p, int mode) {
   return ULTRAGEN_OK;
 }
 
+int ultragen_plan_set_lr_order(ultragen_plan_t* p, int mode) {
+  if (!p || mode < -1 || mode > 1) return ULTRAGEN_ERR_INVALID_ARG;
+  const int old = p->lr_order_req;
+  p->lr_order_req = mode;
+  int st;
+  try {
+    st = ug::build_tables(p);
+  } catch (const std::bad_alloc&) {
+    st = ULTRAGEN_ERR_OOM;
+  }
+  if (st != ULTRAGEN_OK) {
+    p->lr_order_req = old;
+    ug::build_tables(p);
+    return st;
+  }
+  p->dirty = true;
+  return ULTRAGEN_OK;
+}
+
 int ultragen_plan_set_qk_format(ultragen_plan_t* p, int format, int q_exp, int k_exp) {
   if (!p || (format != ULTRAGEN_QK_BF16 && format != ULTRAGEN_QK_E4M3) ||
       q_exp < -ULTRAGEN_QK_EXP_MAX || q_exp > ULTRAGEN_QK_EXP_MAX ||
@@ -633,6 +689,7 @@ int ultragen_plan_info(const ultragen_plan_t* p, ultragen_plan_info_t* o) {
   o->halo_slots_per_window = (int32_t)p->G;
   o->N_kv = p->N_kv;
   o->off_halo = p->off_halo;
+  o->lr_block = p->lr_block;
   o->qk_format = p->qk_format;
   o->q_exp = p->q_exp;
   o->k_exp = p->k_exp;

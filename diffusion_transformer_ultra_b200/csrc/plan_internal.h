@@ -70,6 +70,10 @@ struct ultragen_plan {
   // G K/V slots per window, N_kv = N_tot + nWh * nWw * G
   int halo_req = -1;
   int halo_copy = 0;
+  // LR segment order: requested (-1 auto, 0 raster, 1 blocks of 8 x 16 LR tokens) and in effect
+  // (blocks only with the LR-region scope)
+  int lr_order_req = -1;
+  int lr_block = 0;
   int64_t G = 0, N_kv = 0, off_halo = 0;
   // format of the permuted Q and K: ULTRAGEN_QK_BF16, or ULTRAGEN_QK_E4M3 with the stored
   // values x * 2^-q_exp (Q) and x * 2^-k_exp (K)

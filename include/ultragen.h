@@ -86,6 +86,7 @@ typedef struct {
   int64_t off_halo;           /* first halo-block slot (= N_tot)                         */
   int32_t qk_format;          /* ULTRAGEN_QK_BF16 or ULTRAGEN_QK_E4M3                    */
   int32_t q_exp, k_exp;       /* e4m3 scale exponents (0 for bf16)                       */
+  int32_t lr_block;           /* 1: LR segment in 8 x 16 blocks (ultragen_plan_set_lr_order) */
 } ultragen_plan_info_t;
 
 /* Human-readable name of a status code.  Never NULL. */
@@ -127,6 +128,17 @@ int ultragen_plan_set_split(ultragen_plan_t* plan, int chunk);
  * (rho m, rho n) lies in [wr l - r, (wr+1) l + r) x [wc l - r, (wc+1) l + r).  Rebuilds the
  * tile lists; rope and split settings are kept.  INVALID_ARG for radius < -1. */
 int ultragen_plan_set_lr_scope(ultragen_plan_t* plan, int radius);
+
+/* Order of the LR segment in the permuted layout (no counterpart in the pages; the attention is
+ * the same function).  mode = 0: raster order over the LR grid (h x w), padded to 128.  mode = 1:
+ * blocks of 8 LR rows x 16 columns, one 128-slot tile each, row-major over the grid, raster order
+ * inside a block (LR token (m, n) at off_lr + ((m/8) * ceil(w/16) + n/16) * 128 + (m%8) * 16 +
+ * n%16; edge blocks keep pad slots), so the LR region an HR window sees under
+ * ultragen_plan_set_lr_scope falls into a few dense tiles.  mode = -1 (the default): blocks when
+ * they give fewer tile-list entries.  Blocks apply only with an LR-region scope (radius >= 0);
+ * with all LR tokens visible the order stays raster.  Rebuilds the tile lists; may change
+ * N_tot.  INVALID_ARG for another mode. */
+int ultragen_plan_set_lr_order(ultragen_plan_t* plan, int mode);
 
 /* Compact halo blocks in the K/V layout (no counterpart in the pages; the attention is the
  * same function).  Window w's halo -- the HR tokens of its box grown by b ([UG-note] 关键设计 1/2,

@@ -12,8 +12,8 @@ def to_np64(t):
     return t.detach().to("cpu", torch.float64).numpy()
 
 
-def geometry(wl, lr_radius=-1):
-    return O.Geometry(wl.H, wl.W, wl.l, wl.b, wl.rho, wl.T, lr_radius)
+def geometry(wl, lr_radius=-1, lr_block=False):
+    return O.Geometry(wl.H, wl.W, wl.l, wl.b, wl.rho, wl.T, lr_radius, lr_block=lr_block)
 
 
 def check_attention(got, ref, what=""):
@@ -25,10 +25,10 @@ def check_attention(got, ref, what=""):
     return max_abs, mean_rel
 
 
-def oracle_rows(q, k, v, wl, b, heads, rows, lr_radius=-1, **fwd):
+def oracle_rows(q, k, v, wl, b, heads, rows, lr_radius=-1, lr_block=False, **fwd):
     """Oracle output [len(heads), len(rows), D] for batch b, the given heads and permuted rows
     (``fwd``: further options of the oracle's forward, e.g. the Q/K format)."""
-    g = geometry(wl, lr_radius)
+    g = geometry(wl, lr_radius, lr_block)
     out = []
     for h in heads:
         qh = to_np64(q[b:b + 1, :, h:h + 1, :])

@@ -273,11 +273,16 @@ def test_diagnostics_validation(ffi):
     assert L.ultragen_plan_set_diagnostics(p.handle, 0, 2.0) == 0
 
 
-def compare_region_plan(ffi, geom, r, qtiles=None):
+def compare_region_plan(ffi, geom, r, qtiles=None, order=None):
     p = ffi.Plan(*geom, 2, 64)
     p.set_lr_scope(r)
+    if order is not None:
+        p.set_lr_order(order)
     assert p.info["lr_radius"] == r
-    g = O.Geometry(*geom, lr_radius=r, halo_copy=bool(p.info["halo_copy"]))
+    g = O.Geometry(*geom, lr_radius=r, halo_copy=bool(p.info["halo_copy"]),
+                   lr_block=bool(p.info["lr_block"]))
+    if callable(qtiles):
+        qtiles = qtiles(g)
     perm, row_ptr, entries = p.export()
     np.testing.assert_array_equal(perm, O.perm_map(g))
     np.testing.assert_array_equal(p.export_kv(), O.kv_perm_map(g))
@@ -289,10 +294,32 @@ def compare_region_plan(ffi, geom, r, qtiles=None):
     return g, p
 
 
+@pytest.mark.parametrize("order", [None, 0, 1])
 @pytest.mark.parametrize("name,r", [("tiny", 0), ("1k", 4), ("odd", 3), ("small_l", 1)])
-def test_region_plan_bit_exact(ffi, name, r):
-    g, p = compare_region_plan(ffi, GEOMS[name], r)
+def test_region_plan_bit_exact(ffi, name, r, order):
+    g, p = compare_region_plan(ffi, GEOMS[name], r, order=order)
+    if order is not None:
+        assert p.info["lr_block"] == order
     assert p.info["useful_pairs"] == O.visible_pair_count(g)
+
+
+def test_lr_order_argument_checks_and_auto_choice(ffi):
+    p = ffi.Plan(256, 256, 16, 4, 4, 512, 2, 64)
+    L = ffi.lib()
+    assert L.ultragen_plan_set_lr_order(p.handle, 2) == 1
+    assert L.ultragen_plan_set_lr_order(p.handle, -2) == 1
+    p.set_lr_order(1)
+    assert p.info["lr_block"] == 0                  # all LR visible: the order stays raster
+    p.set_lr_scope(4)
+    auto = p.info["n_entries"]
+    assert p.info["lr_block"] == 1                  # the 4K region: blocks give fewer entries
+    p.set_lr_order(0)
+    assert p.info["lr_block"] == 0 and p.info["n_entries"] > auto
+    p.set_lr_order(-1)
+    assert p.info["lr_block"] == 1 and p.info["n_entries"] == auto
+    q = ffi.Plan(256, 135, 16, 16, 4, 256, 2, 64)   # ragged: raster packs the region better
+    q.set_lr_scope(4)
+    assert q.info["lr_block"] == 0
 
 
 def test_region_plan_large_sampled(ffi):
@@ -301,8 +328,7 @@ def test_region_plan_large_sampled(ffi):
     from test_oracle_pins import closed_form_pairs
     for geom, r in (((256, 256, 16, 4, 4, 512), 4), ((512, 512, 16, 4, 4, 512), 0),
                     ((256, 135, 16, 16, 4, 256), 16)):
-        g = O.Geometry(*geom, lr_radius=r)
-        _, p = compare_region_plan(ffi, geom, r, sample_qtiles(g, n_hr=10))
+        _, p = compare_region_plan(ffi, geom, r, lambda g: sample_qtiles(g, n_hr=10))
         assert p.info["useful_pairs"] == sum(closed_form_pairs(*geom, lr_radius=r).values())
     p = ffi.Plan(64, 64, 16, 4, 4, 512, 2, 64)
     assert ffi.lib().ultragen_plan_set_lr_scope(p.handle, -2) == 1
@@ -341,14 +367,18 @@ def test_plan_matches_oracle_on_random_geometries(ffi):
         T = int(rng.choice([0, 1, 3, 127, 128, 129, 300]))
         r = int(rng.choice([-1, -1, 0, 2, 5])) if rho else -1
         halo = [None, 0, 1][case % 3]
+        order = [None, 1, 0, None][case % 4]
         p = ffi.Plan(H, W, l, b, rho, T, 2, 64)
         if r >= 0:
             p.set_lr_scope(r)
+        if order is not None:
+            p.set_lr_order(order)
         if halo is not None:
             p.set_halo(halo)
         info = p.info
-        g = O.Geometry(H, W, l, b, rho, T, r, halo_copy=bool(info["halo_copy"]))
-        what = f"case {case}: H={H} W={W} l={l} b={b} rho={rho} T={T} r={r} halo={halo}"
+        g = O.Geometry(H, W, l, b, rho, T, r, halo_copy=bool(info["halo_copy"]),
+                       lr_block=bool(info["lr_block"]))
+        what = f"case {case}: H={H} W={W} l={l} b={b} rho={rho} T={T} r={r} halo={halo} order={order}"
         assert (info["N_tot"], info["N_kv"], info["off_lr"]) == (g.N_tot, g.N_kv, g.off_lr), what
         perm, row_ptr, entries = p.export()
         np.testing.assert_array_equal(perm, O.perm_map(g), err_msg=what)

@@ -29,11 +29,13 @@ def _wl(name, **kw):
     return dataclasses.replace(WORKLOADS[name], **kw) if kw else WORKLOADS[name]
 
 
-def run_layer(ug, wl, split=None, poison=True, lr_radius=-1, halo=None):
+def run_layer(ug, wl, split=None, poison=True, lr_radius=-1, halo=None, lr_order=None):
     import torch
     plan = ug.plan_for(wl)
     if lr_radius != -1:
         plan.set_lr_scope(lr_radius)
+    if lr_order is not None:
+        plan.set_lr_order(lr_order)
     if halo is not None:
         plan.set_halo(halo)
     if split is not None:
@@ -212,22 +214,33 @@ def test_attention_full_size_sampled(ug, name, heads):
         check_attention(got[:, real], ref[:, real], f"{name} b={b}")
 
 
-@pytest.mark.parametrize("name,r,heads", [("1k", 4, (0, 11, 23)), ("tiny", 0, (0,)),
-                                          ("4k", 4, (9,)), ("8k", 0, (2,))])
-def test_attention_lr_region_parity(ug, name, r, heads):
-    """The LR-region reading (HR queries see only the anchors of their window, grown by r)."""
+@pytest.mark.parametrize("name,r,heads,order", [("1k", 4, (0, 11, 23), None), ("tiny", 0, (0,), None),
+                                                ("4k", 4, (9,), None), ("8k", 0, (2,), None),
+                                                ("1k", 4, (0, 23), 1), ("tiny", 0, (0,), 1),
+                                                ("odd", 3, (0, 2), 1), ("4k", 4, (9,), 0)])
+def test_attention_lr_region_parity(ug, name, r, heads, order):
+    """The LR-region reading (HR queries see only the anchors of their window, grown by r), with
+    the LR segment in the order the plan picks (4K, 8K: 8 x 16 blocks, R20) or the one forced."""
     import torch
-    wl = _wl(name)
-    plan, (q, k, v), lay, o = run_layer(ug, wl, lr_radius=r)
+    wl = _wl(name) if name in ("tiny", "1k", "4k", "8k") else custom(name)
+    plan, (q, k, v), lay, o = run_layer(ug, wl, lr_radius=r, lr_order=order)
     assert plan.info["lr_radius"] == r
+    lrb = bool(plan.info["lr_block"])
+    if order is not None:
+        assert lrb == bool(order)
+    elif name in ("4k", "8k"):
+        assert lrb                              # the automatic choice takes the blocks there
     assert not torch.isnan(lay.op).any()
-    g = geometry(wl, r)
-    rows = np.arange(g.N_tot) if name in ("1k", "tiny") else sample_rows(wl, n_text=128, n_lr=128)
+    g = geometry(wl, r, lrb)
+    rows = np.arange(g.N_tot) if name in ("1k", "tiny", "odd") else sample_rows(wl, n_text=128, n_lr=128)
+    rows = rows[rows < g.N_tot]
     real = O.perm_map(g)[rows] >= 0
-    ref = oracle_rows(q, k, v, wl, 0, heads, rows, lr_radius=r)
-    got = np.stack([to_np64(lay.op[0, h, torch.as_tensor(rows, device="cuda")]) for h in heads])
+    ref = np.concatenate([oracle_rows(q, k, v, wl, b, heads, rows, lr_radius=r, lr_block=lrb)
+                          for b in range(wl.batch)])
+    got = np.concatenate([np.stack([to_np64(lay.op[b, h, torch.as_tensor(rows, device="cuda")])
+                                    for h in heads]) for b in range(wl.batch)])
     assert np.all(got[:, ~real] == 0)
-    check_attention(got[:, real], ref[:, real], f"{name} lr_radius={r}")
+    check_attention(got[:, real], ref[:, real], f"{name} lr_radius={r} lr_block={lrb}")
 
 
 @pytest.mark.parametrize("name,split,r", [("1k", None, -1), ("1k", 5, -1), ("ragged", None, -1),

@@ -51,6 +51,7 @@ def test_random_layer_parity(ug, c):
     plan = ug.plan_for(wl)
     if c["r"] >= 0:
         plan.set_lr_scope(c["r"])
+        plan.set_lr_order(c["cfg"] % 2)   # both LR orders across the cases
     if c["halo"] is not None:
         plan.set_halo(c["halo"])
     if c["split"] is not None:
@@ -68,7 +69,8 @@ def test_random_layer_parity(ug, c):
     ug.hla_forward_raster(lay.qp, lay.kp, lay.vp, o2, plan)
     assert plan.sync_status() == 0
     torch.cuda.synchronize()
-    g = dataclasses.replace(geometry(wl, c["r"]), halo_copy=bool(plan.info["halo_copy"]))
+    lrb = bool(plan.info["lr_block"])
+    g = dataclasses.replace(geometry(wl, c["r"], lrb), halo_copy=bool(plan.info["halo_copy"]))
     real = O.perm_map(g) >= 0
     rows = np.arange(g.N_tot)
     fwd = {"qk_format": "e4m3"} if c["qk"] == "e4m3" else {}
@@ -76,7 +78,7 @@ def test_random_layer_parity(ug, c):
         for h in range(wl.heads):
             vh = to_np64(v[b:b + 1, :, h:h + 1, :])
             np.testing.assert_array_equal(to_np64(lay.vp[b, h]), O.round_bf16(O.permute_kv(vh, g)[0, 0]))
-        ref = oracle_rows(q, k, v, wl, b, range(wl.heads), rows, lr_radius=c["r"], **fwd)
+        ref = oracle_rows(q, k, v, wl, b, range(wl.heads), rows, lr_radius=c["r"], lr_block=lrb, **fwd)
         got = np.stack([to_np64(lay.op[b, h]) for h in range(wl.heads)])
         assert np.all(got[:, ~real] == 0)
         check_attention(got[:, real], ref[:, real], str(c))
