@@ -20,10 +20,11 @@
  *     streams at once.  The first device call on a plan uploads its tables with a
  *     synchronous copy; make that call before any stream capture.
  *
- * Sequence layout (the "permuted" layout, readings of the pages listed in the design doc):
+ * Sequence layout (the "permuted" layout; where the pages leave it open, the plainest reading):
  *   slots [0, T) text | pad to a multiple of 128 | HR tokens window-first (windows row-major,
  *   l*l slots each, raster order inside; partial edge windows padded) | pad to 128 |
- *   LR tokens raster | pad to 128.   N_tot = number of slots, a multiple of 128.
+ *   LR tokens raster, or in 8 x 16 blocks of the LR grid (ultragen_plan_set_lr_order) |
+ *   pad to 128.   N_tot = number of slots, a multiple of 128.
  *   K/V layout: the same N_tot slots, then, when the plan uses compact halo blocks
  *   (ultragen_plan_set_halo), one block of G slots per window holding that window's halo
  *   tokens; N_kv = N_tot + nWh * nWw * G (N_kv = N_tot without blocks).  Q and O use N_tot.

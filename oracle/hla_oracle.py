@@ -27,7 +27,7 @@ What each function follows:
 Tables returned by the cached geometry helpers (raster_tokens, slot_of_tokens, perm_map,
 slot_info) are shared between calls: callers must not modify them.
 
-Readings taken where the pages are silent or garbled (each is listed in the design doc):
+Readings taken where the pages are silent or garbled:
   R1  l counts latent tokens (l=16 <-> 256x256 pixels at a 16x VAE).
   R2  Halo: the query's own window box grown by b tokens on every side, clipped to the
       image; every query of a window sees the same set.  0 <= b <= l.

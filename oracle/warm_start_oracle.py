@@ -16,7 +16,7 @@ latent grid by interpolation and sharpened, giving the reference X_ref. The star
 is the blend X_hr = alpha * X_T + (1 - alpha) * X_ref of Gaussian noise X_T and that
 reference, where alpha = t / T is the noise level of the intermediate timestep.
 
-Readings taken where the pages leave a step open (each is listed in the design doc):
+Readings taken where the pages leave a step open:
   W1  "Interpolate" is bilinear upsampling from the LR grid (h, w) to the HR grid (H, W)
       with half-pixel centres: along each axis the source coordinate of output index i is
       (i + 0.5) * (h / H) - 0.5, clamped below at 0; the two taps are floor of it and the
