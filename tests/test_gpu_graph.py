@@ -12,13 +12,15 @@ def ug(gpu_required):
     return pkg
 
 
-@pytest.mark.parametrize("name,split", [("1k", None), ("1k", 5), ("ragged", None)])
-def test_layer_replays_from_a_cuda_graph(ug, name, split):
+@pytest.mark.parametrize("name,split,qk", [("1k", None, "bf16"), ("1k", 5, "bf16"),
+                                           ("ragged", None, "bf16"), ("1k", 5, "e4m3")])
+def test_layer_replays_from_a_cuda_graph(ug, name, split, qk):
     import torch
     wl = ug.WORKLOADS[name]
     plan = ug.plan_for(wl)
     if split is not None:
         plan.set_split(split)
+    plan.set_qk_format(qk)
     q, k, v = (x.cuda() for x in ug.make_qkv(wl))
     shape = (wl.batch, plan.info["N_raster"], wl.heads, wl.D)
     lay = ug.Layer(plan, wl.batch)
