@@ -308,11 +308,13 @@ int ultragen_last_launch_count(const ultragen_plan_t* plan);
  *   q, k, v  [batch, N_raster, heads, head_dim] BF16 in HOST memory (page-locked memory lets
  *            the copies overlap the kernels; pageable memory works, serialised)
  *   o        [batch, N_raster, heads, head_dim] BF16 in HOST memory, written in full
+ *   The layer follows the plan's settings at the call (Q/K format, LR scope and order, halo
+ *   blocks, split schedule), exactly as the device entry points would.
  *   Asynchronous: the work is ordered after what `stream` holds at the call, and `stream`
  *   waits for all of it, so o is complete once `stream` is synchronised.  Calls on one runner
  *   must not overlap (one call at a time per runner).  PLAN_MISMATCH when called on another
- *   device than the one the runner was created on, or when the plan's split schedule or halo
- *   blocks now need more storage than was allocated.  Device-side wait timeouts are reported by
+ *   device than the one the runner was created on, or when the plan's split schedule, halo
+ *   blocks or LR order now need more storage than was allocated.  Device-side wait timeouts are reported by
  *   ultragen_sync_status(plan, stream).
  * ultragen_host_runner_last_launch_count(runner): kernels the last forward launched.
  * ultragen_host_runner_destroy(runner): waits for the runner's streams, frees everything.
