@@ -223,6 +223,18 @@ def profiled_traffic(workload: str):
     return ent.get("dram_bytes_per_launch")
 
 
+def cpu_model() -> str:
+    """The host CPU's model name, from /proc/cpuinfo (empty when unavailable)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.lower().startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return ""
+
+
 def cpu_baseline(wl, q, k, v, budget_s: float = 12.0, lr_radius: int = -1, lr_block: bool = False,
                  **fwd):
     """The oracle as it stands, timed on this host on a bounded sample: one head, rows of one
@@ -251,7 +263,7 @@ def cpu_baseline(wl, q, k, v, budget_s: float = 12.0, lr_radius: int = -1, lr_bl
     dt = (time.perf_counter() - t0) / reps
     flops = 4.0 * wl.D * vis_pairs
     return {"value": flops / dt / 1e12, "unit": "useful TFLOP/s", "cores": os.cpu_count(),
-            "kind": "oracle",
+            "cpu_model": cpu_model(), "kind": "oracle",
             "sample": f"1 head, {len(rows)} query rows ({vis_pairs} visible pairs), full RoPE + "
                       f"explicit mask, fp64 NumPy; {reps} rep(s), {dt:.2f} s each"}
 
@@ -279,7 +291,8 @@ def run_reference(args, rank, world):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl.name, "H": wl.H, "W": wl.W, "l": wl.l, "b": wl.b, "rho": wl.rho,
                    "text_len": wl.T, "heads": wl.heads, "head_dim": wl.D, "batch": wl.batch},
-        "cpu_baseline": {"kind": "oracle", "cores": base["cores"], "sample": base["sample"],
+        "cpu_baseline": {"kind": "oracle", "cores": base["cores"], "cpu_model": base["cpu_model"],
+                         "sample": base["sample"],
                          "value": value, "unit": "useful TFLOP/s"},
         "e2e": {"value": value, "unit": "useful TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
