@@ -225,6 +225,7 @@ __global__ void __launch_bounds__(kWarmThreads) warm_start_kernel(const WarmArgs
 // One thread per low-resolution cell: its 3 x 3 neighbourhood, then ry rows of 4 outputs (one
 // 16-byte load of noise and one 16-byte store each); a warp covers 32 cells of one row, so
 // loads and stores are 512-byte runs.
+template <int RY>
 __global__ void __launch_bounds__(kWarmThreads) warm_start_fused_kernel(const WarmArgs a,
                                                                         const WarmFused wf) {
   const int plane = blockIdx.z;
@@ -232,27 +233,30 @@ __global__ void __launch_bounds__(kWarmThreads) warm_start_fused_kernel(const Wa
   const int k = blockIdx.y * (kWarmThreads / 32) + (threadIdx.x >> 5);
   if (l >= a.w || k >= a.h) return;
   const int x = 4 * l;
-  const uint64_t row0 = static_cast<uint64_t>(plane) * a.H + static_cast<uint64_t>(k) * wf.ry;
+  // first output row of the cell; rows of one plane step by W elements
+  const size_t first = (static_cast<size_t>(plane) * a.H + static_cast<size_t>(k) * RY) * a.W + x;
+  float* out = a.out + first;
   // the noise of the cell's outputs first, so the loads are in flight during the arithmetic
-  float4 nz[8];
+  float4 nz[RY];
   if (a.noise) {
+    const float* nzp = a.noise + first;
 #pragma unroll
-    for (int p = 0; p < 8; ++p)
-      if (p < wf.ry)
-        nz[p] = __ldcs(reinterpret_cast<const float4*>(a.noise + (row0 + p) * a.W + x));
+    for (int p = 0; p < RY; ++p)
+      nz[p] = __ldcs(reinterpret_cast<const float4*>(nzp + static_cast<size_t>(p) * a.W));
   }
   const float* L = a.lr + static_cast<size_t>(plane) * a.h * a.w;
+  const int c0 = max(l - 1, 0), c2 = min(l + 1, a.w - 1);
   float X[3][3];
 #pragma unroll
   for (int i = 0; i < 3; ++i) {
     const float* row = L + static_cast<size_t>(min(max(k + i - 1, 0), a.h - 1)) * a.w;
-#pragma unroll
-    for (int j = 0; j < 3; ++j) X[i][j] = __ldg(row + min(max(l + j - 1, 0), a.w - 1));
+    X[i][0] = __ldg(row + c0);
+    X[i][1] = __ldg(row + l);
+    X[i][2] = __ldg(row + c2);
   }
   const float alpha = a.alpha;
 #pragma unroll
-  for (int p = 0; p < 8; ++p) {
-    if (p >= wf.ry) break;
+  for (int p = 0; p < RY; ++p) {
     float Ra[3], Rb[3];
 #pragma unroll
     for (int j = 0; j < 3; ++j) {
@@ -269,9 +273,9 @@ __global__ void __launch_bounds__(kWarmThreads) warm_start_fused_kernel(const Wa
       acc = fmaf(wf.cb[q][1], Rb[1], acc);
       r[q] = fmaf(wf.cb[q][2], Rb[2], acc);
     }
-    const uint64_t flat = (row0 + p) * a.W + x;
-    const float4 n = a.noise ? nz[p] : normals4(flat >> 2, a.seed, a.offset);
-    __stcs(reinterpret_cast<float4*>(a.out + flat),
+    const float4 n = a.noise ? nz[p]
+                             : normals4((first + static_cast<size_t>(p) * a.W) >> 2, a.seed, a.offset);
+    __stcs(reinterpret_cast<float4*>(out + static_cast<size_t>(p) * a.W),
            make_float4(fmaf(alpha, n.x, r[0]), fmaf(alpha, n.y, r[1]), fmaf(alpha, n.z, r[2]),
                        fmaf(alpha, n.w, r[3])));
   }
@@ -287,7 +291,17 @@ cudaError_t launch_warm_start(const WarmArgs& a, cudaStream_t st) {
 
 cudaError_t launch_warm_start_fused(const WarmArgs& a, const WarmFused& f, cudaStream_t st) {
   const dim3 grid((a.w + 31) / 32, (a.h + kWarmThreads / 32 - 1) / (kWarmThreads / 32), a.planes);
-  warm_start_fused_kernel<<<grid, kWarmThreads, 0, st>>>(a, f);
+  switch (f.ry) {   // the row ratio as a constant: fully unrolled rows, no bounds checks
+    case 1: warm_start_fused_kernel<1><<<grid, kWarmThreads, 0, st>>>(a, f); break;
+    case 2: warm_start_fused_kernel<2><<<grid, kWarmThreads, 0, st>>>(a, f); break;
+    case 3: warm_start_fused_kernel<3><<<grid, kWarmThreads, 0, st>>>(a, f); break;
+    case 4: warm_start_fused_kernel<4><<<grid, kWarmThreads, 0, st>>>(a, f); break;
+    case 5: warm_start_fused_kernel<5><<<grid, kWarmThreads, 0, st>>>(a, f); break;
+    case 6: warm_start_fused_kernel<6><<<grid, kWarmThreads, 0, st>>>(a, f); break;
+    case 7: warm_start_fused_kernel<7><<<grid, kWarmThreads, 0, st>>>(a, f); break;
+    case 8: warm_start_fused_kernel<8><<<grid, kWarmThreads, 0, st>>>(a, f); break;
+    default: return cudaErrorInvalidValue;
+  }
   return cudaGetLastError();
 }
 
