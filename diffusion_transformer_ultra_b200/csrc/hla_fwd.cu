@@ -8,7 +8,7 @@
 // CTA organisation (one persistent CTA per SM, 384 threads = 3 warpgroups):
 //   warps 0-3   softmax group 0: owns query tile slot 0 (thread = row, TMEM lane = row)
 //   warps 4-7   softmax group 1: owns query tile slot 1
-//   warp  8     producer: TMA loads of Q (per item) and of K, V tiles into a ring
+//   warp  8     producer: TMA loads of Q (per item) and of K, V tiles in stages
 //   warp  9     MMA issuer: tcgen05.mma for S = Q K^T (both operands in shared memory) and
 //               O += P V (P read from TMEM, V from shared memory); owns TMEM allocation
 //   warps 10-11 idle
@@ -22,8 +22,11 @@
 //
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D, 256+2D).
 // P (bf16, packed in pairs) overwrites the first 64 columns of its S block.
-// Shared memory: Q0, Q1, and NS K/V slots, each [128 rows x D] bf16 stored as D/64 boxes of
-// [128 x 64] with the 128-byte swizzle (TMA writes it, the MMA descriptors read it).
+// Shared memory: Q0, Q1, and NS K/V tile slots, each [128 rows x D] bf16 stored as D/64 boxes
+// of [128 x 64] with the 128-byte swizzle (TMA writes it, the MMA descriptors read it).  K/V
+// tiles travel in stages of two: stage j of an item with n key tiles holds V(j-1) (j > 0) and
+// K(j) (j < n), exactly what step j of the MMA loop reads, so the MMA warp waits on one full
+// barrier per key tile and releases both slots with one commit.
 // With 8-bit Q K^T (QK8, D = 128) Q and K tiles are e4m3 bytes, one [128 x 128] box of 128-byte
 // rows at the start of their slot, and S = Q K^T takes 4 kind::f8f6f4 products of 32
 // K-elements instead of 8 kind::f16 products of 16; V, P and O are unchanged.
@@ -44,16 +47,22 @@ struct FwdCfg {
   static constexpr int BOXES = D / 64;
   static constexpr int BOX_BYTES = 128 * 64 * 2;
   static constexpr int TILE_BYTES = 128 * D * 2;
-  static constexpr int NS = D == 128 ? 4 : 8;
+  static constexpr int NS = D == 128 ? 4 : 8;      // tile slots
+  static constexpr int NSTG = NS / 2;               // stages in flight (two tiles each)
   static constexpr int Q_OFF = 0;
   static constexpr int KV_OFF = 2 * TILE_BYTES;
   static constexpr int BAR_OFF = KV_OFF + NS * TILE_BYTES;
   // barrier indices
-  static constexpr int B_QF = 0, B_QE = 1, B_KVF = 2, B_KVE = 2 + NS, B_SF = 2 + 2 * NS,
-                       B_PF = 4 + 2 * NS, B_OF = 6 + 2 * NS, B_DRAIN = 8 + 2 * NS;
-  static constexpr int NBAR = 9 + 2 * NS;
+  // B_KVF / B_KVE + g: stage slot g full / empty (g < NSTG)
+  static constexpr int B_QF = 0, B_QE = 1, B_KVF = 2, B_KVE = 2 + NSTG, B_SF = 2 + 2 * NSTG,
+                       B_PF = 4 + 2 * NSTG, B_OF = 6 + 2 * NSTG, B_DRAIN = 8 + 2 * NSTG;
+  static constexpr int NBAR = 9 + 2 * NSTG;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;   // + slack for 1024-B alignment
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA exceeds 227 KB");
+  // the tile slots of stage slot g: V at 2 g, K at 2 g + 1
+  static __device__ __forceinline__ uint32_t v_slot(uint32_t g) { return 2 * g; }
+  static __device__ __forceinline__ uint32_t k_slot(uint32_t g) { return 2 * g + 1; }
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t O_COL = 256;
 };
@@ -120,13 +129,22 @@ __device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
   using C = FwdCfg<D>;
   constexpr int QK_BYTES = QK8 ? 128 * D : C::TILE_BYTES;   // one Q or K tile
   const uint32_t sQ = sbase + C::Q_OFF, sKV = sbase + C::KV_OFF, bar = sbase + C::BAR_OFF;
-  uint32_t ld = 0, qi = 0;
+  uint32_t st = 0, qi = 0;                                  // stages and Q loads issued
   bool ok = true;
+  // one tile: e4m3 Q or K is a single [128 x 128]-byte box, bf16 D / 64 boxes of [128 x 64]
+  auto load_tile = [&](const CUtensorMap* tm, bool bytes, uint32_t dst, int y, uint32_t b) {
+    if (bytes) {
+      tma_load_2d(dst, tm, 0, y, b);
+    } else {
+#pragma unroll
+      for (int bx = 0; bx < C::BOXES; ++bx) tma_load_2d(dst + bx * C::BOX_BYTES, tm, bx * 64, y, b);
+    }
+  };
   for (int it = blockIdx.x; it < p.total_items && ok; it += gridDim.x) {
     int bh;
     const int32_t* I = item_at(p, it, bh);
-    const int qt0 = I[0], qt1 = I[1], e0 = I[2], e1 = I[3];
-    if (e1 == e0) continue;
+    const int qt0 = I[0], qt1 = I[1], e0 = I[2], n = I[3] - I[2];
+    if (n == 0) continue;
     if (!mbar_wait(bar + 8 * C::B_QE, (qi & 1) ^ 1, abort_flag, p.err, DEV_TIMEOUT_PRODUCER,
                    p.timeout_ns)) {
       ok = false;
@@ -134,51 +152,34 @@ __device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
     }
     const int ntile = qt1 >= 0 ? 2 : 1;
     mbar_expect_tx(bar + 8 * C::B_QF, ntile * QK_BYTES);
-    for (int t = 0; t < ntile; ++t) {
-      const int y = bh * p.N_tot + (t ? qt1 : qt0) * 128;
-      if (QK8) {
-        tma_load_2d(sQ + t * C::TILE_BYTES, tmQ, 0, y, bar + 8 * C::B_QF);
-      } else {
-#pragma unroll
-        for (int bx = 0; bx < C::BOXES; ++bx)
-          tma_load_2d(sQ + t * C::TILE_BYTES + bx * C::BOX_BYTES, tmQ, bx * 64, y,
-                      bar + 8 * C::B_QF);
-      }
-    }
+    for (int t = 0; t < ntile; ++t)
+      load_tile(tmQ, QK8, sQ + t * C::TILE_BYTES, bh * p.N_tot + (t ? qt1 : qt0) * 128,
+                bar + 8 * C::B_QF);
     ++qi;
-    for (int e = e0; e < e1 && ok; ++e) {
-      const int y = bh * p.N_kv + (__ldg(p.entries + e) & 0x7fffffff) * 128;
-#pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        const uint32_t s = ld % C::NS, ph = (ld / C::NS) & 1;
-        if (!mbar_wait(bar + 8 * (C::B_KVE + s), ph ^ 1, abort_flag, p.err, DEV_TIMEOUT_PRODUCER,
-                       p.timeout_ns)) {
-          ok = false;
-          break;
-        }
-        if (QK8 && !which) {
-          mbar_expect_tx(bar + 8 * (C::B_KVF + s), QK_BYTES);
-          tma_load_2d(sKV + s * C::TILE_BYTES, tmK, 0, y, bar + 8 * (C::B_KVF + s));
-        } else {
-          mbar_expect_tx(bar + 8 * (C::B_KVF + s), C::TILE_BYTES);
-#pragma unroll
-          for (int bx = 0; bx < C::BOXES; ++bx)
-            tma_load_2d(sKV + s * C::TILE_BYTES + bx * C::BOX_BYTES, which ? tmV : tmK, bx * 64,
-                        y, bar + 8 * (C::B_KVF + s));
-        }
-        ++ld;
+    for (int j = 0; j <= n; ++j) {   // stage j: V(j - 1) if j > 0, K(j) if j < n
+      const uint32_t g = st % C::NSTG, ph = (st / C::NSTG) & 1;
+      if (!mbar_wait(bar + 8 * (C::B_KVE + g), ph ^ 1, abort_flag, p.err, DEV_TIMEOUT_PRODUCER,
+                     p.timeout_ns)) {
+        ok = false;
+        break;
       }
+      const uint32_t fb = bar + 8 * (C::B_KVF + g);
+      mbar_expect_tx(fb, (j > 0 ? C::TILE_BYTES : 0) + (j < n ? QK_BYTES : 0));
+      if (j > 0)
+        load_tile(tmV, false, sKV + C::v_slot(g) * C::TILE_BYTES,
+                  bh * p.N_kv + (__ldg(p.entries + e0 + j - 1) & 0x7fffffff) * 128, fb);
+      if (j < n)
+        load_tile(tmK, QK8, sKV + C::k_slot(g) * C::TILE_BYTES,
+                  bh * p.N_kv + (__ldg(p.entries + e0 + j) & 0x7fffffff) * 128, fb);
+      ++st;
     }
   }
   if (!ok) {
     // Abort: wait (bounded) until the copies this thread issued have landed, so that no TMA
     // write targets this CTA's shared memory after it exits.
-    for (uint32_t s = 0; s < (uint32_t)C::NS; ++s) {
-      if (ld <= s) break;
-      const uint32_t last = ld - 1 - ((ld - 1 - s) % C::NS);
-      mbar_wait(bar + 8 * (C::B_KVF + s), (last / C::NS) & 1, nullptr, p.err, DEV_TIMEOUT_DRAIN,
-                kDrainNs);
-    }
+    for (uint32_t g = st >= (uint32_t)C::NSTG ? st - C::NSTG : 0; g < st; ++g)
+      mbar_wait(bar + 8 * (C::B_KVF + g % C::NSTG), (g / C::NSTG) & 1, nullptr, p.err,
+                DEV_TIMEOUT_DRAIN, kDrainNs);
     if (qi > 0) mbar_wait(bar + 8 * C::B_QF, (qi - 1) & 1, nullptr, p.err, DEV_TIMEOUT_DRAIN, kDrainNs);
   }
 }
@@ -222,7 +223,7 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t tbase,
                          volatile int* abort_flag) {
   using C = FwdCfg<D>;
   const uint32_t sQ = sbase + C::Q_OFF, sKV = sbase + C::KV_OFF, bar = sbase + C::BAR_OFF;
-  uint32_t ld = 0, qi = 0, pc0 = 0, pc1 = 0;
+  uint32_t st = 0, qi = 0, pc0 = 0, pc1 = 0;   // stages, Q loads, P phases consumed
   bool withhold = p.fault == 1;   // injected fault: drop the first item's first "S ready"
   auto wait = [&](int b, uint32_t par) {
     return mbar_wait(bar + 8 * b, par, abort_flag, p.err, DEV_TIMEOUT_MMA, p.timeout_ns);
@@ -238,59 +239,37 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t tbase,
     if (!wait(C::B_QF, qi & 1)) { ok = false; break; }
     ++qi;
     tc_fence_after();
-    {  // j = 0: S_t = Q_t K_0^T
-      const uint32_t s = ld % C::NS;
-      if (!wait(C::B_KVF + s, (ld / C::NS) & 1)) { ok = false; break; }
+    // step j of the item reads stage j: S_t(j) = Q_t K(j)^T needs K(j) (j < n), and
+    // O_t += P_t(j - 1) V(j - 1) (j > 0) needs V(j - 1) and the softmax's P_t(j - 1)
+    for (int j = 0; j <= n && ok; ++j) {
+      const uint32_t g = st % C::NSTG;
+      if (!wait(C::B_KVF + g, (st / C::NSTG) & 1)) { ok = false; break; }
       tc_fence_after();
+      const uint32_t sV = sKV + C::v_slot(g) * C::TILE_BYTES, sK = sKV + C::k_slot(g) * C::TILE_BYTES;
       for (int t = 0; t < ntile; ++t) {
-        issue_s<D, QK8>(tbase + 128 * t, sQ + t * C::TILE_BYTES, sKV + s * C::TILE_BYTES);
-        if (withhold && t == 0) {
-          withhold = false;     // nothing completes this barrier: its waiters time out
+        if (j > 0) {
+          uint32_t& pc = t ? pc1 : pc0;
+          if (!wait(C::B_PF + t, pc & 1)) { ok = false; break; }
+          ++pc;
+          tc_fence_after();
+          issue_pv<D>(tbase + C::O_COL + D * t, tbase + 128 * t, sV, j > 1);
+        }
+        if (j < n) {
+          issue_s<D, QK8>(tbase + 128 * t, sQ + t * C::TILE_BYTES, sK);
+          if (withhold && t == 0) {
+            withhold = false;     // nothing completes this barrier: its waiters time out
+          } else {
+            mma_commit(bar + 8 * (C::B_SF + t));
+          }
         } else {
-          mma_commit(bar + 8 * (C::B_SF + t));
+          mma_commit(bar + 8 * (C::B_OF + t));
         }
       }
-      mma_commit(bar + 8 * (C::B_KVE + s));
-    }
-    for (int j = 1; j < n && ok; ++j) {
-      const uint32_t nv = ld + 2 * j - 1, nk = ld + 2 * j;
-      const uint32_t sv = nv % C::NS, sk = nk % C::NS;
-      if (!wait(C::B_KVF + sv, (nv / C::NS) & 1) || !wait(C::B_KVF + sk, (nk / C::NS) & 1)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      for (int t = 0; t < ntile; ++t) {
-        uint32_t& pc = t ? pc1 : pc0;
-        if (!wait(C::B_PF + t, pc & 1)) { ok = false; break; }
-        ++pc;
-        tc_fence_after();
-        issue_pv<D>(tbase + C::O_COL + D * t, tbase + 128 * t, sKV + sv * C::TILE_BYTES, j > 1);
-        issue_s<D, QK8>(tbase + 128 * t, sQ + t * C::TILE_BYTES, sKV + sk * C::TILE_BYTES);
-        mma_commit(bar + 8 * (C::B_SF + t));
-      }
       if (!ok) break;
-      mma_commit(bar + 8 * (C::B_KVE + sv));
-      mma_commit(bar + 8 * (C::B_KVE + sk));
+      mma_commit(bar + 8 * (C::B_KVE + g));     // both tiles of the stage are read
+      if (j == n - 1) mma_commit(bar + 8 * C::B_QE);   // all products that read Q are issued
+      ++st;
     }
-    if (!ok) break;
-    mma_commit(bar + 8 * C::B_QE);   // all products that read Q of this item are issued
-    {
-      const uint32_t nv = ld + 2 * n - 1, sv = nv % C::NS;
-      if (!wait(C::B_KVF + sv, (nv / C::NS) & 1)) { ok = false; break; }
-      tc_fence_after();
-      for (int t = 0; t < ntile; ++t) {
-        uint32_t& pc = t ? pc1 : pc0;
-        if (!wait(C::B_PF + t, pc & 1)) { ok = false; break; }
-        ++pc;
-        tc_fence_after();
-        issue_pv<D>(tbase + C::O_COL + D * t, tbase + 128 * t, sKV + sv * C::TILE_BYTES, n > 1);
-        mma_commit(bar + 8 * (C::B_OF + t));
-      }
-      if (!ok) break;
-      mma_commit(bar + 8 * (C::B_KVE + sv));
-    }
-    ld += 2 * n;
   }
   if (!ok) {
     // Abort: let the products already issued finish before TMEM is released.
@@ -300,6 +279,44 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t tbase,
 }
 
 // ------------------------------------------------------------------------ softmax groups
+// Exponentials of one S row at the running max mu (log2 units): the pair (s[2c], s[2c+1]) is
+// replaced by its packed bf16 P in s[c].  Returns the row sum of this tile's P.
+__device__ __forceinline__ float exp_row(uint32_t (&s)[128], float scale, float mu) {
+  const float2 scale2 = make_float2(scale, scale), nmu2 = make_float2(-mu, -mu);
+  float2 ls[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) ls[i] = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int c2 = 0; c2 < 64; ++c2) {
+    const float2 x =
+        ffma2(make_float2(__uint_as_float(s[2 * c2]), __uint_as_float(s[2 * c2 + 1])), scale2, nmu2);
+    float2 pp;
+    if (pair_on_fma(c2)) {
+      pp = ex2_fma2(x);
+    } else {
+      pp.x = ex2(x.x);
+      pp.y = ex2(x.y);
+    }
+    ls[c2 & 3] = fadd2(ls[c2 & 3], pp);
+    s[c2] = pack_bf16x2(pp.x, pp.y);
+  }
+  const float2 l2 = fadd2(fadd2(ls[0], ls[1]), fadd2(ls[2], ls[3]));
+  return l2.x + l2.y;
+}
+
+// Multiplies the O accumulator row (TMEM) by f, 32 columns at a time.
+template <int D>
+__device__ __forceinline__ void rescale_o(uint32_t tO, float f) {
+#pragma unroll 1
+  for (int ch = 0; ch < D / 32; ++ch) {
+    uint32_t o[32];
+    tmem_ld32_sync(tO + ch * 32, o);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+    tmem_st32(tO + ch * 32, o);
+  }
+}
+
 template <int D>
 __device__ void softmax_role(const FwdParams& p, uint32_t sbase, uint32_t tbase,
                              volatile int* abort_flag) {
@@ -357,67 +374,74 @@ __device__ void softmax_role(const FwdParams& p, uint32_t sbase, uint32_t tbase,
       tc_fence_after();
       uint32_t s[128];
       tmem_ld128_sync(tS, s);
-      // row max (the row is thread-local: no shuffles), 4 chains of three-input max
       if (ent < 0) {
 #pragma unroll
         for (int c = 0; c < 128; ++c)
           if (!((mw[c >> 5] >> (c & 31)) & 1u)) s[c] = 0xff800000u;   // -inf
       }
-      float mx4[4];
+      if (__any_sync(0xffffffffu, m == neg_inf())) {
+        // A row without a running max yet (its first tile, or only masked scores so far):
+        // take the tile max first (thread-local row, 4 chains of three-input max).
+        float mx4[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) mx4[i] = neg_inf();
+        for (int i = 0; i < 4; ++i) mx4[i] = neg_inf();
 #pragma unroll
-      for (int c = 0; c < 128; c += 8) {
+        for (int c = 0; c < 128; c += 8) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          mx4[i] = fmax3(mx4[i], __uint_as_float(s[c + 2 * i]), __uint_as_float(s[c + 2 * i + 1]));
-      }
-      const float mx = fmax3(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]);
-      const float mnew = fmaxf(m, mx * scale);
-      if (j == 0) {
-        m = mnew;
-      } else {
-        // Lazy rescale: keep the running max unless it grew by more than 2^8; the final
-        // division by the matching row sum makes the result exact either way.
-        const bool need = mnew > m + 8.0f;
+          for (int i = 0; i < 4; ++i)
+            mx4[i] = fmax3(mx4[i], __uint_as_float(s[c + 2 * i]), __uint_as_float(s[c + 2 * i + 1]));
+        }
+        const float mx = fmax3(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]);
+        const float mnew = fmaxf(m, mx * scale);
+        // Lazy rescale: a row with a running max keeps it unless it grew by more than 2^8 (the
+        // final division by the matching row sum makes the result exact either way); a row
+        // without one takes the tile max (its O and sum are still zero).
+        const bool need = m != neg_inf() && mnew > m + 8.0f;
         if (__any_sync(0xffffffffu, need)) {
           const float f = need ? ex2(m - mnew) : 1.0f;
-          if (need) {
-            lsum *= f;
-            m = mnew;
-          }
+          if (need) lsum *= f;
           __syncwarp();
+          rescale_o<D>(tO, f);
+        }
+        if (m == neg_inf() || need) m = mnew;
+        lsum += exp_row(s, scale, (m == neg_inf()) ? 0.f : m);
+      } else {
+        // Every row has a running max: take the exponentials at it, with no tile max at all.
+        // The final division by the row sum makes the result exact for any max, and only
+        // overflow must be excluded: a tile sum above 2^12 (also inf or NaN) means some score
+        // may have risen far above the running max, so the tile is redone from S (still in
+        // TMEM) at its exact max, with O and the sum rescaled to it (rare).
+        float part = exp_row(s, scale, m);
+        if (__any_sync(0xffffffffu, !(part <= 4096.0f))) {
+          float mx = neg_inf();
+#pragma unroll 1
+          for (int ch = 0; ch < 4; ++ch) {
+            uint32_t c32[32];
+            tmem_ld32_sync(tS + ch * 32, c32);
+            const uint32_t mwc = ch == 0 ? mw[0] : (ch == 1 ? mw[1] : (ch == 2 ? mw[2] : mw[3]));
 #pragma unroll
-          for (int ch = 0; ch < D / 32; ++ch) {
-            uint32_t o[32];
-            tmem_ld32_sync(tO + ch * 32, o);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
-            tmem_st32(tO + ch * 32, o);
+            for (int c = 0; c < 32; c += 2) {
+              const float a = ((mwc >> c) & 1u) ? __uint_as_float(c32[c]) : neg_inf();
+              const float b = ((mwc >> (c + 1)) & 1u) ? __uint_as_float(c32[c + 1]) : neg_inf();
+              mx = fmax3(mx, a, b);
+            }
           }
-        }
-      }
-      const float mu = (m == neg_inf()) ? 0.f : m;
-      const float2 scale2 = make_float2(scale, scale), nmu2 = make_float2(-mu, -mu);
-      float2 ls[4];
+          const float mnew = fmaxf(m, mx * scale);
+          const float f = ex2(m - mnew);
+          lsum *= f;
+          m = mnew;
+          __syncwarp();
+          rescale_o<D>(tO, f);
+          tmem_ld128_sync(tS, s);
+          if (ent < 0) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) ls[i] = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int c2 = 0; c2 < 64; ++c2) {
-        const float2 x =
-            ffma2(make_float2(__uint_as_float(s[2 * c2]), __uint_as_float(s[2 * c2 + 1])), scale2, nmu2);
-        float2 pp;
-        if (pair_on_fma(c2)) {
-          pp = ex2_fma2(x);
-        } else {
-          pp.x = ex2(x.x);
-          pp.y = ex2(x.y);
+            for (int c = 0; c < 128; ++c)
+              if (!((mw[c >> 5] >> (c & 31)) & 1u)) s[c] = 0xff800000u;
+          }
+          part = exp_row(s, scale, m);
         }
-        ls[c2 & 3] = fadd2(ls[c2 & 3], pp);
-        s[c2] = pack_bf16x2(pp.x, pp.y);
+        lsum += part;
       }
-      const float2 l2 = fadd2(fadd2(ls[0], ls[1]), fadd2(ls[2], ls[3]));
-      lsum += l2.x + l2.y;
       __syncwarp();
       tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(&s[0]));
       tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(&s[32]));
