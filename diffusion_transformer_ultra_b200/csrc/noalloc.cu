@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "kernels.h"
+#include "nvtx_range.h"
 #include "plan_internal.h"
 
 namespace {
@@ -23,20 +24,45 @@ constexpr int kMaxDevices = 64;
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
 std::mutex g_mu;
-float* g_scratch_ptr[kMaxDevices] = {};   // device address of g_scratch, per device
+// device address of g_scratch, per device, and the CUDA context it was looked up in: a context
+// that was torn down and created again (cudaDeviceReset, a framework's reset) loads the module
+// again at another address, so a cached address is only reused within its own context
+float* g_scratch_ptr[kMaxDevices] = {};
+CUcontext g_scratch_ctx[kMaxDevices] = {};
 
-// Host code must not use g_scratch's name as a device address: look the address up once per
-// device, with that device current.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+// The driver's cuCtxGetCurrent, found through the runtime (the library does not link libcuda).
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess) {
+      cudaGetLastError();
+      return static_cast<CtxGetCurrentFn>(nullptr);
+    }
+    return reinterpret_cast<CtxGetCurrentFn>(f);
+  }();
+  return fn;
+}
+
+// Host code must not use g_scratch's name as a device address: look the address up with the
+// device current, once per device and context.
 int scratch_for_device(int dev, float** out) {
   if (dev < 0 || dev >= kMaxDevices) return ULTRAGEN_ERR_UNSUPPORTED;
+  CtxGetCurrentFn get = ctx_get_current();
+  CUcontext ctx = nullptr;
+  if (!get || get(&ctx) != CUDA_SUCCESS || !ctx) return ULTRAGEN_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_ptr[dev]) {
+  if (!g_scratch_ptr[dev] || g_scratch_ctx[dev] != ctx) {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_scratch) != cudaSuccess || !ptr) {
       cudaGetLastError();
       return ULTRAGEN_ERR_CUDA;
     }
     g_scratch_ptr[dev] = static_cast<float*>(ptr);
+    g_scratch_ctx[dev] = ctx;
   }
   *out = g_scratch_ptr[dev];
   return ULTRAGEN_OK;
@@ -49,6 +75,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 extern "C" int ultragen_hla_forward_noalloc(const void* qp, const void* kp, const void* vp,
                                             void* op, const ultragen_plan_t* cplan, int batch,
                                             ultragen_stream_t stream) {
+  ug::NvtxRange nvtx_range("ultragen_hla_forward_noalloc");
   ultragen_plan_t* p = const_cast<ultragen_plan_t*>(cplan);
   if (!p || !qp || !kp || !vp || !op || batch < 1) return ULTRAGEN_ERR_INVALID_ARG;
   const void* ptrs[] = {qp, kp, vp, op};

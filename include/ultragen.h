@@ -51,7 +51,9 @@ enum ultragen_status {
   ULTRAGEN_ERR_OOM = 4,           /* device allocation failed                            */
   ULTRAGEN_ERR_TIMEOUT = 5,       /* a device-side wait ran past its limit               */
   ULTRAGEN_ERR_PLAN_MISMATCH = 6, /* plan built for another shape / device               */
-  ULTRAGEN_ERR_NO_DEVICE = 7      /* no sm_100 device is current                         */
+  ULTRAGEN_ERR_NO_DEVICE = 7,     /* no sm_100 device is current                         */
+  ULTRAGEN_ERR_BOUNDS = 8         /* a debug build (ULTRAGEN_DEBUG) found a plan index or
+                                     tile coordinate outside its table or tensor             */
 };
 
 enum ultragen_dtype { ULTRAGEN_BF16 = 0, ULTRAGEN_F32 = 1 };
@@ -261,8 +263,9 @@ int ultragen_unpermute(const void* op, void* o, int out_dtype, int batch,
  *   partial the merge reads is written earlier in the same call), it keeps the last call's
  *   contents, and all calls share it: calls that overlap on the GPU (two streams, two
  *   threads) race on it and give wrong results.
- *   The first call on a device looks up the array's device address (cudaGetSymbolAddress);
- *   make that first call before any stream capture.
+ *   The first call on a device (and the first after that device's CUDA context was created
+ *   again, e.g. after cudaDeviceReset) looks up the array's device address
+ *   (cudaGetSymbolAddress); make that first call before any stream capture.
  *   The plan's tables must already be on the current device: any earlier device call with
  *   this plan (e.g. ultragen_permute_rope) uploads them; otherwise ULTRAGEN_ERR_PLAN_MISMATCH.
  *   ULTRAGEN_ERR_UNSUPPORTED when batch * heads * workspace_bytes_per_head (see
@@ -274,7 +277,8 @@ int ultragen_hla_forward_noalloc(const void* qp, const void* kp, const void* vp,
                                  const ultragen_plan_t* plan, int batch, ultragen_stream_t stream);
 
 /* Wait for `stream`, then report (and clear) a device-side error raised by this plan's
- * kernels since the last call: ULTRAGEN_ERR_TIMEOUT if a wait ran out. */
+ * kernels since the last call: ULTRAGEN_ERR_TIMEOUT if a wait ran out, ULTRAGEN_ERR_BOUNDS if a
+ * debug build's index check stopped a kernel. */
 int ultragen_sync_status(const ultragen_plan_t* plan, ultragen_stream_t stream);
 
 /* Diagnostics (no counterpart in the pages).  wait_limit_s (1 ms .. 60 s, default 2 s) bounds
