@@ -12,13 +12,15 @@ import os
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libultragen.so")
+# the in-tree library; ULTRAGEN_LIB_PATH selects another build of it (e.g. the debug build,
+# libultragen_debug.so)
+LIB_PATH = os.environ.get("ULTRAGEN_LIB_PATH") or os.path.join(_HERE, "libultragen.so")
 
 OK = 0
 STATUS = {
     0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "CUDA error",
     4: "out of memory", 5: "device wait timed out", 6: "plan does not match the call",
-    7: "no sm_100 device",
+    7: "no sm_100 device", 8: "index outside its table (debug build check)",
 }
 BF16, F32 = 0, 1
 QK_BF16, QK_E4M3 = 0, 1          # storage of the permuted Q and K (Plan.set_qk_format)

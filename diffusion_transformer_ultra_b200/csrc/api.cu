@@ -8,6 +8,7 @@
 #include <mutex>
 
 #include "kernels.h"
+#include "nvtx_range.h"
 #include "warm_fused.h"
 #include "plan_internal.h"
 
@@ -272,6 +273,8 @@ int launch_attention(const ultragen_plan_t* p, const void* qp, const void* kp, c
   f.raster = raster;
   f.N_raster = (int)p->N_raster;
   f.heads = heads;
+  f.n_entries = (int)p->entries.size();
+  f.n_mask_words = (int)p->mask_pool.size();
   const int grid = (int)std::min<int64_t>(items, sm_count());
   // few items per CTA: hand them out item-major, longest first, so that the last round holds
   // the short ones; otherwise head-major keeps one head's shared key tiles (its LR segment)
@@ -322,6 +325,9 @@ int launch_permute(const ultragen_plan_t* p, const void* q, const void* k, const
   a.perm = p->dev.perm;
   a.slot_pos = p->dev.slot_pos;
   a.rope = p->dev.rope;
+  a.err = p->dev.error;
+  a.rope_rows = std::max(p->H, p->W);
+  a.n_halo_dst = (int)p->halo_dst.size();
   // rows: every Q slot, then the pad slots of the halo blocks (their token slots are written
   // with their source rows)
   const int64_t n_pad = p->halo_copy ? (int64_t)p->halo_pad.size() : 0;
@@ -359,6 +365,7 @@ int ultragen_plan_destroy(ultragen_plan_t* p) {
 int ultragen_permute_rope(const void* q, const void* k, const void* v, int in_dtype, void* qp,
                           void* kp, void* vp, int batch, const ultragen_plan_t* cplan,
                           ultragen_stream_t stream) {
+  ug::NvtxRange nvtx_range("ultragen_permute_rope");
   ultragen_plan_t* p = const_cast<ultragen_plan_t*>(cplan);
   if (!p || !q || !k || !v || !qp || !kp || !vp || batch < 1) return ULTRAGEN_ERR_INVALID_ARG;
   if (in_dtype != ULTRAGEN_BF16 && in_dtype != ULTRAGEN_F32) return ULTRAGEN_ERR_INVALID_ARG;
@@ -416,11 +423,13 @@ static int hla_forward_impl(const void* qp, const void* kp, const void* vp, void
 
 int ultragen_hla_forward(const void* qp, const void* kp, const void* vp, void* op,
                          const ultragen_plan_t* plan, int batch, ultragen_stream_t stream) {
+  ug::NvtxRange nvtx_range("ultragen_hla_forward");
   return hla_forward_impl(qp, kp, vp, op, plan, batch, stream, 0);
 }
 
 int ultragen_hla_forward_raster(const void* qp, const void* kp, const void* vp, void* o,
                                 const ultragen_plan_t* plan, int batch, ultragen_stream_t stream) {
+  ug::NvtxRange nvtx_range("ultragen_hla_forward_raster");
   if (plan && (int64_t)batch * plan->heads * plan->N_raster >= ((int64_t)1 << 31))
     return ULTRAGEN_ERR_UNSUPPORTED;
   return hla_forward_impl(qp, kp, vp, o, plan, batch, stream, 1);
@@ -428,6 +437,7 @@ int ultragen_hla_forward_raster(const void* qp, const void* kp, const void* vp, 
 
 int ultragen_unpermute(const void* op, void* o, int out_dtype, int batch,
                        const ultragen_plan_t* cplan, ultragen_stream_t stream) {
+  ug::NvtxRange nvtx_range("ultragen_unpermute");
   ultragen_plan_t* p = const_cast<ultragen_plan_t*>(cplan);
   if (!p || !op || !o || batch < 1) return ULTRAGEN_ERR_INVALID_ARG;
   if (out_dtype != ULTRAGEN_BF16 && out_dtype != ULTRAGEN_F32) return ULTRAGEN_ERR_INVALID_ARG;
@@ -452,6 +462,7 @@ int ultragen_unpermute(const void* op, void* o, int out_dtype, int batch,
 }
 
 int ultragen_sync_status(const ultragen_plan_t* cplan, ultragen_stream_t stream) {
+  ug::NvtxRange nvtx_range("ultragen_sync_status");
   ultragen_plan_t* p = const_cast<ultragen_plan_t*>(cplan);
   if (!p) return ULTRAGEN_ERR_INVALID_ARG;
   cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
@@ -462,7 +473,7 @@ int ultragen_sync_status(const ultragen_plan_t* cplan, ultragen_stream_t stream)
     return cuda_status(cudaGetLastError());
   if (h != 0) {
     cudaMemset(p->dev.error, 0, sizeof(int));
-    return ULTRAGEN_ERR_TIMEOUT;
+    return h == ug::DEV_BOUNDS ? ULTRAGEN_ERR_BOUNDS : ULTRAGEN_ERR_TIMEOUT;
   }
   return ULTRAGEN_OK;
 }
@@ -472,6 +483,7 @@ int ultragen_last_launch_count(const ultragen_plan_t* p) { return p ? p->last_la
 int ultragen_warm_start(const float* x_lr, const float* noise, float* x_hr, int batch,
                         int channels, int h, int w, int H, int W, float alpha, float sharpen,
                         uint64_t seed, uint64_t offset, ultragen_stream_t stream) {
+  ug::NvtxRange nvtx_range("ultragen_warm_start");
   if (!x_lr || !x_hr || batch < 1 || channels < 1 || h < 1 || w < 1 || H < 1 || W < 1)
     return ULTRAGEN_ERR_INVALID_ARG;
   if (!std::isfinite(alpha) || !std::isfinite(sharpen) || sharpen < 0.0f)

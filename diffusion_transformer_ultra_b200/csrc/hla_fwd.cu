@@ -35,12 +35,31 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <mutex>
 
 #include "exp2_poly.h"
 #include "kernels.h"
 #include "ptx.cuh"
 
+#ifndef ULTRAGEN_DEBUG
+#define ULTRAGEN_DEBUG 0
+#endif
+
 namespace ug {
+
+// Index checks of debug builds (ULTRAGEN_DEBUG): a plan index or tile coordinate outside its
+// table or tensor stops the CTA before the access, the way a timed-out wait does (abort flag,
+// DEV_BOUNDS in the error word).  Release builds compile them away.
+__device__ __forceinline__ bool bounds_fail(volatile int* abort_flag, int* err) {
+  *abort_flag = 1;
+  atomicExch(err, DEV_BOUNDS);
+  return false;
+}
+#if ULTRAGEN_DEBUG
+#define UG_CHECK(cond) ((cond) || bounds_fail(abort_flag, p.err))
+#else
+#define UG_CHECK(cond) true
+#endif
 
 template <int D>
 struct FwdCfg {
@@ -144,6 +163,12 @@ __device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
     int bh;
     const int32_t* I = item_at(p, it, bh);
     const int qt0 = I[0], qt1 = I[1], e0 = I[2], n = I[3] - I[2];
+    if (!UG_CHECK(bh >= 0 && bh < p.units && e0 >= 0 && n >= 0 && e0 + n <= p.n_entries &&
+                  qt0 >= 0 && qt0 * 128 < p.N_tot &&
+                  (qt1 == -1 || (qt1 >= 0 && qt1 * 128 < p.N_tot)))) {
+      ok = false;
+      break;
+    }
     if (n == 0) continue;
     if (!mbar_wait(bar + 8 * C::B_QE, (qi & 1) ^ 1, abort_flag, p.err, DEV_TIMEOUT_PRODUCER,
                    p.timeout_ns)) {
@@ -164,6 +189,11 @@ __device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
         break;
       }
       const uint32_t fb = bar + 8 * (C::B_KVF + g);
+      if (!UG_CHECK((j == 0 || ((__ldg(p.entries + e0 + j - 1) & 0x7fffffff) + 1) * 128 <= p.N_kv) &&
+                    (j == n || ((__ldg(p.entries + e0 + j) & 0x7fffffff) + 1) * 128 <= p.N_kv))) {
+        ok = false;
+        break;
+      }
       mbar_expect_tx(fb, (j > 0 ? C::TILE_BYTES : 0) + (j < n ? QK_BYTES : 0));
       if (j > 0)
         load_tile(tmV, false, sKV + C::v_slot(g) * C::TILE_BYTES,
@@ -345,8 +375,10 @@ __device__ void softmax_role(const FwdParams& p, uint32_t sbase, uint32_t tbase,
     }
     // output row: permuted [bh][slot], or raster [b][token][h] (pad rows have no raster row)
     __nv_bfloat16* orow;
+    if (!UG_CHECK(slot < p.N_tot && ws_slot < p.n_ws_head)) return;
     if (p.raster) {
       const int tok = __ldg(p.perm + slot);
+      if (!UG_CHECK(tok < p.N_raster)) return;
       const int b = bh / p.heads, hh = bh - (bh / p.heads) * p.heads;
       orow = tok >= 0 ? p.out + (((size_t)b * p.N_raster + tok) * p.heads + hh) * D : nullptr;
     } else {
@@ -363,6 +395,9 @@ __device__ void softmax_role(const FwdParams& p, uint32_t sbase, uint32_t tbase,
       const int ent = __ldg(p.entries + e0 + j);
       uint32_t mw[4] = {~0u, ~0u, ~0u, ~0u};
       if (ent < 0) {
+        if (!UG_CHECK(__ldg(p.mask_off + e0 + j) >= 0 &&
+                      __ldg(p.mask_off + e0 + j) + cls * 4 + 4 <= p.n_mask_words))
+          return;
         const uint32_t* mp = p.mask_pool + __ldg(p.mask_off + e0 + j) + cls * 4;
 #pragma unroll
         for (int w = 0; w < 4; ++w) mw[w] = __ldg(mp + w);
@@ -567,19 +602,30 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D, bool QK8>
 static cudaError_t launch_d(const void* tmQ, const void* tmK, const void* tmV, const FwdParams& p,
                             int grid, cudaStream_t st) {
-  static bool attr_set = false;
+  // The shared-memory size attribute belongs to the kernel on each device: set it once per
+  // device (one process may drive several GPUs, from several threads).
+  constexpr int kMaxDev = 64;
+  static std::mutex mu;
+  static bool attr_set[kMaxDev] = {};
   const int smem = FwdCfg<D>::SMEM_BYTES;
-  if (!attr_set) {
-    // The register split above is only sound if the kernel really launches with
-    // kRegsLaunch registers per thread; refuse to launch otherwise.
-    cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, hla_fwd_kernel<D, QK8>);
-    if (e != cudaSuccess) return e;
-    if (fa.numRegs != kRegsLaunch) return cudaErrorInvalidConfiguration;
-    e = cudaFuncSetAttribute(hla_fwd_kernel<D, QK8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!attr_set[dev]) {
+      // The register split above is only sound if the kernel really launches with
+      // kRegsLaunch registers per thread; refuse to launch otherwise.
+      cudaFuncAttributes fa;
+      e = cudaFuncGetAttributes(&fa, hla_fwd_kernel<D, QK8>);
+      if (e != cudaSuccess) return e;
+      if (fa.numRegs != kRegsLaunch) return cudaErrorInvalidConfiguration;
+      e = cudaFuncSetAttribute(hla_fwd_kernel<D, QK8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               smem);
+      if (e != cudaSuccess) return e;
+      attr_set[dev] = true;
+    }
   }
   hla_fwd_kernel<D, QK8><<<grid, kThreads, smem, st>>>(*static_cast<const CUtensorMap*>(tmQ),
                                                         *static_cast<const CUtensorMap*>(tmK),

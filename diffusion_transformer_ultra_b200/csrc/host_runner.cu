@@ -16,6 +16,7 @@
 #include <new>
 
 #include "kernels.h"
+#include "nvtx_range.h"
 #include "plan_internal.h"
 
 struct ultragen_host_runner {
@@ -117,6 +118,7 @@ int ultragen_host_runner_create(ultragen_plan_t* p, int batch, int heads_per_chu
 
 int ultragen_host_runner_forward(ultragen_host_runner_t* r, const void* q, const void* k,
                                  const void* v, void* o, ultragen_stream_t stream) {
+  ug::NvtxRange nvtx_range("ultragen_host_runner_forward");
   if (!r || !q || !k || !v || !o) return ULTRAGEN_ERR_INVALID_ARG;
   ultragen_plan_t* p = r->plan;
   int dev = -1;

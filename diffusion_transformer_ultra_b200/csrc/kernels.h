@@ -45,6 +45,10 @@ struct PermuteArgs {
   const int32_t* halo_dst;
   int off_hr, N_hrp;
   int pair_a0, pair_a01;           // pairs [0,a0) axis 0, [a0,a01) axis 1, rest axis 2
+  // index checks of debug builds (ULTRAGEN_DEBUG): the device error word and table sizes
+  int* err = nullptr;
+  int rope_rows = 0;               // rows of the cos/sin table
+  int n_halo_dst = 0;              // halo-copy targets
 };
 
 struct UnpermuteArgs {
@@ -93,7 +97,13 @@ struct FwdParams {
   int fault = 0;                   // 1: withhold one "S ready" signal (tests the timeout path)
   int raster = 0;                  // 1: out is raster [B, N_raster, heads, D] (pad rows skipped)
   int N_raster = 0, heads = 1;
+  int n_entries = 0;               // table sizes for the index checks of debug builds
+  int n_mask_words = 0;
 };
+
+// Device error codes shared by the kernels and the host (ultragen_sync_status): the bounded
+// waits write DEV_TIMEOUT_* (ptx.cuh); the index checks of debug builds write DEV_BOUNDS.
+constexpr int DEV_BOUNDS = 0x105;
 
 struct WarmArgs {
   const float* lr;                 // [planes, h, w] low-resolution latent

@@ -14,9 +14,24 @@
 
 #include "kernels.h"
 
+#ifndef ULTRAGEN_DEBUG
+#define ULTRAGEN_DEBUG 0
+#endif
+
 namespace ug {
 
 namespace {
+
+// Index checks of debug builds (ULTRAGEN_DEBUG): a plan index outside its table is recorded in
+// the device error word (DEV_BOUNDS) and the row is skipped instead of read or written.
+// Release builds compile them away.
+__device__ __forceinline__ bool index_ok(bool cond, int* err) {
+  if (ULTRAGEN_DEBUG && !cond) {
+    if (err) atomicExch(err, DEV_BOUNDS);
+    return false;
+  }
+  return true;
+}
 
 __device__ __forceinline__ void load8(const __nv_bfloat16* src, float (&x)[8]) {
   const uint4 u = __ldg(reinterpret_cast<const uint4*>(src));
@@ -98,7 +113,9 @@ __global__ void __launch_bounds__(256) permute_rope_kernel(PermuteArgs a) {
       // indices past N_tot are the halo blocks' pad slots; their token slots are written with
       // the source token's row below
       const int slot = idx < a.N_tot ? idx : __ldg(a.halo_pad + (idx - a.N_tot));
+      if (!index_ok(slot >= 0 && slot < a.N_kv, a.err)) continue;
       const int r = __ldg(a.perm + slot);
+      if (!index_ok(r < a.N_raster, a.err)) continue;
       kvb[u] = (b * a.heads + h) * a.N_kv;
       dst[u] = kvb[u] + slot;
       if (idx < a.N_tot) dq[u] = (b * a.heads + h) * a.N_tot + slot;
@@ -107,6 +124,11 @@ __global__ void __launch_bounds__(256) permute_rope_kernel(PermuteArgs a) {
       const uint32_t sp = __ldg(a.slot_pos + slot);
       pos_r[u] = (int)(sp >> 16);
       pos_c[u] = (int)(sp & 0xffffu);
+      if (!index_ok(pos_r[u] < a.rope_rows && pos_c[u] < a.rope_rows, a.err)) {
+        dst[u] = dq[u] = -1;
+        real[u] = false;
+        continue;
+      }
       const int64_t src = ((int64_t)(b * a.N_raster + r) * a.heads + h) * D + c * 8;
       load8(qin + src, xq[u]);
       load8(kin + src, xk[u]);
@@ -115,6 +137,7 @@ __global__ void __launch_bounds__(256) permute_rope_kernel(PermuteArgs a) {
       if (a.halo_ptr && k >= 0 && k < a.N_hrp) {
         hb[u] = __ldg(a.halo_ptr + k);
         he[u] = __ldg(a.halo_ptr + k + 1);
+        if (!index_ok(hb[u] >= 0 && he[u] <= a.n_halo_dst, a.err)) he[u] = hb[u] = 0;
         if (he[u] > hb[u]) h0[u] = __ldg(a.halo_dst + hb[u]);
       }
     }
@@ -169,6 +192,7 @@ __global__ void __launch_bounds__(256) permute_rope_kernel(PermuteArgs a) {
         // with the row)
         for (int e = hb[u]; e < he[u]; ++e) {
           const int tgt = e == hb[u] ? h0[u] : __ldg(a.halo_dst + e);
+          if (!index_ok(tgt >= 0 && tgt < a.N_kv, a.err)) continue;
           const int64_t oh = (int64_t)(kvb[u] + tgt) * D + c * 8;
           if (QK8)
             *reinterpret_cast<uint2*>(static_cast<uint8_t*>(a.out[1]) + oh) = ok8;

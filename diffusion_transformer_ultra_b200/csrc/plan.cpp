@@ -18,6 +18,7 @@
 #include <cstring>
 #include <new>
 
+#include "nvtx_range.h"
 #include "plan_internal.h"
 
 namespace ug {
@@ -538,12 +539,14 @@ const char* ultragen_status_string(int s) {
     case ULTRAGEN_ERR_TIMEOUT: return "device wait timed out";
     case ULTRAGEN_ERR_PLAN_MISMATCH: return "plan does not match the call";
     case ULTRAGEN_ERR_NO_DEVICE: return "no sm_100 device";
+    case ULTRAGEN_ERR_BOUNDS: return "index outside its table (debug build check)";
     default: return "unknown status";
   }
 }
 
 int ultragen_plan(int H, int W, int l, int b, int rho, int text_len, int heads, int head_dim,
                   ultragen_plan_t** out) {
+  ug::NvtxRange nvtx_range("ultragen_plan");
   if (!out) return ULTRAGEN_ERR_INVALID_ARG;
   *out = nullptr;
   if (H < 1 || W < 1 || l < 1 || b < 0 || rho < 0 || text_len < 0 || heads < 1)
