@@ -67,9 +67,19 @@ def parse():
     ap.add_argument("--e2e-heads-per-chunk", type=int, default=2,
                     help="head slice per pipelined unit of the host-buffer (e2e) measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--split", default="layers", choices=["layers", "heads"],
+                    help="multi-GPU: layers = an independent layer per rank (weak scaling); heads = "
+                         "one layer's heads split across the ranks (strong scaling)")
+    ap.add_argument("--extra-workloads", default=None,
+                    help="comma list of further workloads timed after the main one and reported "
+                         "under 'workloads' (default: 8k,1k,ragged for the default 4k run; "
+                         "'none' to skip)")
     args = ap.parse_args()
+    default_run = args.workload is None
     if args.workload is None:
         args.workload = "warm_8k" if args.op == "warm_start" else "4k"
+    if args.extra_workloads is None:
+        args.extra_workloads = "8k,1k,ragged" if default_run and args.op == "hla" else "none"
     return args
 
 
@@ -235,11 +245,32 @@ def cpu_model() -> str:
     return ""
 
 
+def blas_threads():
+    """Threads of the BLAS libraries NumPy uses, as threadpoolctl reports them."""
+    try:
+        from threadpoolctl import threadpool_info
+        return max((i.get("num_threads") or 0 for i in threadpool_info()
+                    if i.get("user_api") == "blas"), default=None)
+    except Exception:
+        return None
+
+
+def inputs_sha256(*tensors) -> str:
+    """SHA-256 of the input tensors' bytes, in order (the exact bf16 values timed)."""
+    h = hashlib.sha256()
+    for t in tensors:
+        h.update(t.contiguous().view(-1).view(__import__("torch").uint8).numpy().tobytes())
+    return h.hexdigest()
+
+
 def cpu_baseline(wl, q, k, v, budget_s: float = 12.0, lr_radius: int = -1, lr_block: bool = False,
-                 **fwd):
+                 one_core: bool = True, **fwd):
     """The oracle as it stands, timed on this host on a bounded sample: one head, rows of one
-    interior window plus text and LR rows, growing until about `budget_s` of CPU work
-    (``fwd``: the oracle forward's Q/K format options)."""
+    interior window plus text and LR rows, repeated until about `budget_s` of CPU work, with
+    the BLAS libraries on all cores and (one_core) again on one core.  The dense oracle costs
+    the same per query row whatever its segment (every row is scored against all N_tot keys),
+    so the time per sampled row, times the layer's rows, heads and batch, extrapolates to the
+    whole layer (``fwd``: the oracle forward's Q/K format options)."""
     import numpy as np
 
     from oracle import hla_oracle as O
@@ -253,19 +284,40 @@ def cpu_baseline(wl, q, k, v, budget_s: float = 12.0, lr_radius: int = -1, lr_bl
     rows = np.array(sorted(set(rows)), np.int64)
     vis_pairs = int(O.visible_rows(g, rows).sum())
     qh, kh, vh = (x[:1, :, :1, :].to(dtype=__import__("torch").float64).numpy() for x in (q, k, v))
-    t0 = time.perf_counter()
-    reps = 0
-    while True:
-        O.forward(qh, kh, vh, g, wl.axes, rows=rows, **fwd)
-        reps += 1
-        if time.perf_counter() - t0 > budget_s:
-            break
-    dt = (time.perf_counter() - t0) / reps
+
+    def timed(budget):
+        t0 = time.perf_counter()
+        reps = 0
+        while True:
+            O.forward(qh, kh, vh, g, wl.axes, rows=rows, **fwd)
+            reps += 1
+            if time.perf_counter() - t0 > budget:
+                break
+        return (time.perf_counter() - t0) / reps, reps
+
+    dt, reps = timed(budget_s)
+    threads = blas_threads()
     flops = 4.0 * wl.D * vis_pairs
-    return {"value": flops / dt / 1e12, "unit": "useful TFLOP/s", "cores": os.cpu_count(),
-            "cpu_model": cpu_model(), "kind": "oracle",
-            "sample": f"1 head, {len(rows)} query rows ({vis_pairs} visible pairs), full RoPE + "
-                      f"explicit mask, fp64 NumPy; {reps} rep(s), {dt:.2f} s each"}
+    real_rows = wl.n_raster                         # every real token is one query row
+    full_s = dt / len(rows) * real_rows * wl.heads * wl.batch
+    out = {"value": flops / dt / 1e12, "unit": "useful TFLOP/s", "cores": os.cpu_count(),
+           "blas_threads": threads, "cpu_model": cpu_model(), "kind": "oracle",
+           "sample": f"1 head, {len(rows)} query rows ({vis_pairs} visible pairs), full RoPE + "
+                     f"explicit mask, fp64 NumPy; {reps} rep(s), {dt:.2f} s each",
+           "full_layer_s_extrapolated": full_s,
+           "full_layer_note": f"extrapolated: {dt / len(rows) * 1e3:.2f} ms per sampled query row x "
+                              f"{real_rows} rows x {wl.heads} heads x batch {wl.batch}"}
+    if one_core:
+        try:
+            from threadpoolctl import threadpool_limits
+            with threadpool_limits(limits=1):
+                dt1, reps1 = timed(budget_s / 2)
+            out["one_core"] = {"value": flops / dt1 / 1e12, "unit": "useful TFLOP/s",
+                               "blas_threads": 1, "s_per_rep": dt1, "reps": reps1,
+                               "full_layer_s_extrapolated": dt1 / len(rows) * real_rows * wl.heads * wl.batch}
+        except Exception as e:            # threadpoolctl missing: say so instead of guessing
+            out["one_core"] = {"unavailable": str(e)}
+    return out
 
 
 def run_reference(args, rank, world):
@@ -279,7 +331,7 @@ def run_reference(args, rank, world):
     base = None
     for i in range(args.warmup + args.steps):
         t0 = time.perf_counter()
-        r = cpu_baseline(wl, q, k, v, budget_s=0.0)
+        r = cpu_baseline(wl, q, k, v, budget_s=0.0, one_core=False)
         if i >= args.warmup:
             per_step.append(time.perf_counter() - t0)
             base = r
@@ -292,7 +344,8 @@ def run_reference(args, rank, world):
         "config": {"workload": wl.name, "H": wl.H, "W": wl.W, "l": wl.l, "b": wl.b, "rho": wl.rho,
                    "text_len": wl.T, "heads": wl.heads, "head_dim": wl.D, "batch": wl.batch},
         "cpu_baseline": {"kind": "oracle", "cores": base["cores"], "cpu_model": base["cpu_model"],
-                         "sample": base["sample"],
+                         "blas_threads": base["blas_threads"], "sample": base["sample"],
+                         "full_layer_s_extrapolated": base["full_layer_s_extrapolated"],
                          "value": value, "unit": "useful TFLOP/s"},
         "e2e": {"value": value, "unit": "useful TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
@@ -457,32 +510,33 @@ def main_warm(args, rank, world, local):
         dist.destroy_process_group()
 
 
-def main():
-    args = parse()
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.op == "warm_start":
-        main_warm(args, rank, world, local)
-        return
-    if args.impl == "reference":
-        run_reference(args, rank, world)
-        return
+def roofline_peak(pk, src, e4m3: bool):
+    """The tensor roofline denominators: the measured burst dense-bf16 figure for `frac` (one
+    denominator for every workload), the power-capped sustained one beside it."""
+    burst, sust = pk["bf16_tflops"], pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    note = f"{src} bf16 dense, burst (frac); sustained under the power cap (frac_sustained)"
+    if e4m3:
+        # half the useful FLOPs (Q K^T) at the e4m3 rate, nominally twice the bf16 rate, half
+        # (P V) at the bf16 rate: the mixed peak is 1 / (0.5 / 2P + 0.5 / P) = 4P / 3
+        burst, sust = burst * 4.0 / 3.0, sust * 4.0 / 3.0
+        note += "; x 4/3 (nominal ratio, not a measured e4m3 peak) for the mixed e4m3 Q K^T + bf16 P V"
+    return burst, sust, note
+
+
+def measure_layer(ug, args, wl, world, local, rank, heads_range=None, with_e2e=False,
+                  with_cpu=False):
+    """One workload: build the plan, time `args.steps` steps (permute_rope, attention with the
+    unpermute in its epilogue, the split merge when there is one) after the warm-up, and return
+    its record.  heads_range = (h0, h1): this rank runs those heads of the layer (split mode)."""
+    import dataclasses
 
     import torch
     import torch.distributed as dist
 
-    import diffusion_transformer_ultra_b200 as ug
-    torch.cuda.set_device(local)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
-
-    wl = ug.WORKLOADS[args.workload]
-    if args.heads:
-        import dataclasses
-        wl = dataclasses.replace(wl, heads=args.heads)
-    plan = ug.plan_for(wl)
+    full_heads = wl.heads
+    h0, h1 = heads_range if heads_range else (0, wl.heads)
+    wlr = dataclasses.replace(wl, heads=h1 - h0) if heads_range else wl
+    plan = ug.plan_for(wlr)
     if args.lr_radius != -1:
         plan.set_lr_scope(args.lr_radius)
     if args.lr_order != -1:
@@ -494,9 +548,13 @@ def main():
         plan.set_qk_format("e4m3", args.q_exp, args.k_exp)
     info = plan.info
     q, k, v = ug.make_qkv(wl)
+    sha = inputs_sha256(q, k, v) if rank == 0 else None
+    if heads_range:
+        from diffusion_transformer_ultra_b200.sharding import head_slice
+        q, k, v = (head_slice(x, h0, h1) for x in (q, k, v))
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
-    lay = ug.Layer(plan, wl.batch)
-    o = torch.empty((wl.batch, info["N_raster"], wl.heads, wl.D), dtype=torch.bfloat16, device="cuda")
+    lay = ug.Layer(plan, wlr.batch)
+    o = torch.empty((wlr.batch, info["N_raster"], wlr.heads, wlr.D), dtype=torch.bfloat16, device="cuda")
     stream = torch.cuda.current_stream()
 
     def step(evs=None):
@@ -549,34 +607,43 @@ def main():
     ms_attn = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     ms_unperm = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
     ms_step = max_over_ranks(ms_total, world, "cuda") / args.steps
+    ms_attn_max = max_over_ranks(ms_attn, world, "cuda")
 
-    flops = 4.0 * wl.D * info["useful_pairs"] * wl.heads * wl.batch
-    value = job_tflops(flops, world, ms_step)
+    flops_rank = 4.0 * wlr.D * info["useful_pairs"] * wlr.heads * wlr.batch
+    flops_layer = 4.0 * wl.D * info["useful_pairs"] * full_heads * wl.batch
+    if heads_range:   # strong scaling: the job is one layer, done when the slowest rank is
+        value = flops_layer / (ms_step * 1e-3) / 1e12
+    else:             # weak scaling: every rank runs its own layer
+        value = job_tflops(flops_rank, world, ms_step)
     pk, src = peaks()
-    attn_tflops = flops / (ms_attn * 1e-3) / 1e12
-    elem = wl.batch * wl.heads * info["N_tot"] * wl.D
-    kv_elem = wl.batch * wl.heads * info["N_kv"] * wl.D
+    attn_tflops = flops_rank / (ms_attn * 1e-3) / 1e12
+    elem = wlr.batch * wlr.heads * info["N_tot"] * wlr.D
+    kv_elem = wlr.batch * wlr.heads * info["N_kv"] * wlr.D
     in_size = 2 if wl.dtype == "bf16" else 4
     qk_size = 1 if e4m3 else 2
     # permute_rope: every raster row of Q, K, V read once (halo copies are written from the
     # same read), Q written over N_tot slots and K, V over N_kv slots (pad slots as zeros)
-    perm_bytes = (3 * wl.batch * info["N_raster"] * wl.heads * wl.D * in_size
+    perm_bytes = (3 * wlr.batch * info["N_raster"] * wlr.heads * wlr.D * in_size
                   + (elem + kv_elem) * qk_size + kv_elem * 2)
-    unperm_bytes = elem * 2 + wl.batch * info["N_raster"] * wl.heads * wl.D * 2
-    traffic = profiled_traffic(wl.name + ("-e4m3" if e4m3 else ""))
+    perm_bytes_method = 6 * wlr.batch * info["N_raster"] * wlr.heads * wlr.D * in_size
+    unperm_bytes = elem * 2 + wlr.batch * info["N_raster"] * wlr.heads * wlr.D * 2
+    traffic = None if heads_range else profiled_traffic(wl.name + ("-e4m3" if e4m3 else ""))
+    burst, sust, peak_note = roofline_peak(pk, src, e4m3)
 
     e2e = None
-    if not args.no_e2e:
+    if with_e2e and not args.no_e2e:
         # the public host-buffer call: page-locked Q/K/V in, O out, copies overlapped with the
         # kernels of other head slices
         qh, kh, vh = (x.to(torch.bfloat16).pin_memory() for x in (q, k, v))
         oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-        runner = ug.HostRunner(plan, wl.batch, args.e2e_heads_per_chunk)
+        runner = ug.HostRunner(plan, wlr.batch, args.e2e_heads_per_chunk)
         for _ in range(2):
             runner(qh, kh, vh, oh)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         n_e2e = max(3, args.steps // 4)
+        if world > 1:
+            dist.barrier()
         e0.record(stream)
         for _ in range(n_e2e):
             runner(qh, kh, vh, oh)
@@ -585,7 +652,9 @@ def main():
         if plan.sync_status() != 0:
             raise RuntimeError("device error during the end-to-end steps")
         ms_e2e = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world, "cuda")
-        e2e = {"value": job_tflops(flops, world, ms_e2e), "unit": "useful TFLOP/s",
+        e2e_value = (flops_layer / (ms_e2e * 1e-3) / 1e12 if heads_range
+                     else job_tflops(flops_rank, world, ms_e2e))
+        e2e = {"value": e2e_value, "unit": "useful TFLOP/s",
                "ms_per_step": ms_e2e, "api": "ultragen_host_runner_forward (host buffers)",
                "heads_per_chunk": args.e2e_heads_per_chunk,
                "h2d_bytes_per_step": 3 * qh.numel() * qh.element_size(),
@@ -593,59 +662,112 @@ def main():
         runner.close()
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if with_cpu and rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl, q, k, v, lr_radius=args.lr_radius, lr_block=bool(info["lr_block"]),
                            **({"qk_format": "e4m3", "q_exp": args.q_exp, "k_exp": args.k_exp}
                               if e4m3 else {}))
 
-    # roofline denominator: the burst bf16 figure while the SM clock held its maximum during
-    # the timed steps, the sustained (power-capped) one once the clock dropped under the cap
-    capped = bool(clocks.get("sm_mhz") and clocks.get("sm_max_mhz")
-                  and clocks["sm_mhz"] < 0.97 * clocks["sm_max_mhz"])
-    if capped:
-        peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
-        peak_note = f"{src} bf16 dense, sustained (the power cap held the SM clock at {clocks.get('sm_mhz')} MHz)"
-    else:
-        peak = pk["bf16_tflops"]
-        peak_note = f"{src} bf16 dense, burst (SM clock at its maximum during the timed steps)"
-    if e4m3:
-        # half the useful FLOPs (Q K^T) at the e4m3 rate, nominally twice the bf16 rate, half
-        # (P V) at the bf16 rate: the mixed peak is 1 / (0.5 / 2P + 0.5 / P) = 4P / 3
-        peak *= 4.0 / 3.0
-        peak_note += "; x 4/3 for the mixed e4m3 Q K^T (nominal 2x bf16) + bf16 P V contraction"
+    rec = {
+        "workload": wl.name + ("" if args.lr_radius < 0 else f"-lr-region-r{args.lr_radius}")
+                    + ("-e4m3-qk" if e4m3 else ""),
+        "value": value, "unit": "useful TFLOP/s", "ms_per_step": ms_step,
+        "ms_per_layer_attention": ms_attn_max,
+        "config": {"H": wl.H, "W": wl.W, "l": wl.l, "b": wl.b, "rho": wl.rho, "text_len": wl.T,
+                   "lr_radius": args.lr_radius, "heads": full_heads, "head_dim": wl.D,
+                   "batch": wl.batch, "N_tot": info["N_tot"],
+                   "useful_pairs_per_head": info["useful_pairs"],
+                   "halo_blocks": bool(info["halo_copy"]), "N_kv": info["N_kv"],
+                   "lr_blocks": bool(info["lr_block"]), "qk_format": args.qk,
+                   **({"q_exp": args.q_exp, "k_exp": args.k_exp} if e4m3 else {}),
+                   "inputs_sha256": sha,
+                   "l2": "inputs larger than L2 (permuted Q %.0f MB, K %.0f MB, V %.0f MB); no flush"
+                         % (elem * qk_size / 1e6, kv_elem * qk_size / 1e6, kv_elem * 2 / 1e6)
+                         if elem * qk_size > 126e6 else
+                         "inputs smaller than L2 (permuted Q %.0f MB); steady-state layer, no flush"
+                         % (elem * qk_size / 1e6)},
+        "ms_per_kernel": {"permute_rope": ms_perm, "hla_forward": ms_attn,
+                          "unpermute": ms_unperm if args.unfused else "in hla_forward's epilogue"},
+        "path": "permute_rope + hla_forward + unpermute" if args.unfused
+                else "permute_rope + hla_forward_raster (unpermute fused)",
+        "hla_forward_tflops": attn_tflops,
+        "permute_rope_gbs": perm_bytes / (ms_perm * 1e-3) / 1e9,
+        "permute_rope_gbs_method_bytes": perm_bytes_method / (ms_perm * 1e-3) / 1e9,
+        "unpermute_gbs": unperm_bytes / (ms_unperm * 1e-3) / 1e9 if args.unfused else None,
+        "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": burst, "unit": "TFLOP/s",
+                     "frac": attn_tflops / burst, "frac_sustained": attn_tflops / sust,
+                     "peak_sustained": sust, "traffic": traffic, "peak_source": peak_note,
+                     "algorithmic_flops_per_launch": flops_rank},
+        "e2e": e2e, "gpu_launches": launches, "clocks": clocks, "cpu_baseline": cpu,
+    }
+    del qd, kd, vd, lay, o, plan
+    torch.cuda.empty_cache()
+    return rec
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.op == "warm_start":
+        main_warm(args, rank, world, local)
+        return
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import diffusion_transformer_ultra_b200 as ug
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    def workload(name):
+        wl = ug.WORKLOADS[name]
+        if args.heads:
+            import dataclasses
+            wl = dataclasses.replace(wl, heads=args.heads)
+        return wl
+
+    def heads_of(wl):
+        if args.split != "heads" or world == 1:
+            return None
+        from diffusion_transformer_ultra_b200.sharding import head_range
+        return head_range(wl.heads, world, rank)
+
+    wl = workload(args.workload)
+    main_rec = measure_layer(ug, args, wl, world, local, rank, heads_of(wl), with_e2e=True,
+                             with_cpu=True)
+    extra = {}
+    for name in [w for w in args.extra_workloads.split(",") if w and w != "none"]:
+        if name == args.workload:
+            continue
+        ew = workload(name)
+        extra[name] = measure_layer(ug, args, ew, world, local, rank, heads_of(ew))
     if rank == 0:
+        split = heads_of(wl)
         line = {
-            "metric": METRIC, "value": value, "unit": "useful TFLOP/s", "n_gpus": world,
-            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "e4m3 Q.K^T (fp32 acc) + bf16 P.V" if e4m3 else "bf16",
+            "metric": METRIC, "value": main_rec["value"], "unit": "useful TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": main_rec["ms_per_step"],
+            "higher_is_better": True, "scaling": "strong" if split else "weak", "vs_baseline": None,
+            "dtype": "e4m3 Q.K^T (fp32 acc) + bf16 P.V" if args.qk == "e4m3" else "bf16",
             "data": "synthetic (seeded N(0,1) + smooth 2D sinusoid Q/K/V; no weights needed)",
-            "config": {"workload": wl.name + ("" if args.lr_radius < 0 else f"-lr-region-r{args.lr_radius}")
-                                   + ("-e4m3-qk" if e4m3 else ""),
-                       "H": wl.H, "W": wl.W, "l": wl.l, "b": wl.b,
-                       "rho": wl.rho, "text_len": wl.T, "lr_radius": args.lr_radius, "heads": wl.heads, "head_dim": wl.D,
-                       "batch": wl.batch, "N_tot": info["N_tot"], "useful_pairs_per_head": info["useful_pairs"],
-                       "halo_blocks": bool(info["halo_copy"]), "N_kv": info["N_kv"],
-                       "lr_blocks": bool(info["lr_block"]),
-                       "qk_format": args.qk, **({"q_exp": args.q_exp, "k_exp": args.k_exp} if e4m3 else {}),
-                       "l2": "inputs larger than L2 (permuted Q %.0f MB, K %.0f MB, V %.0f MB); no flush"
-                             % (elem * qk_size / 1e6, kv_elem * qk_size / 1e6, kv_elem * 2 / 1e6),
-                       "parallelism": f"independent layer per rank x{world}"},
-            "ms_per_kernel": {"permute_rope": ms_perm, "hla_forward": ms_attn,
-                              "unpermute": ms_unperm if args.unfused else "in hla_forward's epilogue"},
-            "path": "permute_rope + hla_forward + unpermute" if args.unfused
-                    else "permute_rope + hla_forward_raster (unpermute fused)",
-            "hla_forward_tflops": attn_tflops,
-            "permute_rope_gbs": perm_bytes / (ms_perm * 1e-3) / 1e9,
-            "unpermute_gbs": unperm_bytes / (ms_unperm * 1e-3) / 1e9 if args.unfused else None,
-            "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
-                         "frac": attn_tflops / peak, "traffic": traffic,
-                         "peak_source": peak_note,
-                         "algorithmic_flops_per_launch": flops},
-            "e2e": e2e,
-            "gpu_launches": launches,
-            "clocks": clocks,
-            "cpu_baseline": cpu,
+            "config": {"workload": main_rec["workload"], **main_rec["config"],
+                       "parallelism": (f"heads split across {world} ranks (rank 0: heads "
+                                       f"{split[0]}..{split[1] - 1}), no data exchange" if split
+                                       else f"independent layer per rank x{world}")},
+            **{k_: main_rec[k_] for k_ in ("ms_per_kernel", "path", "hla_forward_tflops",
+                                           "permute_rope_gbs", "permute_rope_gbs_method_bytes",
+                                           "unpermute_gbs", "roofline", "e2e", "gpu_launches",
+                                           "clocks", "cpu_baseline")},
+            "workloads": {n: {k_: r[k_] for k_ in ("value", "unit", "ms_per_step",
+                                                    "ms_per_layer_attention", "hla_forward_tflops",
+                                                    "ms_per_kernel", "roofline", "clocks",
+                                                    "gpu_launches", "permute_rope_gbs")}
+                          | {"config": r["config"]} for n, r in extra.items()},
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -63,3 +63,27 @@ def test_host_runner_pageable_memory(ug):
     torch.cuda.synchronize()
     assert plan.sync_status() == 0
     assert torch.equal(oh.view(torch.int16), o_dev.cpu().view(torch.int16))
+
+
+def test_host_runner_at_the_benchmarked_4k_configuration(ug):
+    """The end-to-end figure's own call: the 4K layer in bf16 with the plan's automatic choice
+    (compact halo blocks at 4K) and 2-head units, bit for bit the device path's output."""
+    import torch
+    wl = ug.WORKLOADS["4k"]
+    plan = ug.plan_for(wl)
+    assert plan.info["halo_copy"] > 0          # the automatic choice takes halo blocks here
+    q, k, v = ug.make_qkv(wl)
+    shape = (wl.batch, plan.info["N_raster"], wl.heads, wl.D)
+    lay = ug.Layer(plan, wl.batch)
+    o_dev = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+    lay(q.cuda(), k.cuda(), v.cuda(), o_dev)
+    torch.cuda.synchronize()
+    assert plan.sync_status() == 0
+    qh, kh, vh = (x.pin_memory() for x in (q, k, v))
+    oh = torch.full(shape, float("nan"), dtype=torch.bfloat16).pin_memory()
+    run = ug.HostRunner(plan, wl.batch, 2)
+    run(qh, kh, vh, oh)
+    torch.cuda.synchronize()
+    assert plan.sync_status() == 0
+    assert torch.equal(oh.view(torch.int16), o_dev.cpu().view(torch.int16))
+    run.close()

@@ -214,6 +214,37 @@ def test_attention_full_size_sampled(ug, name, heads):
         check_attention(got[:, real], ref[:, real], f"{name} b={b}")
 
 
+@pytest.mark.parametrize("name,heads,windows", [("4k", (0, 12, 23), "corners"),
+                                                 ("8k", (0, 11, 23), "corners")])
+def test_benchmarked_raster_call_at_full_size(ug, name, heads, windows):
+    """The call bench.py times, in its own configuration: permute_rope + hla_forward_raster on
+    the default plan (all LR tokens, compact halo blocks chosen automatically), checked on the
+    raster output against the oracle for sampled rows of three heads, the corner (edge)
+    windows and the centre window among them."""
+    import torch
+    wl = _wl(name)
+    plan = ug.plan_for(wl)
+    assert plan.info["halo_copy"] > 0
+    q, k, v = ug.make_qkv(wl)
+    lay = ug.Layer(plan, wl.batch)
+    o = torch.full((wl.batch, plan.info["N_raster"], wl.heads, wl.D), float("nan"),
+                   dtype=torch.bfloat16, device="cuda")
+    ug.permute_rope(q.cuda(), k.cuda(), v.cuda(), lay.qp, lay.kp, lay.vp, plan)
+    ug.hla_forward_raster(lay.qp, lay.kp, lay.vp, o, plan)
+    assert plan.sync_status() == 0
+    torch.cuda.synchronize()
+    assert not torch.isnan(o).any()
+    g = geometry(wl)
+    rows = sample_rows(wl, n_text=128, n_lr=128, windows=windows)
+    tok = O.perm_map(g)[rows]
+    real = tok >= 0
+    rows, tok = rows[real], tok[real]
+    got_all = o[0][torch.as_tensor(tok, device="cuda")]            # [rows, heads, D]
+    ref = oracle_rows(q, k, v, wl, 0, heads, rows)
+    got = np.stack([to_np64(got_all[:, h]) for h in heads])
+    check_attention(got, ref, f"{name} raster, heads {heads}")
+
+
 @pytest.mark.parametrize("name,r,heads,order", [("1k", 4, (0, 11, 23), None), ("tiny", 0, (0,), None),
                                                 ("4k", 4, (9,), None), ("8k", 0, (2,), None),
                                                 ("1k", 4, (0, 23), 1), ("tiny", 0, (0,), 1),
