@@ -218,20 +218,20 @@ __device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
 template <int D, bool QK8>
 __device__ __forceinline__ void issue_s(uint32_t tmem_d, uint32_t sQt, uint32_t sK) {
   using C = FwdCfg<D>;
+  constexpr uint32_t hi = desc_hi_sw128(1024);
+  const uint32_t qlo = desc_lo(sQt, 16), klo = desc_lo(sK, 16);
   if (QK8) {
     // e4m3 rows of 128 bytes: each product takes the next 32 bytes (32 K-elements) of the row
     constexpr uint32_t idS = idesc_e4m3(128, 128);
 #pragma unroll
     for (int kk = 0; kk < D / 32; ++kk)
-      mma_ss_f8(tmem_d, smem_desc_sw128(sQt + kk * 32, 16, 1024),
-                smem_desc_sw128(sK + kk * 32, 16, 1024), idS, kk > 0 ? 1u : 0u);
+      mma_ss_f8_w(tmem_d, qlo + kk * 2, klo + kk * 2, hi, idS, kk > 0 ? 1u : 0u);
   } else {
     constexpr uint32_t idS = idesc_bf16(128, 128, 0);
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
-      const uint32_t off = (kk / 4) * C::BOX_BYTES + (kk % 4) * 32;
-      mma_ss(tmem_d, smem_desc_sw128(sQt + off, 16, 1024), smem_desc_sw128(sK + off, 16, 1024),
-             idS, kk > 0 ? 1u : 0u);
+      const uint32_t off = ((kk / 4) * C::BOX_BYTES + (kk % 4) * 32) >> 4;
+      mma_ss_w(tmem_d, qlo + off, klo + off, hi, idS, kk > 0 ? 1u : 0u);
     }
   }
 }
@@ -241,11 +241,12 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem_d, uint32_t tmem_p, uint3
                                          bool accumulate) {
   using C = FwdCfg<D>;
   constexpr uint32_t idO = idesc_bf16(128, D, 1);
+  constexpr uint32_t hi = desc_hi_sw128(1024);
+  const uint32_t vlo = desc_lo(sV, C::BOX_BYTES);
 #pragma unroll
-  for (int kk = 0; kk < 8; ++kk) {
-    mma_ts(tmem_d, tmem_p + kk * 8, smem_desc_sw128(sV + kk * 2048, C::BOX_BYTES, 1024), idO,
-           (accumulate || kk > 0) ? 1u : 0u);
-  }
+  for (int kk = 0; kk < 8; ++kk)
+    mma_ts_w(tmem_d, tmem_p + kk * 8, vlo + kk * (2048 >> 4), hi, idO,
+             (accumulate || kk > 0) ? 1u : 0u);
 }
 
 template <int D, bool QK8>
