@@ -587,6 +587,10 @@ def measure_layer(ug, args, wl, world, local, rank, heads_range=None, with_e2e=F
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local)
+    # the attention kernel's own clock record (SM cycles over nanoseconds of its first CTA),
+    # for the timed launches only
+    plan.set_clock_record(True)
+    plan.read_clock()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -598,6 +602,12 @@ def measure_layer(ug, args, wl, world, local, rank, heads_range=None, with_e2e=F
     end.record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop()
+    kclock = plan.read_clock()
+    plan.set_clock_record(False)
+    clocks["kernel_sm_mhz"] = kclock["sm_mhz"]
+    clocks["kernel_clock_note"] = ("hla_forward's own record: SM cycles (clock64) over nanoseconds "
+                                   "(globaltimer) of its first CTA, summed over the %d timed launches"
+                                   % kclock["launches"])
     if world > 1:
         dist.barrier()
     if plan.sync_status() != 0:
@@ -696,6 +706,7 @@ def measure_layer(ug, args, wl, world, local, rank, heads_range=None, with_e2e=F
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": burst, "unit": "TFLOP/s",
                      "frac": attn_tflops / burst, "frac_sustained": attn_tflops / sust,
                      "peak_sustained": sust, "traffic": traffic, "peak_source": peak_note,
+                     "kernel_sm_mhz": kclock["sm_mhz"],
                      "algorithmic_flops_per_launch": flops_rank},
         "e2e": e2e, "gpu_launches": launches, "clocks": clocks, "cpu_baseline": cpu,
     }

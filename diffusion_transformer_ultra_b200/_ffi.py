@@ -36,6 +36,7 @@ SYMBOLS = (
     "ultragen_host_runner_forward", "ultragen_host_runner_last_launch_count",
     "ultragen_host_runner_destroy", "ultragen_plan_set_halo", "ultragen_plan_export_kv",
     "ultragen_plan_set_qk_format", "ultragen_plan_set_lr_order",
+    "ultragen_plan_set_clock_record", "ultragen_plan_read_clock",
 )
 
 
@@ -92,6 +93,8 @@ def lib() -> ctypes.CDLL:
     L.ultragen_plan_export_kv.argtypes = [vp, vp]
     L.ultragen_plan_set_qk_format.argtypes = [vp, cint, cint, cint]
     L.ultragen_plan_set_lr_order.argtypes = [vp, cint]
+    L.ultragen_plan_set_clock_record.argtypes = [vp, cint]
+    L.ultragen_plan_read_clock.argtypes = [vp, vp]
     L.ultragen_plan_info.argtypes = [vp, ctypes.POINTER(PlanInfo)]
     L.ultragen_plan_export.argtypes = [vp, vp, vp, vp]
     L.ultragen_plan_export_rowmasks.argtypes = [vp, cint, vp]
@@ -201,6 +204,19 @@ class Plan:
     def set_diagnostics(self, fault: int = 0, wait_limit_s: float = 2.0):
         _check("ultragen_plan_set_diagnostics",
                lib().ultragen_plan_set_diagnostics(self._h, int(fault), float(wait_limit_s)))
+
+    def set_clock_record(self, on: bool = True):
+        _check("ultragen_plan_set_clock_record",
+               lib().ultragen_plan_set_clock_record(self._h, 1 if on else 0))
+
+    def read_clock(self) -> dict:
+        """The attention launches' clock record since the last read: launches, SM cycles and
+        nanoseconds of the first CTA summed, and their ratio in MHz (then cleared)."""
+        out = (ctypes.c_uint64 * 3)()
+        _check("ultragen_plan_read_clock", lib().ultragen_plan_read_clock(self._h, out))
+        n, cyc, ns = int(out[0]), int(out[1]), int(out[2])
+        return {"launches": n, "cycles": cyc, "ns": ns,
+                "sm_mhz": (1e3 * cyc / ns) if ns else None}
 
     def sync_status(self, stream=None) -> int:
         return lib().ultragen_sync_status(self._h, _stream_ptr(stream))

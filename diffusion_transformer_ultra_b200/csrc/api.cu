@@ -33,7 +33,7 @@ void free_device(ultragen_plan_t* p) {
   DeviceTables& d = p->dev;
   void* ptrs[] = {d.items, d.entries, d.mask_off, d.mask_pool, d.perm, d.inv_perm,
                   d.slot_pos, d.halo_ptr, d.halo_dst, d.halo_pad, d.item_order, d.rope,
-                  d.combine, d.error, d.ws};
+                  d.combine, d.error, d.clock, d.ws};
   for (void* q : ptrs)
     if (q) cudaFree(q);
   d = DeviceTables();
@@ -81,7 +81,8 @@ int ensure_device(ultragen_plan_t* p) {
       (st = upload(&d.halo_dst, p->halo_dst)) || (st = upload(&d.halo_pad, p->halo_pad)) ||
       (st = upload(&d.item_order, p->item_order)) ||
       (st = upload(&d.rope, rope)) ||
-      (st = upload(&d.combine, comb)) || (st = upload(&d.error, std::vector<int>(1, 0)))) {
+      (st = upload(&d.combine, comb)) || (st = upload(&d.error, std::vector<int>(1, 0))) ||
+      (st = upload(&d.clock, std::vector<unsigned long long>(5, 0ull)))) {
     free_device(p);
     return st;
   }
@@ -275,6 +276,7 @@ int launch_attention(const ultragen_plan_t* p, const void* qp, const void* kp, c
   f.heads = heads;
   f.n_entries = (int)p->entries.size();
   f.n_mask_words = (int)p->mask_pool.size();
+  f.clock = p->clock_record ? p->dev.clock : nullptr;
   const int grid = (int)std::min<int64_t>(items, sm_count());
   // few items per CTA: hand them out item-major, longest first, so that the last round holds
   // the short ones; otherwise head-major keeps one head's shared key tiles (its LR segment)
@@ -520,6 +522,24 @@ int ultragen_warm_start(const float* x_lr, const float* noise, float* x_hr, int 
     return cuda_status(launch_warm_start_fused(a, f, s));
   }
   return cuda_status(launch_warm_start(a, s));
+}
+
+int ultragen_plan_set_clock_record(ultragen_plan_t* p, int on) {
+  if (!p || on < 0 || on > 1) return ULTRAGEN_ERR_INVALID_ARG;
+  p->clock_record = on;
+  return ULTRAGEN_OK;
+}
+
+int ultragen_plan_read_clock(const ultragen_plan_t* p, uint64_t out[3]) {
+  if (!p || !out) return ULTRAGEN_ERR_INVALID_ARG;
+  out[0] = out[1] = out[2] = 0;
+  if (!p->dev.valid || !p->dev.clock) return ULTRAGEN_OK;
+  unsigned long long h[3];   // words 3, 4 are the running launch's start (scratch)
+  if (cudaMemcpy(h, p->dev.clock, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess ||
+      cudaMemset(p->dev.clock, 0, sizeof(h)) != cudaSuccess)
+    return cuda_status(cudaGetLastError());
+  for (int i = 0; i < 3; ++i) out[i] = h[i];
+  return ULTRAGEN_OK;
 }
 
 int ultragen_plan_set_diagnostics(ultragen_plan_t* p, int fault, double wait_limit_s) {

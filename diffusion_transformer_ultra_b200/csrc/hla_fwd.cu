@@ -302,6 +302,12 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t tbase,
       ++st;
     }
   }
+  if (p.clock != nullptr && blockIdx.x == 0) {
+    volatile unsigned long long* start = p.clock + 3;   // written by thread 0 at entry
+    atomicAdd(p.clock, 1ull);
+    atomicAdd(p.clock + 1, (unsigned long long)clock64() - start[0]);
+    atomicAdd(p.clock + 2, globaltimer_ns() - start[1]);
+  }
   if (!ok) {
     // Abort: let the products already issued finish before TMEM is released.
     mma_commit(bar + 8 * C::B_DRAIN);
@@ -548,8 +554,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // launch clock record: the first CTA lives for the whole persistent launch (the start values
+  // wait in shared memory, not in registers the softmax roles need)
 
   if (threadIdx.x == 0) {
+    // launch clock record: the first CTA lives for the whole persistent launch; its start goes
+    // to the record's scratch words, its end is taken when its MMA warp has issued its last
+    // product (the last item's epilogue, a few thousand cycles of millions, is left out)
+    if (p.clock != nullptr && blockIdx.x == 0) {
+      p.clock[3] = (unsigned long long)clock64();
+      p.clock[4] = globaltimer_ns();
+    }
     mbar_init(bar + 8 * C::B_QF, 1);
     mbar_init(bar + 8 * C::B_QE, 1);
     for (int s = 0; s < C::NS; ++s) {

@@ -99,6 +99,9 @@ struct FwdParams {
   int N_raster = 0, heads = 1;
   int n_entries = 0;               // table sizes for the index checks of debug builds
   int n_mask_words = 0;
+  // launch clock record: CTA 0 adds 1, its cycles and its nanoseconds to words 0-2, keeping
+  // its start in words 3-4 (null: not recorded)
+  unsigned long long* clock = nullptr;
 };
 
 // Device error codes shared by the kernels and the host (ultragen_sync_status): the bounded

@@ -45,6 +45,7 @@ struct DeviceTables {
   float* rope = nullptr;           // [max(H,W)][head_dim/2][2] (cos, sin)
   int32_t* combine = nullptr;      // CombineGroup[]
   int* error = nullptr;            // device error word
+  unsigned long long* clock = nullptr;   // launch clock record: launches, cycles, ns; 2 scratch
   float* ws = nullptr;             // split partials
   size_t ws_bytes = 0;
 };
@@ -82,6 +83,8 @@ struct ultragen_plan {
   // diagnostics: device wait limit and injected fault (ultragen_plan_set_diagnostics)
   unsigned long long wait_limit_ns = 2000ull * 1000 * 1000;
   int fault = 0;
+  // launch clock record (ultragen_plan_set_clock_record)
+  int clock_record = 0;
 
   // host tables
   std::vector<int32_t> perm;       // K/V slot -> raster (-1 pad), N_kv long; Q slots are its

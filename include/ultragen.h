@@ -289,6 +289,21 @@ int ultragen_sync_status(const ultragen_plan_t* plan, ultragen_stream_t stream);
  * fault = 0 is normal operation.  INVALID_ARG outside these ranges. */
 int ultragen_plan_set_diagnostics(ultragen_plan_t* plan, int fault, double wait_limit_s);
 
+/* Launch clock record (no counterpart in the pages; measurement support).  With on = 1, every
+ * attention launch of this plan adds, from its first CTA (which lives for the whole persistent
+ * launch), the SM cycles (clock64) and the nanoseconds (globaltimer) from that CTA's start to
+ * the issue of its last tensor-core product (the last item's epilogue, a few thousand cycles of
+ * millions, is left out) to a small device record that the plan owns; on = 0 stops recording.
+ * Cycles over nanoseconds is the SM clock the kernel actually ran at, which under a power cap
+ * can be well below what a driver query reports.  The record is uploaded with the plan's tables
+ * (any device call).  INVALID_ARG for a null plan or on not 0/1. */
+int ultragen_plan_set_clock_record(ultragen_plan_t* plan, int on);
+
+/* Copies the record to out[3] = {launches, cycles, nanoseconds} summed since the last read,
+ * then clears it.  Host, synchronous (cudaMemcpy: it waits for the device); call it after the
+ * launches of interest completed.  All zeros when the plan has no tables on the device yet. */
+int ultragen_plan_read_clock(const ultragen_plan_t* plan, uint64_t out[3]);
+
 /* Kernel launches the last device call of this plan issued (for launch accounting). */
 int ultragen_last_launch_count(const ultragen_plan_t* plan);
 

@@ -43,6 +43,20 @@ def test_status_strings(ffi):
     assert L.ultragen_status_string(99).decode() == "unknown status"
 
 
+def test_clock_record_arguments(ffi):
+    import ctypes as C
+    L = ffi.lib()
+    buf = (C.c_uint64 * 3)(7, 7, 7)
+    assert L.ultragen_plan_set_clock_record(None, 1) == 1
+    assert L.ultragen_plan_read_clock(None, buf) == 1
+    p = ffi.Plan(32, 32, 8, 2, 4, 16, 1, 64)
+    assert L.ultragen_plan_set_clock_record(p.handle, 2) == 1
+    assert L.ultragen_plan_read_clock(p.handle, None) == 1
+    p.set_clock_record(True)
+    # no tables on a device yet: an empty record
+    assert p.read_clock() == {"launches": 0, "cycles": 0, "ns": 0, "sm_mhz": None}
+
+
 def test_debug_build_compiles_and_exports_every_symbol(ffi):
     """The ULTRAGEN_DEBUG build (index checks in the kernels) builds in-tree and exports the
     same C ABI; nothing here calls into a GPU."""

@@ -43,3 +43,27 @@ def test_withheld_signal_times_out_and_context_survives(ug, qk):
     assert fresh.sync_status() == 0
     torch.cuda.synchronize()
     assert torch.equal(lay.op.view(torch.int16), lay2.op.view(torch.int16))
+
+
+def test_launch_clock_record(ug):
+    """The launch clock record counts the attention launches and gives the SM clock they ran
+    at (cycles of the first CTA over its nanoseconds), then clears."""
+    import torch
+    wl = ug.WORKLOADS["1k"]
+    q, k, v = (t.cuda() for t in ug.make_qkv(wl))
+    plan = ug.plan_for(wl)
+    lay = ug.Layer(plan, wl.batch)
+    ug.permute_rope(q, k, v, lay.qp, lay.kp, lay.vp, plan)
+    plan.set_clock_record(True)
+    for _ in range(3):
+        ug.hla_forward(lay.qp, lay.kp, lay.vp, lay.op, plan)
+    assert plan.sync_status() == 0
+    rec = plan.read_clock()
+    assert rec["launches"] == 3
+    assert 300.0 < rec["sm_mhz"] < 2500.0, rec
+    assert plan.read_clock()["launches"] == 0
+    plan.set_clock_record(False)
+    ug.hla_forward(lay.qp, lay.kp, lay.vp, lay.op, plan)
+    assert plan.sync_status() == 0
+    assert plan.read_clock()["launches"] == 0
+    torch.cuda.synchronize()
