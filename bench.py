@@ -51,8 +51,9 @@ def parse():
                     help="HR->LR scope: -1 all LR tokens (default); r >= 0 the window's anchors grown by r")
     ap.add_argument("--lr-order", type=int, default=-1, choices=[-1, 0, 1],
                     help="LR segment order with an LR-region scope: -1 automatic (default), 0 raster, 1 8x16 blocks")
-    ap.add_argument("--halo", type=int, default=-1, choices=[-1, 0, 1],
-                    help="compact halo blocks in the K/V layout: -1 automatic (default), 0 off, 1 on")
+    ap.add_argument("--halo", type=int, default=-1, choices=[-1, 0, 1, 2],
+                    help="compact halo blocks in the K/V layout: -1 automatic (default), 0 off, "
+                         "1 copied by the permute, 2 gathered by the attention")
     ap.add_argument("--qk", default="bf16", choices=["bf16", "e4m3"],
                     help="storage of the permuted Q and K: bf16 (default) or scaled e4m3 with 8-bit Q K^T")
     ap.add_argument("--q-exp", type=int, default=0, help="e4m3 Q stores x * 2^-q_exp")
@@ -628,11 +629,12 @@ def measure_layer(ug, args, wl, world, local, rank, heads_range=None, with_e2e=F
     pk, src = peaks()
     attn_tflops = flops_rank / (ms_attn * 1e-3) / 1e12
     elem = wlr.batch * wlr.heads * info["N_tot"] * wlr.D
-    kv_elem = wlr.batch * wlr.heads * info["N_kv"] * wlr.D
+    kv_elem = wlr.batch * wlr.heads * info["kv_rows"] * wlr.D
     in_size = 2 if wl.dtype == "bf16" else 4
     qk_size = 1 if e4m3 else 2
-    # permute_rope: every raster row of Q, K, V read once (halo copies are written from the
-    # same read), Q written over N_tot slots and K, V over N_kv slots (pad slots as zeros)
+    # permute_rope: every raster row of Q, K, V read once (copied halo blocks are written from
+    # the same read), Q written over N_tot slots and K, V over kv_rows slots (pad slots as
+    # zeros); gathered halo blocks cost the permute nothing
     perm_bytes = (3 * wlr.batch * info["N_raster"] * wlr.heads * wlr.D * in_size
                   + (elem + kv_elem) * qk_size + kv_elem * 2)
     perm_bytes_method = 6 * wlr.batch * info["N_raster"] * wlr.heads * wlr.D * in_size
@@ -686,7 +688,8 @@ def measure_layer(ug, args, wl, world, local, rank, heads_range=None, with_e2e=F
                    "lr_radius": args.lr_radius, "heads": full_heads, "head_dim": wl.D,
                    "batch": wl.batch, "N_tot": info["N_tot"],
                    "useful_pairs_per_head": info["useful_pairs"],
-                   "halo_blocks": bool(info["halo_copy"]), "N_kv": info["N_kv"],
+                   "halo_blocks": ["none", "copied", "gathered"][info["halo_copy"]],
+                   "N_kv": info["N_kv"], "kv_rows": info["kv_rows"],
                    "lr_blocks": bool(info["lr_block"]), "qk_format": args.qk,
                    **({"q_exp": args.q_exp, "k_exp": args.k_exp} if e4m3 else {}),
                    "inputs_sha256": sha,

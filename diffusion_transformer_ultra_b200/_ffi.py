@@ -37,6 +37,7 @@ SYMBOLS = (
     "ultragen_host_runner_destroy", "ultragen_plan_set_halo", "ultragen_plan_export_kv",
     "ultragen_plan_set_qk_format", "ultragen_plan_set_lr_order",
     "ultragen_plan_set_clock_record", "ultragen_plan_read_clock",
+    "ultragen_plan_export_halo_ops",
 )
 
 
@@ -55,7 +56,8 @@ class PlanInfo(ctypes.Structure):
         ("lr_radius", ctypes.c_int32), ("halo_copy", ctypes.c_int32),
         ("halo_slots_per_window", ctypes.c_int32), ("N_kv", ctypes.c_int64),
         ("off_halo", ctypes.c_int64), ("qk_format", ctypes.c_int32), ("q_exp", ctypes.c_int32),
-        ("k_exp", ctypes.c_int32), ("lr_block", ctypes.c_int32),
+        ("k_exp", ctypes.c_int32), ("lr_block", ctypes.c_int32), ("kv_rows", ctypes.c_int64),
+        ("n_halo_ops", ctypes.c_int32),
     ]
 
     def as_dict(self):
@@ -91,6 +93,7 @@ def lib() -> ctypes.CDLL:
     L.ultragen_plan_set_lr_scope.argtypes = [vp, cint]
     L.ultragen_plan_set_halo.argtypes = [vp, cint]
     L.ultragen_plan_export_kv.argtypes = [vp, vp]
+    L.ultragen_plan_export_halo_ops.argtypes = [vp, vp]
     L.ultragen_plan_set_qk_format.argtypes = [vp, cint, cint, cint]
     L.ultragen_plan_set_lr_order.argtypes = [vp, cint]
     L.ultragen_plan_set_clock_record.argtypes = [vp, cint]
@@ -186,6 +189,12 @@ class Plan:
         _check("ultragen_plan_export_kv", lib().ultragen_plan_export_kv(self._h, kv.ctypes.data))
         return kv
 
+    def export_halo_ops(self):
+        ops = np.zeros(max(1, self.info["n_halo_ops"]), np.int32)
+        _check("ultragen_plan_export_halo_ops",
+               lib().ultragen_plan_export_halo_ops(self._h, ops.ctypes.data))
+        return ops[:self.info["n_halo_ops"]]
+
     def export(self):
         i = self.info
         perm = np.empty(i["N_tot"], np.int32)
@@ -262,7 +271,7 @@ def permute_rope(q, k, v, qp, kp, vp, plan: Plan, stream=None):
     B = q.shape[0]
     raster = (B, i["N_raster"], i["heads"], i["head_dim"])
     q_shape = (B, i["heads"], i["N_tot"], i["head_dim"])
-    kv_shape = (B, i["heads"], i["N_kv"], i["head_dim"])
+    kv_shape = (B, i["heads"], i["kv_rows"], i["head_dim"])
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, raster, (torch.bfloat16, torch.float32), n)
     if not (q.dtype == k.dtype == v.dtype):
@@ -282,7 +291,7 @@ def hla_forward(qp, kp, vp, op, plan: Plan, stream=None):
     i = plan.info
     B = qp.shape[0]
     shape = (B, i["heads"], i["N_tot"], i["head_dim"])
-    kv_shape = (B, i["heads"], i["N_kv"], i["head_dim"])
+    kv_shape = (B, i["heads"], i["kv_rows"], i["head_dim"])
     _need(qp, shape, plan.qk_dtypes(), "qp")
     _need(op, shape, (torch.bfloat16,), "op")
     _need(kp, kv_shape, plan.qk_dtypes(), "kp")
@@ -298,8 +307,8 @@ def hla_forward_raster(qp, kp, vp, o, plan: Plan, stream=None):
     i = plan.info
     B = qp.shape[0]
     _need(qp, (B, i["heads"], i["N_tot"], i["head_dim"]), plan.qk_dtypes(), "qp")
-    _need(kp, (B, i["heads"], i["N_kv"], i["head_dim"]), plan.qk_dtypes(), "kp")
-    _need(vp, (B, i["heads"], i["N_kv"], i["head_dim"]), (torch.bfloat16,), "vp")
+    _need(kp, (B, i["heads"], i["kv_rows"], i["head_dim"]), plan.qk_dtypes(), "kp")
+    _need(vp, (B, i["heads"], i["kv_rows"], i["head_dim"]), (torch.bfloat16,), "vp")
     _need(o, (B, i["N_raster"], i["heads"], i["head_dim"]), (torch.bfloat16,), "o")
     _check("ultragen_hla_forward_raster", lib().ultragen_hla_forward_raster(
         qp.data_ptr(), kp.data_ptr(), vp.data_ptr(), o.data_ptr(), plan.handle, B,
@@ -314,7 +323,7 @@ def hla_forward_noalloc(qp, kp, vp, op, plan: Plan, stream=None):
     i = plan.info
     B = qp.shape[0]
     shape = (B, i["heads"], i["N_tot"], i["head_dim"])
-    kv_shape = (B, i["heads"], i["N_kv"], i["head_dim"])
+    kv_shape = (B, i["heads"], i["kv_rows"], i["head_dim"])
     _need(qp, shape, plan.qk_dtypes(), "qp")
     _need(op, shape, (torch.bfloat16,), "op")
     _need(kp, kv_shape, plan.qk_dtypes(), "kp")
@@ -405,7 +414,7 @@ class Layer:
         i = plan.info
         self.plan = plan
         shape = (batch, i["heads"], i["N_tot"], i["head_dim"])
-        kv_shape = (batch, i["heads"], i["N_kv"], i["head_dim"])
+        kv_shape = (batch, i["heads"], i["kv_rows"], i["head_dim"])
         qk = plan.qk_dtypes()[0]
         self.qp = torch.empty(shape, dtype=qk, device=device)
         self.op = torch.empty(shape, dtype=torch.bfloat16, device=device)

@@ -32,7 +32,7 @@ int upload(T** dst, const std::vector<T>& src) {
 void free_device(ultragen_plan_t* p) {
   DeviceTables& d = p->dev;
   void* ptrs[] = {d.items, d.entries, d.mask_off, d.mask_pool, d.perm, d.inv_perm,
-                  d.slot_pos, d.halo_ptr, d.halo_dst, d.halo_pad, d.item_order, d.rope,
+                  d.slot_pos, d.halo_ptr, d.halo_dst, d.halo_pad, d.halo_ops, d.item_order, d.rope,
                   d.combine, d.error, d.clock, d.ws};
   for (void* q : ptrs)
     if (q) cudaFree(q);
@@ -79,7 +79,7 @@ int ensure_device(ultragen_plan_t* p) {
       (st = upload(&d.perm, p->perm)) || (st = upload(&d.inv_perm, p->inv_perm)) ||
       (st = upload(&d.slot_pos, p->slot_pos)) || (st = upload(&d.halo_ptr, p->halo_ptr)) ||
       (st = upload(&d.halo_dst, p->halo_dst)) || (st = upload(&d.halo_pad, p->halo_pad)) ||
-      (st = upload(&d.item_order, p->item_order)) ||
+      (st = upload(&d.halo_ops, p->halo_ops)) || (st = upload(&d.item_order, p->item_order)) ||
       (st = upload(&d.rope, rope)) ||
       (st = upload(&d.combine, comb)) || (st = upload(&d.error, std::vector<int>(1, 0))) ||
       (st = upload(&d.clock, std::vector<unsigned long long>(5, 0ull)))) {
@@ -216,6 +216,27 @@ int make_tmap_u8(CUtensorMap* m, const void* base, uint64_t rows, int D) {
   return r == CUDA_SUCCESS ? ULTRAGEN_OK : ULTRAGEN_ERR_CUDA;
 }
 
+// The window segment of permuted K or V as a 5D view (element, column and row in the window,
+// window, batch-head) with [inner x nc x nr] boxes and the 128-byte swizzle: one box is one
+// piece of a halo block (nr x nc tokens of one window, raster order), landing as nr * nc
+// consecutive 128-byte rows.  inner = 64 bf16 elements, or 128 bytes of e4m3 (bytes = 1).
+int make_tmap_window(CUtensorMap* m, const void* kv, const ultragen_plan_t* p, uint64_t units,
+                     int nc, int nr, int bytes) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return ULTRAGEN_ERR_CUDA;
+  const uint64_t es = bytes ? 1 : 2, row = (uint64_t)p->D * es, l = (uint64_t)p->l;
+  const cuuint64_t dims[5] = {(cuuint64_t)p->D, l, l, (cuuint64_t)p->nWh * p->nWw, units};
+  const cuuint64_t strides[4] = {row, l * row, l * l * row, (cuuint64_t)p->kv_rows * row};
+  const cuuint32_t box[5] = {bytes ? 128u : 64u, (cuuint32_t)nc, (cuuint32_t)nr, 1, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  const void* base = static_cast<const uint8_t*>(kv) + (uint64_t)p->off_hr * row;
+  CUresult r = fn(m, bytes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ULTRAGEN_OK : ULTRAGEN_ERR_CUDA;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int sm_count() {
@@ -237,7 +258,7 @@ size_t split_workspace_bytes(const ultragen_plan_t* p, int64_t units) {
 int launch_attention(const ultragen_plan_t* p, const void* qp, const void* kp, const void* vp,
                      void* op, int units, int heads, int raster, float* ws, cudaStream_t s,
                      int* launches) {
-  const int64_t rows = (int64_t)units * p->N_tot, kv_rows = (int64_t)units * p->N_kv;
+  const int64_t rows = (int64_t)units * p->N_tot, kv_rows = (int64_t)units * p->kv_rows;
   const int64_t items = (int64_t)units * (int64_t)p->items.size();
   alignas(64) CUtensorMap tq, tk, tv;
   const int qk8 = p->qk_format == ULTRAGEN_QK_E4M3;
@@ -250,6 +271,17 @@ int launch_attention(const ultragen_plan_t* p, const void* qp, const void* kp, c
     return st;
   }
   if ((st = make_tmap(&tv, vp, kv_rows, p->D))) return st;
+  // gathered halo tiles: K and V window views with the three piece boxes (b x l, l x b, b x b)
+  HaloMaps hm;
+  std::memset(&hm, 0, sizeof(hm));
+  const int gather = p->halo_copy == 2;
+  if (gather) {
+    const int shp[3][2] = {{p->l, p->b}, {p->b, p->l}, {p->b, p->b}};   // (nc, nr)
+    for (int s = 0; s < 3; ++s)
+      if ((st = make_tmap_window(&hm.m[s], kp, p, units, shp[s][0], shp[s][1], qk8)) ||
+          (st = make_tmap_window(&hm.m[3 + s], vp, p, units, shp[s][0], shp[s][1], 0)))
+        return st;
+  }
   FwdParams f;
   f.items = p->dev.items;
   f.entries = p->dev.entries;
@@ -262,7 +294,16 @@ int launch_attention(const ultragen_plan_t* p, const void* qp, const void* kp, c
   f.n_items_head = (int)p->items.size();
   f.total_items = (int)items;
   f.N_tot = (int)p->N_tot;
-  f.N_kv = (int)p->N_kv;
+  f.N_kv = (int)p->kv_rows;
+  f.n_ktiles = (int)(p->N_kv / kTile);
+  if (gather) {
+    f.halo_ops = p->dev.halo_ops;
+    f.halo_tile0 = (int)(p->off_halo / kTile);
+    f.halo_gtiles = (int)(p->G / kTile);
+    f.nWh = p->nWh;
+    f.nWw = p->nWw;
+    f.n_halo_ops = (int)p->halo_ops.size();
+  }
   f.off_hr = (int)p->off_hr;
   f.l2 = p->l * p->l;
   f.n_ws_head = p->n_split_items;
@@ -286,7 +327,7 @@ int launch_attention(const ultragen_plan_t* p, const void* qp, const void* kp, c
   f.item_order = p->dev.item_order;
   *launches = 0;
   if (grid > 0) {
-    st = cuda_status(launch_hla_fwd(&tq, &tk, &tv, f, p->D, qk8, grid, s));
+    st = cuda_status(launch_hla_fwd(&tq, &tk, &tv, &hm, f, p->D, qk8, grid, s));
     if (st) return st;
     ++*launches;
   }
@@ -332,10 +373,10 @@ int launch_permute(const ultragen_plan_t* p, const void* q, const void* k, const
   a.n_halo_dst = (int)p->halo_dst.size();
   // rows: every Q slot, then the pad slots of the halo blocks (their token slots are written
   // with their source rows)
-  const int64_t n_pad = p->halo_copy ? (int64_t)p->halo_pad.size() : 0;
+  const int64_t n_pad = p->halo_copy == 1 ? (int64_t)p->halo_pad.size() : 0;
   a.rows_total = (int64_t)batch * heads * (p->N_tot + n_pad);
   a.N_tot = (int)p->N_tot;
-  a.N_kv = (int)p->N_kv;
+  a.N_kv = (int)p->kv_rows;
   a.halo_pad = p->dev.halo_pad;
   a.div_rows = FastDiv((uint32_t)(p->N_tot + n_pad));
   a.N_raster = (int)p->N_raster;
@@ -343,7 +384,7 @@ int launch_permute(const ultragen_plan_t* p, const void* q, const void* k, const
   a.div_heads = FastDiv((uint32_t)heads);
   a.pair_a0 = p->axes[0] / 2;
   a.pair_a01 = (p->axes[0] + p->axes[1]) / 2;
-  a.halo_ptr = p->halo_copy ? p->dev.halo_ptr : nullptr;
+  a.halo_ptr = p->halo_copy == 1 ? p->dev.halo_ptr : nullptr;
   a.halo_dst = p->dev.halo_dst;
   a.off_hr = (int)p->off_hr;
   a.N_hrp = (int)p->N_hrp;
@@ -374,7 +415,7 @@ int ultragen_permute_rope(const void* q, const void* k, const void* v, int in_dt
   const void* ptrs[] = {q, k, v, qp, kp, vp};
   for (const void* x : ptrs)
     if (!aligned16(x)) return ULTRAGEN_ERR_INVALID_ARG;
-  if ((int64_t)batch * p->heads * p->N_kv >= ((int64_t)1 << 31) ||
+  if ((int64_t)batch * p->heads * p->kv_rows >= ((int64_t)1 << 31) ||
       (int64_t)batch * p->heads * p->N_raster >= ((int64_t)1 << 31))
     return ULTRAGEN_ERR_UNSUPPORTED;
   int st = ensure_device(p);
@@ -393,7 +434,7 @@ static int hla_forward_impl(const void* qp, const void* kp, const void* vp, void
   const void* ptrs[] = {qp, kp, vp, op};
   for (const void* x : ptrs)
     if (!aligned16(x)) return ULTRAGEN_ERR_INVALID_ARG;
-  const int64_t rows = (int64_t)batch * p->heads * p->N_kv;
+  const int64_t rows = (int64_t)batch * p->heads * p->kv_rows;
   const int64_t items = (int64_t)batch * p->heads * (int64_t)p->items.size();
   if (rows >= ((int64_t)1 << 31) || items >= ((int64_t)1 << 31)) return ULTRAGEN_ERR_UNSUPPORTED;
   int st = ensure_device(p);

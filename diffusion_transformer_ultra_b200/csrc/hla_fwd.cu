@@ -143,8 +143,8 @@ __device__ __forceinline__ const int32_t* item_at(const FwdParams& p, int it, in
 // ------------------------------------------------------------------------ producer warp
 template <int D, bool QK8>
 __device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
-                              const CUtensorMap* tmV, const FwdParams& p, uint32_t sbase,
-                              volatile int* abort_flag) {
+                              const CUtensorMap* tmV, const HaloMaps* hm, const FwdParams& p,
+                              uint32_t sbase, volatile int* abort_flag) {
   using C = FwdCfg<D>;
   constexpr int QK_BYTES = QK8 ? 128 * D : C::TILE_BYTES;   // one Q or K tile
   const uint32_t sQ = sbase + C::Q_OFF, sKV = sbase + C::KV_OFF, bar = sbase + C::BAR_OFF;
@@ -158,6 +158,42 @@ __device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
 #pragma unroll
       for (int bx = 0; bx < C::BOXES; ++bx) tma_load_2d(dst + bx * C::BOX_BYTES, tm, bx * 64, y, b);
     }
+  };
+  // key (isv = 0) or value (1) tile kt of (batch, head) bh: a window-first tile, or a tile of a
+  // window's halo block assembled from its neighbours' window-first slots, one box per piece
+  // (b x l, l x b or b x b tokens of one window, raster order) and zero-filled boxes for the
+  // gaps.  Every box lands at a multiple of 8 rows (1 KB) of the 128-byte-swizzled slot, so
+  // the tile reads exactly as if its 128 rows had been copied there.
+  auto load_kv = [&](bool isv, uint32_t dst, int kt, int bh, uint32_t b) {
+    if (p.halo_ops == nullptr || kt < p.halo_tile0) {
+      load_tile(isv ? tmV : tmK, !isv && QK8, dst, bh * p.N_kv + kt * 128, b);
+      return true;
+    }
+    const int v = kt - p.halo_tile0;
+    const int w = v / p.halo_gtiles, tb = v - w * p.halo_gtiles;
+    const int wr = w / p.nWw, wc = w - wr * p.nWw;
+    const int o0 = __ldg(p.halo_ops + tb), o1 = __ldg(p.halo_ops + tb + 1);
+    if (!UG_CHECK(o0 > p.halo_gtiles && o0 <= o1 && o1 <= p.n_halo_ops)) return false;
+    for (int o = o0; o < o1; ++o) {
+      const uint32_t c = (uint32_t)__ldg(p.halo_ops + o);
+      const int row = c & 127, shape = (c >> 7) & 3;
+      const int sr = wr + (int)((c >> 10) & 3) - 1, sc = wc + (int)((c >> 12) & 3) - 1;
+      const int i0 = (c >> 14) & 255, j0 = (c >> 22) & 255;
+      if (!UG_CHECK(shape <= 2 && row % 8 == 0)) return false;
+      // a zero box, or a piece of a window outside the image, reads window -1: out of bounds
+      // as a whole, it lands as zeros
+      const bool zero = ((c >> 9) & 1) || sr < 0 || sr >= p.nWh || sc < 0 || sc >= p.nWw;
+      const int win = zero ? -1 : sr * p.nWw + sc;
+      const CUtensorMap* tm = &hm->m[(isv ? 3 : 0) + shape];
+      if (!isv && QK8) {
+        tma_load_5d(dst + row * 128, tm, 0, j0, i0, win, bh, b);
+      } else {
+#pragma unroll
+        for (int bx = 0; bx < C::BOXES; ++bx)
+          tma_load_5d(dst + bx * C::BOX_BYTES + row * 128, tm, bx * 64, j0, i0, win, bh, b);
+      }
+    }
+    return true;
   };
   for (int it = blockIdx.x; it < p.total_items && ok; it += gridDim.x) {
     int bh;
@@ -189,19 +225,22 @@ __device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
         break;
       }
       const uint32_t fb = bar + 8 * (C::B_KVF + g);
-      if (!UG_CHECK((j == 0 || ((__ldg(p.entries + e0 + j - 1) & 0x7fffffff) + 1) * 128 <= p.N_kv) &&
-                    (j == n || ((__ldg(p.entries + e0 + j) & 0x7fffffff) + 1) * 128 <= p.N_kv))) {
+      const int kv = j > 0 ? (__ldg(p.entries + e0 + j - 1) & 0x7fffffff) : 0;
+      const int kk = j < n ? (__ldg(p.entries + e0 + j) & 0x7fffffff) : 0;
+      if (!UG_CHECK(kv < p.n_ktiles && kk < p.n_ktiles)) {
         ok = false;
         break;
       }
       mbar_expect_tx(fb, (j > 0 ? C::TILE_BYTES : 0) + (j < n ? QK_BYTES : 0));
-      if (j > 0)
-        load_tile(tmV, false, sKV + C::v_slot(g) * C::TILE_BYTES,
-                  bh * p.N_kv + (__ldg(p.entries + e0 + j - 1) & 0x7fffffff) * 128, fb);
-      if (j < n)
-        load_tile(tmK, QK8, sKV + C::k_slot(g) * C::TILE_BYTES,
-                  bh * p.N_kv + (__ldg(p.entries + e0 + j) & 0x7fffffff) * 128, fb);
       ++st;
+      if (j > 0 && !load_kv(true, sKV + C::v_slot(g) * C::TILE_BYTES, kv, bh, fb)) {
+        ok = false;
+        break;
+      }
+      if (j < n && !load_kv(false, sKV + C::k_slot(g) * C::TILE_BYTES, kk, bh, fb)) {
+        ok = false;
+        break;
+      }
     }
   }
   if (!ok) {
@@ -544,7 +583,8 @@ __device__ void softmax_role(const FwdParams& p, uint32_t sbase, uint32_t tbase,
 template <int D, bool QK8>
 __global__ void __launch_bounds__(kThreads, 1)
     hla_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ HaloMaps hm,
+                   const FwdParams p) {
   using C = FwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -597,7 +637,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp >= 8) {
     regs_shrink<kRegsControl>();
     if (warp == kWarpProducer) {
-      if (lane == 0) producer_role<D, QK8>(&tmQ, &tmK, &tmV, p, sbase, abort_flag);
+      if (lane == 0) producer_role<D, QK8>(&tmQ, &tmK, &tmV, &hm, p, sbase, abort_flag);
     } else if (warp == kWarpMma) {
       if (lane == 0) mma_role<D, QK8>(p, sbase, tbase, abort_flag);
     }
@@ -616,8 +656,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int D, bool QK8>
-static cudaError_t launch_d(const void* tmQ, const void* tmK, const void* tmV, const FwdParams& p,
-                            int grid, cudaStream_t st) {
+static cudaError_t launch_d(const void* tmQ, const void* tmK, const void* tmV,
+                            const HaloMaps* hm, const FwdParams& p, int grid, cudaStream_t st) {
   // The shared-memory size attribute belongs to the kernel on each device: set it once per
   // device (one process may drive several GPUs, from several threads).
   constexpr int kMaxDev = 64;
@@ -645,18 +685,19 @@ static cudaError_t launch_d(const void* tmQ, const void* tmK, const void* tmV, c
   }
   hla_fwd_kernel<D, QK8><<<grid, kThreads, smem, st>>>(*static_cast<const CUtensorMap*>(tmQ),
                                                         *static_cast<const CUtensorMap*>(tmK),
-                                                        *static_cast<const CUtensorMap*>(tmV), p);
+                                                        *static_cast<const CUtensorMap*>(tmV), *hm,
+                                                        p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_hla_fwd(const void* tmQ, const void* tmK, const void* tmV, const FwdParams& p,
-                           int D, int qk8, int grid, cudaStream_t st) {
+cudaError_t launch_hla_fwd(const void* tmQ, const void* tmK, const void* tmV, const HaloMaps* hm,
+                           const FwdParams& p, int D, int qk8, int grid, cudaStream_t st) {
   if (qk8) {
     if (D != 128) return cudaErrorInvalidValue;
-    return launch_d<128, true>(tmQ, tmK, tmV, p, grid, st);
+    return launch_d<128, true>(tmQ, tmK, tmV, hm, p, grid, st);
   }
-  return D == 128 ? launch_d<128, false>(tmQ, tmK, tmV, p, grid, st)
-                  : launch_d<64, false>(tmQ, tmK, tmV, p, grid, st);
+  return D == 128 ? launch_d<128, false>(tmQ, tmK, tmV, hm, p, grid, st)
+                  : launch_d<64, false>(tmQ, tmK, tmV, hm, p, grid, st);
 }
 
 }  // namespace ug

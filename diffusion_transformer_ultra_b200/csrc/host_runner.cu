@@ -74,7 +74,7 @@ int ultragen_host_runner_create(ultragen_plan_t* p, int batch, int heads_per_chu
   *out = nullptr;
   if (!p || batch < 1 || heads_per_chunk < 1) return ULTRAGEN_ERR_INVALID_ARG;
   const int hpc = std::min(heads_per_chunk, p->heads);
-  if ((int64_t)hpc * p->N_kv >= ((int64_t)1 << 31) ||
+  if ((int64_t)hpc * p->kv_rows >= ((int64_t)1 << 31) ||
       (int64_t)hpc * p->N_raster >= ((int64_t)1 << 31) ||
       (int64_t)hpc * (int64_t)p->items.size() >= ((int64_t)1 << 31))
     return ULTRAGEN_ERR_UNSUPPORTED;
@@ -88,8 +88,8 @@ int ultragen_host_runner_create(ultragen_plan_t* p, int batch, int heads_per_chu
   cudaGetDevice(&r->device);
   r->stage_elems = (size_t)p->N_raster * hpc * p->D;
   const size_t stage_bytes = r->stage_elems * 2;
-  r->kv_rows = p->N_kv;
-  const size_t perm_bytes = (size_t)hpc * p->N_kv * p->D * 2;   // Q uses the first N_tot rows
+  r->kv_rows = p->kv_rows;
+  const size_t perm_bytes = (size_t)hpc * p->kv_rows * p->D * 2;   // Q uses the first N_tot rows
   r->ws_bytes = std::max<size_t>(ug::split_workspace_bytes(p, hpc), 16);
   cudaError_t e = cudaSuccess;
   for (auto& set : r->in_stage)
@@ -129,7 +129,7 @@ int ultragen_host_runner_forward(ultragen_host_runner_t* r, const void* q, const
   int st = ug::ensure_device_tables(p);   // a no-op unless the plan changed since creation
   if (st) return st;
   // a split schedule changed after creation may need more partial storage than was allocated
-  if (ug::split_workspace_bytes(p, r->hpc) > r->ws_bytes || p->N_kv > r->kv_rows)
+  if (ug::split_workspace_bytes(p, r->hpc) > r->ws_bytes || p->kv_rows > r->kv_rows)
     return ULTRAGEN_ERR_PLAN_MISMATCH;
   const cudaStream_t user = reinterpret_cast<cudaStream_t>(stream);
   const int H = p->heads, D = p->D;

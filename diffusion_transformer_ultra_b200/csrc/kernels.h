@@ -88,7 +88,13 @@ struct FwdParams {
   const int32_t* item_order = nullptr;
   int total_items;
   int N_tot;                       // Q / O rows per (batch, head)
-  int N_kv;                        // K / V rows per (batch, head)
+  int N_kv;                        // K / V rows per (batch, head) in the buffers
+  int n_ktiles = 0;                // key tiles the entries may name (the halo blocks' included)
+  // gathered halo tiles (halo mode 2; null otherwise): key tiles from halo_tile0 on are the
+  // halo blocks' tiles, halo_gtiles per window, assembled from the window segment with the
+  // copies of halo_ops (CSR per tile of a block, then one packed word per copy)
+  const int32_t* halo_ops = nullptr;
+  int halo_tile0 = 0, halo_gtiles = 1, nWh = 1, nWw = 1, n_halo_ops = 0;
   int off_hr;
   int l2;                          // l * l
   int n_ws_head;
@@ -133,7 +139,13 @@ int sm_count();
 cudaError_t launch_warm_start(const WarmArgs& a, cudaStream_t st);
 // Launches the block-sparse attention kernel; tensor maps are built by the caller.
 // qk8 = 1: tmQ and tmK are byte maps of e4m3 Q and K (D = 128 only).
+// Window views of K (0-2) and V (3-5) with the b x l, l x b and b x b piece boxes of the
+// gathered halo tiles (unused without them).
+struct HaloMaps {
+  CUtensorMap m[6];
+};
 cudaError_t launch_hla_fwd(const void* tmQ, const void* tmK, const void* tmV,
-                           const FwdParams& p, int D, int qk8, int grid, cudaStream_t st);
+                           const HaloMaps* halo, const FwdParams& p, int D, int qk8, int grid,
+                           cudaStream_t st);
 
 }  // namespace ug

@@ -81,7 +81,7 @@ extern "C" int ultragen_hla_forward_noalloc(const void* qp, const void* kp, cons
   const void* ptrs[] = {qp, kp, vp, op};
   for (const void* x : ptrs)
     if (!aligned16(x)) return ULTRAGEN_ERR_INVALID_ARG;
-  const int64_t rows = (int64_t)batch * p->heads * p->N_kv;
+  const int64_t rows = (int64_t)batch * p->heads * p->kv_rows;
   const int64_t items = (int64_t)batch * p->heads * (int64_t)p->items.size();
   if (rows >= ((int64_t)1 << 31) || items >= ((int64_t)1 << 31)) return ULTRAGEN_ERR_UNSUPPORTED;
 

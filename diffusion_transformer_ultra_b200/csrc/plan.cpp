@@ -89,15 +89,23 @@ void add_range(std::vector<int>& v, int64_t s_begin, int64_t s_end) {
   for (int64_t t = s_begin / kTile; t <= (s_end - 1) / kTile; ++t) v.push_back((int)t);
 }
 
-// Window w's halo (R18): the HR tokens of its grown box outside the window, raster order.
+// Window w's halo block (R18): eight pieces of its grown box outside the window -- the top and
+// bottom strips (b x l), the left and right strips (l x b), then the top-left, top-right,
+// bottom-left and bottom-right corners (b x b) -- each in raster order, at the slot offsets of
+// ug::halo_pieces.  f(slot in the block, i, j, real) for every piece position; positions
+// outside the image are pad slots.
 template <typename F>
-void for_each_halo_token(const ultragen_plan_t* p, int w, F&& f) {
+void for_each_halo_slot(const ultragen_plan_t* p, int w, F&& f) {
   const int wr = w / p->nWw, wc = w % p->nWw;
-  const int r0 = std::max(0, wr * p->l - p->b), r1 = std::min(p->H, (wr + 1) * p->l + p->b);
-  const int c0 = std::max(0, wc * p->l - p->b), c1 = std::min(p->W, (wc + 1) * p->l + p->b);
-  for (int i = r0; i < r1; ++i)
-    for (int j = c0; j < c1; ++j)
-      if (i / p->l != wr || j / p->l != wc) f(i, j);
+  const std::array<ug::HaloPiece, 8> pc = ug::halo_pieces(p->l, p->b);
+  for (const ug::HaloPiece& q : pc) {
+    const int i0 = wr * p->l + q.di, j0 = wc * p->l + q.dj;
+    for (int a = 0; a < q.nr; ++a)
+      for (int c = 0; c < q.nc; ++c) {
+        const int i = i0 + a, j = j0 + c;
+        f(q.off + (int64_t)a * q.nc + c, i, j, i >= 0 && i < p->H && j >= 0 && j < p->W);
+      }
+  }
 }
 
 int build_tables_mode(ultragen_plan_t* p, int halo, int lr_block);
@@ -126,20 +134,17 @@ int build_tables(ultragen_plan_t* p) {
   }
   if (p->halo_req == 0 || p->b == 0) return build_tables_mode(p, 0, lrb);
   if (p->halo_req == 1) return build_tables_mode(p, 1, lrb);
+  if (p->halo_req == 2) {
+    if (!ug::halo_gather_supported(p->l, p->b, p->qk_format)) return ULTRAGEN_ERR_UNSUPPORTED;
+    return build_tables_mode(p, 2, lrb);
+  }
   int st = build_tables_mode(p, 0, lrb);
   if (st) return st;
   // entries the halo blocks would replace: each HR query tile's neighbour-window tiles give way
   // to its windows' halo tiles
   const int64_t l2 = (int64_t)p->l * p->l;
-  std::vector<int> halo_tiles(p->nWh * p->nWw);
-  int64_t g_max = 0;
-  for (int w = 0; w < p->nWh * p->nWw; ++w) {
-    int64_t n = 0;
-    for_each_halo_token(p, w, [&](int, int) { ++n; });
-    halo_tiles[w] = (int)((n + kTile - 1) / kTile);
-    g_max = std::max(g_max, n);
-  }
-  const int64_t G = (g_max + kTile - 1) / kTile * kTile;
+  const int64_t G = ug::halo_block_slots(p->l, p->b);
+  std::vector<int> halo_tiles(p->nWh * p->nWw, (int)(G / kTile));
   int64_t saved = 0;
   for (int t = (int)(p->off_hr / kTile); t < (int)(p->off_lr / kTile); ++t) {
     if (p->qt_wfirst[t] < 0) continue;
@@ -152,8 +157,12 @@ int build_tables(ultragen_plan_t* p) {
     }
     for (int c = 0; c < C; ++c) saved -= halo_tiles[wf + c];
   }
+  // gathered halo tiles cost the permute nothing: take them whenever they save entries; copied
+  // blocks only when the saved entries outweigh the copies
+  const bool gather = ug::halo_gather_supported(p->l, p->b, p->qk_format);
   const double copy_tiles = (double)p->nWh * p->nWw * (G / kTile);
-  if ((double)saved > 3.3 * copy_tiles) return build_tables_mode(p, 1, lrb);
+  if (gather ? saved > 0 : (double)saved > 3.3 * copy_tiles)
+    return build_tables_mode(p, gather ? 2 : 1, lrb);
   return ULTRAGEN_OK;
 }
 
@@ -177,18 +186,12 @@ int build_tables_mode(ultragen_plan_t* p, int halo, int lr_block) {
   p->n_qtiles = (int)(p->N_tot / kTile);
   const int nW = p->nWh * p->nWw;
   p->halo_copy = halo;
-  p->G = 0;
-  if (halo) {
-    int64_t g_max = 0;
-    for (int w = 0; w < nW; ++w) {
-      int64_t n = 0;
-      for_each_halo_token(p, w, [&](int, int) { ++n; });
-      g_max = std::max(g_max, n);
-    }
-    p->G = (g_max + kTile - 1) / kTile * kTile;
-  }
+  p->G = halo ? ug::halo_block_slots(p->l, p->b) : 0;
   p->off_halo = p->N_tot;
   p->N_kv = p->N_tot + (int64_t)nW * p->G;
+  // gathered halo blocks (mode 2) exist only as tiles the attention assembles: the K/V buffers
+  // hold the N_tot window-first slots
+  p->kv_rows = halo == 2 ? p->N_tot : p->N_kv;
   if (p->N_kv > (int64_t)1 << 30) return ULTRAGEN_ERR_UNSUPPORTED;
 
   const int64_t N = p->N_kv;
@@ -222,17 +225,21 @@ int build_tables_mode(ultragen_plan_t* p, int halo, int lr_block) {
       p->slot_pos[s] = ((uint32_t)i << 16) | (uint32_t)j;
     }
   }
-  // compact halo blocks of K/V (R18): window w's halo tokens at off_halo + w * G, and for the
-  // permute, each window-segment slot's list of halo-block copies (CSR)
+  // compact halo blocks of K/V (R18): window w's block at off_halo + w * G; with copied blocks
+  // (mode 1), for the permute, each window-segment slot's list of halo-block copies (CSR) and
+  // the blocks' pad slots
   p->halo_ptr.clear();
   p->halo_dst.clear();
   p->halo_pad.clear();
+  p->halo_ops.clear();
+  if (halo == 2) p->halo_ops = ug::halo_gather_ops(p->l, p->b);
   if (halo) {
     std::vector<int32_t> count(p->N_hrp + 1, 0);
     for (int w = 0; w < nW; ++w) {
-      int64_t s = p->off_halo + (int64_t)w * p->G;
-      for_each_halo_token(p, w, [&](int i, int j) {
-        const int64_t r = p->T + (int64_t)i * p->W + j;
+      const int64_t hb = p->off_halo + (int64_t)w * p->G;
+      for_each_halo_slot(p, w, [&](int64_t k, int i, int j, bool real) {
+        if (!real) return;
+        const int64_t s = hb + k, r = p->T + (int64_t)i * p->W + j;
         p->perm[s] = (int32_t)r;
         p->seg[s] = SEG_HALO;
         p->ci[s] = i;
@@ -240,21 +247,24 @@ int build_tables_mode(ultragen_plan_t* p, int halo, int lr_block) {
         p->owner[s] = w;
         p->slot_pos[s] = ((uint32_t)i << 16) | (uint32_t)j;
         ++count[p->inv_perm[r] - p->off_hr + 1];
-        ++s;
       });
-      for (; s < p->off_halo + (int64_t)(w + 1) * p->G; ++s) p->halo_pad.push_back((int32_t)s);
+      if (halo == 1)
+        for (int64_t k = 0; k < p->G; ++k)
+          if (p->perm[hb + k] < 0) p->halo_pad.push_back((int32_t)(hb + k));
     }
-    for (int64_t k = 0; k < p->N_hrp; ++k) count[k + 1] += count[k];
-    p->halo_ptr = count;
-    p->halo_dst.assign(count[p->N_hrp], -1);
-    std::vector<int32_t> fill(count.begin(), count.end() - 1);
-    for (int w = 0; w < nW; ++w) {
-      int64_t s = p->off_halo + (int64_t)w * p->G;
-      for_each_halo_token(p, w, [&](int i, int j) {
-        const int64_t r = p->T + (int64_t)i * p->W + j;
-        p->halo_dst[fill[p->inv_perm[r] - p->off_hr]++] = (int32_t)s;
-        ++s;
-      });
+    if (halo == 1) {
+      for (int64_t k = 0; k < p->N_hrp; ++k) count[k + 1] += count[k];
+      p->halo_ptr = count;
+      p->halo_dst.assign(count[p->N_hrp], -1);
+      std::vector<int32_t> fill(count.begin(), count.end() - 1);
+      for (int w = 0; w < nW; ++w) {
+        const int64_t hb = p->off_halo + (int64_t)w * p->G;
+        for_each_halo_slot(p, w, [&](int64_t k, int i, int j, bool real) {
+          if (!real) return;
+          const int64_t r = p->T + (int64_t)i * p->W + j;
+          p->halo_dst[fill[p->inv_perm[r] - p->off_hr]++] = (int32_t)(hb + k);
+        });
+      }
     }
   }
   // LR tokens at positions (rho m, rho n) ([UG-note] 关键设计 2)
@@ -619,7 +629,7 @@ int ultragen_plan_set_lr_scope(ultragen_plan_t* p, int radius) {
 }
 
 int ultragen_plan_set_halo(ultragen_plan_t* p, int mode) {
-  if (!p || mode < -1 || mode > 1) return ULTRAGEN_ERR_INVALID_ARG;
+  if (!p || mode < -1 || mode > 2) return ULTRAGEN_ERR_INVALID_ARG;
   const int old = p->halo_req;
   p->halo_req = mode;
   int st;
@@ -689,6 +699,8 @@ int ultragen_plan_info(const ultragen_plan_t* p, ultragen_plan_info_t* o) {
   o->workspace_bytes_per_head = (int64_t)p->n_split_items * 2 * ug::kTile * (p->D + 1) * 4;
   o->lr_radius = p->lr_radius;
   o->halo_copy = p->halo_copy;
+  o->kv_rows = p->kv_rows;
+  o->n_halo_ops = (int32_t)p->halo_ops.size();
   o->halo_slots_per_window = (int32_t)p->G;
   o->N_kv = p->N_kv;
   o->off_halo = p->off_halo;
@@ -711,6 +723,13 @@ int ultragen_plan_export(const ultragen_plan_t* p, int32_t* perm, int32_t* row_p
 int ultragen_plan_export_kv(const ultragen_plan_t* p, int32_t* kv_perm) {
   if (!p || !kv_perm) return ULTRAGEN_ERR_INVALID_ARG;
   std::memcpy(kv_perm, p->perm.data(), (size_t)p->N_kv * sizeof(int32_t));
+  return ULTRAGEN_OK;
+}
+
+int ultragen_plan_export_halo_ops(const ultragen_plan_t* p, int32_t* out) {
+  if (!p || !out) return ULTRAGEN_ERR_INVALID_ARG;
+  if (!p->halo_ops.empty())
+    std::memcpy(out, p->halo_ops.data(), p->halo_ops.size() * sizeof(int32_t));
   return ULTRAGEN_OK;
 }
 

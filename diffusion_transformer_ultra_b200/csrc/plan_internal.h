@@ -1,6 +1,7 @@
 // Internal plan representation shared by the host plan builder and the device entry points.
 #pragma once
 
+#include <array>
 #include <cstdint>
 #include <vector>
 
@@ -9,6 +10,99 @@
 namespace ug {
 
 constexpr int kTile = 128;          // query and key tile edge (rows / columns)
+
+// One piece of a window's halo block (R18): rows [di, di + nr) x cols [dj, dj + nc) relative
+// to the window's top-left token, stored in raster order from slot `off` of the block.
+struct HaloPiece {
+  int di, dj, nr, nc;
+  int64_t off;
+};
+
+// The eight pieces in block order -- top, bottom (b x l), left, right (l x b), top-left,
+// top-right, bottom-left, bottom-right (b x b) -- each from the next multiple of 8 slots; a
+// piece of at most 128 slots does not cross a multiple of 128 (a longer one starts on one).
+inline std::array<HaloPiece, 8> halo_pieces(int l, int b) {
+  const int sh[8][4] = {{-b, 0, b, l}, {l, 0, b, l}, {0, -b, l, b}, {0, l, l, b},
+                        {-b, -b, b, b}, {-b, l, b, b}, {l, -b, b, b}, {l, l, b, b}};
+  std::array<HaloPiece, 8> out{};
+  int64_t off = 0;
+  for (int k = 0; k < 8; ++k) {
+    const int64_t n = (int64_t)sh[k][2] * sh[k][3];
+    off = (off + 7) / 8 * 8;
+    if ((n <= kTile && off / kTile != (off + n - 1) / kTile) || (n > kTile && off % kTile))
+      off = (off / kTile + 1) * kTile;
+    out[k] = HaloPiece{sh[k][0], sh[k][1], sh[k][2], sh[k][3], off};
+    off += n;
+  }
+  return out;
+}
+
+// Slots of a halo block: its pieces, padded to a multiple of 128.
+inline int64_t halo_block_slots(int l, int b) {
+  const HaloPiece q = halo_pieces(l, b)[7];
+  return (q.off + (int64_t)q.nr * q.nc + kTile - 1) / kTile * kTile;
+}
+
+// Whether the attention can assemble the halo tiles itself from the window-first K/V (halo
+// mode 2): every piece fits one tile and starts, ends and leaves gaps on multiples of b * b
+// rows (8 at least), so that each piece is one TMA box landing on a 1 KB boundary of the
+// 128-byte-swizzled slot and the gaps can be zero-filled with b x b boxes; box sides up to 256.
+inline bool halo_gather_supported(int l, int b, int qk_format) {
+  (void)qk_format;
+  if (b < 1 || b >= l || l > 256 || (int64_t)b * b % 8 != 0) return false;
+  const std::array<HaloPiece, 8> pc = halo_pieces(l, b);
+  const int64_t unit = (int64_t)b * b;
+  for (const HaloPiece& q : pc) {
+    const int64_t n = (int64_t)q.nr * q.nc;
+    if (n > kTile || q.off % unit || n % unit) return false;
+  }
+  return true;
+}
+
+// Copy lists of gathered halo tiles (halo mode 2).  The first G/128 + 1 words bound each tile's
+// copies (CSR, indices into the same array); a copy is one word: its first row in the tile
+// (bits 0-6), box shape (7-8: 0 b x l, 1 l x b, 2 b x b), zero fill (9), source window offset
+// plus one in rows (10-11) and columns (12-13), and the box's first local row (14-21) and
+// column (22-29) in that window.  Together a tile's copies cover its 128 rows exactly: the
+// gaps between pieces and after the last are zero-filled boxes.
+inline std::vector<int32_t> halo_gather_ops(int l, int b) {
+  const std::array<HaloPiece, 8> pc = halo_pieces(l, b);
+  const int64_t G = halo_block_slots(l, b);
+  const int gt = (int)(G / kTile);
+  const auto word = [](int row, int shape, int zero, int dwr, int dwc, int i0, int j0) {
+    return (int32_t)((uint32_t)row | (uint32_t)shape << 7 | (uint32_t)zero << 9 |
+                     (uint32_t)(dwr + 1) << 10 | (uint32_t)(dwc + 1) << 12 |
+                     (uint32_t)i0 << 14 | (uint32_t)j0 << 22);
+  };
+  std::vector<std::vector<int32_t>> tiles(gt);
+  // zero boxes over rows [r0, r1) of tile t: b x l boxes while they fit, then b x b
+  const auto fill = [&](int t, int r0, int r1) {
+    while (r0 < r1) {
+      const int shape = r1 - r0 >= b * l ? 0 : 2;
+      tiles[t].push_back(word(r0, shape, 1, 0, 0, 0, 0));
+      r0 += shape == 0 ? b * l : b * b;
+    }
+  };
+  std::vector<int> cursor(gt, 0);
+  for (int k = 0; k < 8; ++k) {
+    const HaloPiece& q = pc[k];
+    const int t = (int)(q.off / kTile), r = (int)(q.off % kTile);
+    fill(t, cursor[t], r);
+    const int dwr = q.di < 0 ? -1 : (q.di >= l ? 1 : 0);
+    const int dwc = q.dj < 0 ? -1 : (q.dj >= l ? 1 : 0);
+    tiles[t].push_back(word(r, k < 2 ? 0 : (k < 4 ? 1 : 2), 0, dwr, dwc, q.di - dwr * l,
+                            q.dj - dwc * l));
+    cursor[t] = r + q.nr * q.nc;
+  }
+  for (int t = 0; t < gt; ++t) fill(t, cursor[t], kTile);
+  std::vector<int32_t> out(gt + 1);
+  for (int t = 0; t < gt; ++t) {
+    out[t] = (int32_t)out.size();
+    out.insert(out.end(), tiles[t].begin(), tiles[t].end());
+  }
+  out[gt] = (int32_t)out.size();
+  return out;
+}
 constexpr int kItemInts = 8;        // int32 fields per work item
 
 // SEG_HALO: a K/V slot of a window's compact halo block
@@ -41,6 +135,7 @@ struct DeviceTables {
   int32_t* halo_ptr = nullptr;     // halo-block copies of each window-segment slot (CSR)
   int32_t* halo_dst = nullptr;
   int32_t* halo_pad = nullptr;     // pad slots of the halo blocks
+  int32_t* halo_ops = nullptr;     // gathered halo tiles: per-tile copy lists (halo_gather_ops)
   int32_t* item_order = nullptr;   // items by decreasing key-tile count
   float* rope = nullptr;           // [max(H,W)][head_dim/2][2] (cos, sin)
   int32_t* combine = nullptr;      // CombineGroup[]
@@ -76,6 +171,9 @@ struct ultragen_plan {
   int lr_order_req = -1;
   int lr_block = 0;
   int64_t G = 0, N_kv = 0, off_halo = 0;
+  // rows per (batch, head) of the K/V buffers: N_kv, or N_tot when the attention gathers the
+  // halo tiles itself (halo_copy == 2)
+  int64_t kv_rows = 0;
   // format of the permuted Q and K: ULTRAGEN_QK_BF16, or ULTRAGEN_QK_E4M3 with the stored
   // values x * 2^-q_exp (Q) and x * 2^-k_exp (K)
   int qk_format = 0;
@@ -94,6 +192,7 @@ struct ultragen_plan {
   std::vector<int32_t> ci, cj;     // per K/V slot coordinates (HR: i,j; LR: m,n; text: t,0)
   std::vector<int32_t> owner;      // per K/V slot: window of an HR or halo slot, else -1
   std::vector<uint32_t> slot_pos;  // per K/V slot packed RoPE positions
+  std::vector<int32_t> halo_ops;   // gathered halo tiles (halo_copy == 2): halo_gather_ops(l, b)
   std::vector<int32_t> halo_ptr;   // halo blocks: CSR over window-segment slots (N_hrp + 1) of
   std::vector<int32_t> halo_dst;   //   the halo-block slots that copy the slot's token
   std::vector<int32_t> halo_pad;   // halo-block slots that hold no token (written as zeros)

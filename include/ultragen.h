@@ -83,13 +83,17 @@ typedef struct {
   int32_t n_split_items;      /* items that write split partials (per head)             */
   int64_t workspace_bytes_per_head; /* split partial storage per (batch, head)          */
   int32_t lr_radius;          /* HR -> LR scope (ultragen_plan_set_lr_scope)            */
-  int32_t halo_copy;          /* 1: K/V carry compact halo blocks (ultragen_plan_set_halo) */
+  int32_t halo_copy;          /* halo blocks (ultragen_plan_set_halo): 0 none, 1 copied by
+                                 the permute, 2 gathered by the attention              */
   int32_t halo_slots_per_window; /* G: slots of one window's halo block (0 without)      */
-  int64_t N_kv;               /* K/V slots: N_tot + nWh * nWw * G                        */
+  int64_t N_kv;               /* K/V slots the tile lists address: N_tot + nWh * nWw * G */
   int64_t off_halo;           /* first halo-block slot (= N_tot)                         */
   int32_t qk_format;          /* ULTRAGEN_QK_BF16 or ULTRAGEN_QK_E4M3                    */
   int32_t q_exp, k_exp;       /* e4m3 scale exponents (0 for bf16)                       */
   int32_t lr_block;           /* 1: LR segment in 8 x 16 blocks (ultragen_plan_set_lr_order) */
+  int64_t kv_rows;            /* rows per (batch, head) of the K/V buffers: N_kv, or N_tot
+                                 when the attention gathers the halo blocks (halo_copy 2) */
+  int32_t n_halo_ops;         /* words of ultragen_plan_export_halo_ops (0 without gathering) */
 } ultragen_plan_info_t;
 
 /* Human-readable name of a status code.  Never NULL. */
@@ -145,14 +149,24 @@ int ultragen_plan_set_lr_order(ultragen_plan_t* plan, int mode);
 
 /* Compact halo blocks in the K/V layout (no counterpart in the pages; the attention is the
  * same function).  Window w's halo -- the HR tokens of its box grown by b ([UG-note] 关键设计 1/2,
- * "adjacent boundary tokens"), clipped to the image, outside the window itself -- is copied
- * by ultragen_permute_rope, in raster order of the box, into K/V slots
- * [off_halo + w*G, off_halo + (w+1)*G), G = the largest halo padded to 128.  An HR query of
- * window w then reads its neighbours' tokens from that one dense block instead of partial
- * tiles of up to 8 neighbouring windows; nothing else sees the blocks.  mode = 1 on, 0 off,
- * -1 automatic (the default: on when the tile steps saved outweigh the copies, e.g. b = 4 with
- * l = 16; off when b = 0 or when the neighbours' tiles are all fully visible, e.g. b = l).
- * Rebuilds the tile lists; changes N_kv.  INVALID_ARG for another mode. */
+ * "adjacent boundary tokens"), outside the window itself -- forms K/V slots
+ * [off_halo + w*G, off_halo + (w+1)*G) in eight pieces: the top and bottom strips (b x l), the
+ * left and right strips (l x b) and the four corners (b x b), each in raster order from the
+ * next multiple of 8 slots, a piece of at most 128 slots never crossing a multiple of 128;
+ * piece positions outside the image are pad slots, and G is the pieces' length padded to 128.
+ * An HR query of window w then reads its neighbours' tokens from that one dense block instead
+ * of partial tiles of up to 8 neighbouring windows; nothing else sees the blocks.
+ *   mode 1: ultragen_permute_rope copies the blocks into the K/V buffers (kv_rows = N_kv).
+ *   mode 2: the blocks stay virtual: the attention assembles each halo tile itself with one
+ *           tile copy per piece from the neighbours' window-first slots (kv_rows = N_tot, no
+ *           copies).  It needs every piece within one tile and pieces, gaps and offsets on
+ *           multiples of b*b slots (at least 8), b < l <= 256 (e.g. l = 16 with b = 4 or 8);
+ *           ULTRAGEN_ERR_UNSUPPORTED otherwise.
+ *   mode 0: no blocks.  mode -1 (the default): mode 2 when it is possible and saves tile steps,
+ *           else mode 1 when the steps saved outweigh the copies (e.g. b = 4 with l = 16), else
+ *           none (always none for b = 0, and when the neighbours' tiles are all fully visible,
+ *           e.g. b = l).
+ * Rebuilds the tile lists; changes N_kv and kv_rows.  INVALID_ARG for another mode. */
 int ultragen_plan_set_halo(ultragen_plan_t* plan, int mode);
 
 /* Storage format of the permuted Q and K, and so the precision of the logits Q K^T (no
@@ -187,6 +201,16 @@ int ultragen_plan_export(const ultragen_plan_t* plan, int32_t* perm, int32_t* ro
  * N_tot entries equal perm; halo-block slots follow), -1 for pad slots.  Entries of the tile
  * lists index K/V tiles of this layout. */
 int ultragen_plan_export_kv(const ultragen_plan_t* plan, int32_t* kv_perm);
+
+/* Host copy of the copy lists of gathered halo tiles (halo_copy 2): out [n_halo_ops] int32.
+ * Words 0..G/128 bound the copies of each tile of a halo block (indices into out); each copy
+ * is one word: bits 0-6 its first row in the tile (a multiple of 8), 7-8 the box (0: b rows
+ * x l columns, 1: l x b, 2: b x b tokens), 9 zero fill, 10-11 and 12-13 the source window's
+ * offset from the block's window plus one (rows, columns), 14-21 and 22-29 the box's first
+ * row and column in that window.  A box lands as its tokens in raster order; a zero box, or
+ * one whose window lies outside the image, lands as zeros.  The copies of a tile cover its
+ * 128 rows exactly once.  n_halo_ops is 0 without gathered tiles (nothing is written). */
+int ultragen_plan_export_halo_ops(const ultragen_plan_t* plan, int32_t* out);
 
 /* Per-row visibility of query tile `qtile`: out[e][r][w] (uint32) for each of the tile's
  * entries e, rows r in [0,128), words w in [0,4); bit c%32 of word c/32 = key column c of

@@ -49,11 +49,18 @@ Readings taken where the pages are silent or garbled:
   R15 Pad slots are not tokens: never visible as keys; pad query rows output 0; tile lists
       are derived from the mask rows of real tokens only.
   R18 Optional compact halo blocks (halo_copy): the K/V layout appends, per window w, a block
-      of G slots (G = the largest halo padded to 128) holding w's halo tokens -- the HR tokens
-      of its grown box outside the window, in raster order of the box.  An HR query of window
-      w then takes the other windows' tokens of its box from w's block instead of their
-      window segments; halo blocks are visible to nothing else.  Every query sees the same
-      tokens as without them, so the attention output is the same function.
+      of G slots holding w's halo tokens -- the HR tokens of its grown box outside the window.
+      The block is eight pieces, in this order: the top and bottom strips (b rows x l
+      columns, in the window's columns), the left and right strips (l rows x b columns, in the
+      window's rows), and the top-left, top-right, bottom-left and bottom-right corners (b x b);
+      each piece is in raster order of its rectangle, starts on a multiple of 8 slots, and a
+      piece of at most 128 slots does not cross a multiple of 128 (a longer one starts on
+      one).  A piece position outside the image is a pad slot, so every window's block has the
+      same shape; G is its length padded to 128.  (A strip of a window is then a box of the
+      window-first layout, which a tile copy can fetch.)  An HR query of window w takes the
+      other windows' tokens of its box from w's block instead of their window segments; halo
+      blocks are visible to nothing else.  Every query sees the same tokens as without them,
+      so the attention output is the same function.
   R20 Optional block order of the LR segment (lr_block; a layout choice for the LR-region
       reading of R3): LR token (m, n) takes slot off_lr + ((m // 8) * nbw + n // 16) * 128 +
       (m % 8) * 16 + n % 16, nbw = ceil(w / 16), so every 128-slot tile holds one 8 x 16 block
@@ -166,11 +173,12 @@ class Geometry:
 
     @property
     def G(self) -> int:
-        """Slots of one window's halo block in the K/V layout (R18): the largest halo, padded
+        """Slots of one window's halo block in the K/V layout (R18): the packed pieces, padded
         to a multiple of 128; 0 without halo blocks."""
         if not self.halo_copy:
             return 0
-        return pad128(max(len(halo_tokens(self, w)) for w in range(self.n_windows)))
+        kind, r, c, off = halo_pieces(self)[-1]
+        return pad128(off + r * c)
 
     @property
     def off_halo(self) -> int:
@@ -303,16 +311,69 @@ def halo_tokens(g: Geometry, w: int) -> tuple:
     return tuple(out)
 
 
+# the eight pieces of a halo block, in block order: (row offset, column offset) of each
+# piece's rectangle from the window's top-left token, in units where "-b" is b before the
+# window and "l" is right after it; and its shape in (b or l) units
+HALO_PIECES = ("top", "bottom", "left", "right", "top_left", "top_right", "bottom_left",
+               "bottom_right")
+
+
+def halo_piece_rect(g: Geometry, kind: str, wr: int, wc: int):
+    """Rows [i0, i0 + nr) x cols [j0, j0 + nc) of image coordinates covered by one piece of
+    window (wr, wc)'s halo (R18); coordinates may fall outside the image."""
+    top, left = wr * g.l, wc * g.l
+    rows = {"top": (top - g.b, g.b), "bottom": (top + g.l, g.b), "left": (top, g.l),
+            "right": (top, g.l), "top_left": (top - g.b, g.b), "top_right": (top - g.b, g.b),
+            "bottom_left": (top + g.l, g.b), "bottom_right": (top + g.l, g.b)}[kind]
+    cols = {"top": (left, g.l), "bottom": (left, g.l), "left": (left - g.b, g.b),
+            "right": (left + g.l, g.b), "top_left": (left - g.b, g.b),
+            "top_right": (left + g.l, g.b), "bottom_left": (left - g.b, g.b),
+            "bottom_right": (left + g.l, g.b)}[kind]
+    return rows[0], cols[0], rows[1], cols[1]
+
+
+@functools.lru_cache(maxsize=64)
+def halo_pieces(g: Geometry):
+    """(kind, rows, cols, slot offset) of the eight pieces of a halo block (R18): each at the
+    next multiple of 8; a piece of at most 128 slots that would cross a multiple of 128 moves
+    to it, and a longer piece starts on one."""
+    out, off = [], 0
+    for kind in HALO_PIECES:
+        _, _, nr, nc = halo_piece_rect(g, kind, 0, 0)
+        n = nr * nc
+        off = -(-off // 8) * 8
+        if n > 128 or (off % 128) + n > 128:
+            off = pad128(off) if off % 128 else off
+        out.append((kind, nr, nc, off))
+        off += n
+    return tuple(out)
+
+
+@functools.lru_cache(maxsize=4096)
+def halo_layout(g: Geometry, w: int) -> tuple:
+    """Window w's halo block (R18): G entries, the raster index of the token in each slot or
+    -1 for a pad slot."""
+    wr, wc = divmod(w, g.nWw)
+    out = [-1] * g.G
+    for kind, nr, nc, off in halo_pieces(g):
+        i0, j0, _, _ = halo_piece_rect(g, kind, wr, wc)
+        for a in range(nr):
+            for c in range(nc):
+                i, j = i0 + a, j0 + c
+                if 0 <= i < g.H and 0 <= j < g.W:
+                    out[off + a * nc + c] = g.T + i * g.W + j
+    return tuple(out)
+
+
 @functools.lru_cache(maxsize=8)
 def kv_perm_map(g: Geometry) -> np.ndarray:
     """K/V slot -> raster index (-1 pad): the permuted layout, then window w's halo block at
-    off_halo + w * G holding halo_tokens(w) in order (R18)."""
+    off_halo + w * G in the piece order of halo_layout (R18)."""
     kv = np.full(g.N_kv, -1, np.int64)
     kv[:g.N_tot] = perm_map(g)
     if g.halo_copy:
         for w in range(g.n_windows):
-            toks = halo_tokens(g, w)
-            kv[g.off_halo + w * g.G:g.off_halo + w * g.G + len(toks)] = toks
+            kv[g.off_halo + w * g.G:g.off_halo + (w + 1) * g.G] = halo_layout(g, w)
     return kv
 
 

@@ -209,6 +209,60 @@ def test_plan_bit_exact_full(ffi, name, halo):
     assert p.info["useful_pairs"] == O.visible_pair_count(g)
 
 
+# shapes whose halo tiles the attention can gather (b * b a multiple of 8, pieces within one
+# tile), with partial windows at the right and bottom edges
+GATHER_GEOMS = {
+    "1k": GEOMS["1k"],
+    "l16_b8": (48, 40, 16, 8, 4, 20),
+    "l32_b4": (70, 52, 32, 4, 4, 33),
+    "l8_b4": (20, 36, 8, 4, 2, 5),
+}
+
+
+@pytest.mark.parametrize("name", sorted(GATHER_GEOMS))
+def test_plan_bit_exact_gathered_halo(ffi, name):
+    g, p = compare_plan(ffi, GATHER_GEOMS[name], halo=2)
+    assert p.info["halo_copy"] == 2 and p.info["kv_rows"] == p.info["N_tot"]
+
+
+@pytest.mark.parametrize("name", sorted(GATHER_GEOMS))
+def test_gathered_halo_tiles_assemble_the_oracle_blocks(ffi, name):
+    """Replays the attention's halo-tile copies on the host: every box is read from the window
+    segment the way the tiled copy reads it (raster order of the box; zeros for a zero box or
+    a window outside the image) and must rebuild each halo-block tile of the oracle's K/V slot
+    map token for token, every row written exactly once, every box on an 8-row boundary."""
+    geom = GATHER_GEOMS[name]
+    p = ffi.Plan(*geom, 2, 64)
+    p.set_halo(2)
+    g = O.Geometry(*geom, halo_copy=True)
+    kv, perm, ops = O.kv_perm_map(g), O.perm_map(g), p.export_halo_ops()
+    l, b, G = g.l, g.b, g.G
+    gt = G // 128
+    shapes = [(b, l), (l, b), (b, b)]                      # (rows, columns) of a box
+    assert len(ops) == p.info["n_halo_ops"] and ops[0] == gt + 1 and ops[gt] == len(ops)
+    for w in range(g.nWh * g.nWw):
+        wr, wc = divmod(w, g.nWw)
+        for t in range(gt):
+            got = np.full(128, -2, np.int64)
+            for o in range(ops[t], ops[t + 1]):
+                c = int(ops[o])
+                row, shape, zero = c & 127, (c >> 7) & 3, (c >> 9) & 1
+                sr, sc = wr + ((c >> 10) & 3) - 1, wc + ((c >> 12) & 3) - 1
+                i0, j0 = (c >> 14) & 255, (c >> 22) & 255
+                nr, nc = shapes[shape]
+                assert row % 8 == 0 and row + nr * nc <= 128
+                assert i0 + nr <= l and j0 + nc <= l
+                outside = zero or not (0 <= sr < g.nWh and 0 <= sc < g.nWw)
+                for a in range(nr):
+                    for cc in range(nc):
+                        assert got[row + a * nc + cc] == -2, "row written twice"
+                        src = g.off_hr + (sr * g.nWw + sc) * l * l + (i0 + a) * l + j0 + cc
+                        got[row + a * nc + cc] = -1 if outside else perm[src]
+            assert (got != -2).all(), "row left unwritten"
+            s0 = g.off_halo + w * G + t * 128
+            np.testing.assert_array_equal(got, kv[s0:s0 + 128], err_msg=f"window {w} tile {t}")
+
+
 def test_qk_format_argument_checks(ffi):
     """The Q/K storage format: validated on the host, kept across plan rebuilds, and the
     bf16 format carries no exponents."""
@@ -222,6 +276,7 @@ def test_qk_format_argument_checks(ffi):
     assert L.ultragen_plan_set_qk_format(p.handle, 1, 0, -33) == 1
     p.set_qk_format("e4m3", -32, 32)
     assert (p.info["qk_format"], p.info["q_exp"], p.info["k_exp"]) == (ffi.QK_E4M3, -32, 32)
+    p.set_halo(0)
     entries = p.info["n_entries"]
     p.set_halo(1)
     p.set_split(3)
@@ -237,16 +292,30 @@ def test_qk_format_argument_checks(ffi):
 
 def test_halo_mode_argument_checks_and_auto_choice(ffi):
     p = ffi.Plan(64, 64, 16, 4, 4, 512, 2, 64)
-    assert ffi.lib().ultragen_plan_set_halo(p.handle, 2) == 1
+    assert ffi.lib().ultragen_plan_set_halo(p.handle, 3) == 1
     assert ffi.lib().ultragen_plan_set_halo(p.handle, -2) == 1
     useful = p.info["useful_pairs"]
-    for mode in (0, 1, -1):
+    for mode in (0, 1, 2, -1):
         p.set_halo(mode)
         assert p.info["useful_pairs"] == useful            # the same attention either way
     p.set_halo(1)
     assert p.info["halo_copy"] == 1 and p.info["N_kv"] > p.info["N_tot"]
+    assert p.info["kv_rows"] == p.info["N_kv"]            # the permute copies the blocks
+    entries = p.info["n_entries"]
+    p.set_halo(2)
+    assert p.info["halo_copy"] == 2 and p.info["N_kv"] > p.info["N_tot"]
+    assert p.info["kv_rows"] == p.info["N_tot"]           # the attention gathers them
+    assert p.info["n_entries"] == entries                 # over the same tile lists
     p.set_halo(0)
-    assert p.info["halo_copy"] == 0 and p.info["N_kv"] == p.info["N_tot"]
+    assert p.info["halo_copy"] == 0 and p.info["N_kv"] == p.info["N_tot"] == p.info["kv_rows"]
+    # l = 16, b = 4 can be gathered, so the automatic choice gathers
+    p.set_halo(-1)
+    assert p.info["halo_copy"] == 2
+    # b = 3: a corner of 9 tokens cannot land on a 1 KB boundary; copied blocks still work
+    s = ffi.Plan(64, 64, 16, 3, 4, 512, 2, 64)
+    assert ffi.lib().ultragen_plan_set_halo(s.handle, 2) == 2
+    s.set_halo(1)
+    assert s.info["halo_copy"] == 1
     # b = l: every neighbour tile is fully visible, so the automatic choice keeps them
     q = ffi.Plan(256, 135, 16, 16, 4, 256, 2, 64)
     assert q.info["halo_copy"] == 0

@@ -92,7 +92,7 @@ def expected_fp8_inputs(wl, q, k, v, b, h, halo):
             O.round_bf16(O.permute_kv(vh, g)[0, 0]))
 
 
-@pytest.mark.parametrize("name,halo,q_exp,k_exp", [("1k", None, 0, 0), ("1k", 1, -2, 3),
+@pytest.mark.parametrize("name,halo,q_exp,k_exp", [("1k", None, 0, 0), ("1k", 1, -2, 3), ("1k", 2, 1, 0),
                                                    ("odd", 1, 1, 0), ("thin", None, 0, -1),
                                                    ("win32_rho2", None, 0, 0)])
 def test_permute_stores_e4m3_codes(ug, name, halo, q_exp, k_exp):
@@ -102,7 +102,7 @@ def test_permute_stores_e4m3_codes(ug, name, halo, q_exp, k_exp):
     heads = range(wl.heads) if wl.heads <= 3 else (0, wl.heads // 2, wl.heads - 1)
     for b in range(wl.batch):
         for h in heads:
-            xq, mq, xk, mk, ev = expected_fp8_inputs(wl, q, k, v, b, h, bool(plan.info["halo_copy"]))
+            xq, mq, xk, mk, ev = expected_fp8_inputs(wl, q, k, v, b, h, plan.info["halo_copy"] == 1)
             gq = lay.qp[b, h].to(torch.float64).cpu().numpy() * 2.0 ** q_exp
             gk = lay.kp[b, h].to(torch.float64).cpu().numpy() * 2.0 ** k_exp
             check_stored(gq, xq, mq, q_exp, f"{name} Q b={b} h={h}")

@@ -71,6 +71,11 @@ CUSTOM = {
                         batch=2, axes=(16, 24, 24)),
     "rho_exceeds": dict(name="rho_exceeds", cfg=18, H=4, W=4, l=2, b=2, rho=8, T=1, heads=1, D=128, batch=1),
     "thin": dict(name="thin", cfg=19, H=3, W=130, l=4, b=1, rho=2, T=129, heads=2, D=128, batch=1),
+    # halo tiles the attention gathers itself (b * b a multiple of 8), partial edge windows
+    "l16_b8": dict(name="l16_b8", cfg=20, H=48, W=40, l=16, b=8, rho=4, T=20, heads=2, D=128, batch=2),
+    "l32_b4": dict(name="l32_b4", cfg=21, H=70, W=52, l=32, b=4, rho=4, T=33, heads=2, D=64, batch=1,
+                   axes=(16, 24, 24)),
+    "l8_b4": dict(name="l8_b4", cfg=22, H=20, W=36, l=8, b=4, rho=2, T=5, heads=3, D=128, batch=1),
 }
 
 
@@ -117,14 +122,17 @@ def ulp_bf16(x):
 @pytest.mark.parametrize("name,halo", [("tiny", None), ("1k", None), ("ragged", None), ("odd", None),
                                        ("small_l", None), ("text_only_pad", None), ("single", None),
                                        ("win_exceeds", None), ("thin", None), ("1k", 1), ("odd", 1),
-                                       ("thin", 1)])
+                                       ("thin", 1), ("1k", 2), ("l16_b8", 2), ("l32_b4", 2),
+                                       ("l8_b4", 2)])
 def test_permute_rope_parity(ug, name, halo):
     wl = _wl(name) if name in ("tiny", "1k", "ragged") else custom(name)
     plan, (q, k, v), lay, _ = run_layer(ug, wl, halo=halo)
     heads = range(wl.heads) if wl.heads <= 3 else (0, wl.heads // 2, wl.heads - 1)
     for b in range(wl.batch):
         for h in heads:
-            eq, ek, ev, mq, mk = expected_qkv_perm(wl, q, k, v, b, h, bool(plan.info["halo_copy"]))
+            # copied halo blocks (mode 1) are part of the K/V buffers; gathered ones (mode 2)
+            # are not
+            eq, ek, ev, mq, mk = expected_qkv_perm(wl, q, k, v, b, h, plan.info["halo_copy"] == 1)
             gq, gk, gv = (to_np64(t[b, h]) for t in (lay.qp, lay.kp, lay.vp))
             np.testing.assert_array_equal(gv, ev, err_msg="V gather must be bit-exact")
             for got, exp, mag, nm in ((gq, eq, mq, "Q"), (gk, ek, mk, "K")):
@@ -167,7 +175,11 @@ def test_unpermute_inverts_permute_bitwise(ug, name):
     ("tiny", None, 1), ("1k", None, 1), ("1k", 5, 1), ("odd", 3, 1), ("small_l", None, 1),
     ("win32_rho2", None, 1), ("win_exceeds", None, 1), ("thin", 1, 1),
     # and forced off where the automatic choice takes them
-    ("win32_rho2", None, 0)])
+    ("win32_rho2", None, 0),
+    # halo tiles gathered by the attention from the window segment (the automatic choice for
+    # l = 16, b = 4), with split groups and partial edge windows; copied and no blocks beside
+    ("1k", 5, 2), ("l16_b8", None, 2), ("l16_b8", 3, 2), ("l32_b4", None, 2), ("l8_b4", None, 2),
+    ("l16_b8", None, 1), ("1k", None, 0)])
 def test_attention_full_parity(ug, name, split, halo):
     wl = _wl(name) if name in ("tiny", "1k") else custom(name)
     plan, (q, k, v), lay, o = run_layer(ug, wl, split=split, halo=halo)

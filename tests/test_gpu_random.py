@@ -70,7 +70,8 @@ def test_random_layer_parity(ug, c):
     assert plan.sync_status() == 0
     torch.cuda.synchronize()
     lrb = bool(plan.info["lr_block"])
-    g = dataclasses.replace(geometry(wl, c["r"], lrb), halo_copy=bool(plan.info["halo_copy"]))
+    # the K/V buffers hold copied halo blocks (mode 1), not gathered ones (mode 2)
+    g = dataclasses.replace(geometry(wl, c["r"], lrb), halo_copy=plan.info["halo_copy"] == 1)
     real = O.perm_map(g) >= 0
     rows = np.arange(g.N_tot)
     fwd = {"qk_format": "e4m3"} if c["qk"] == "e4m3" else {}

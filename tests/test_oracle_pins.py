@@ -555,6 +555,44 @@ def test_halo_tokens_by_whole_image_scan(geo):
 
 
 @pytest.mark.parametrize("geo", HALO_GEOMS)
+def test_halo_block_layout_by_brute_force(geo):
+    """Each window's block holds exactly its halo tokens once, at the slots a plain walk of the
+    eight pieces gives: top, bottom (b x l), left, right (l x b), the four corners (b x b),
+    each in raster order from the next multiple of 8, not crossing a multiple of 128 unless
+    longer than 128; out-of-image positions are pad slots."""
+    g = O.Geometry(*geo, halo_copy=True)
+    l, b = g.l, g.b
+    shapes = [(b, l), (b, l), (l, b), (l, b), (b, b), (b, b), (b, b), (b, b)]
+    offs, off = [], 0
+    for nr, nc in shapes:
+        while off % 8:
+            off += 1
+        if nr * nc <= 128 and off // 128 != (off + nr * nc - 1) // 128:
+            off = (off // 128 + 1) * 128
+        if nr * nc > 128 and off % 128:
+            off = (off // 128 + 1) * 128
+        offs.append(off)
+        off += nr * nc
+    assert g.G == -(-off // 128) * 128
+    for w in range(g.n_windows):
+        wr, wc = divmod(w, g.nWw)
+        T0, L0 = wr * l, wc * l
+        starts = [(T0 - b, L0), (T0 + l, L0), (T0, L0 - b), (T0, L0 + l),
+                  (T0 - b, L0 - b), (T0 - b, L0 + l), (T0 + l, L0 - b), (T0 + l, L0 + l)]
+        exp = [-1] * g.G
+        for (i0, j0), (nr, nc), o in zip(starts, shapes, offs):
+            for a in range(nr):
+                for c in range(nc):
+                    i, j = i0 + a, j0 + c
+                    if 0 <= i < g.H and 0 <= j < g.W:
+                        exp[o + a * nc + c] = g.T + i * g.W + j
+        lay = list(O.halo_layout(g, w))
+        assert lay == exp
+        real = [t for t in lay if t >= 0]
+        assert sorted(real) == sorted(O.halo_tokens(g, w)) and len(set(real)) == len(real)
+
+
+@pytest.mark.parametrize("geo", HALO_GEOMS)
 def test_halo_blocks_leave_every_query_seeing_the_same_tokens(geo):
     g0, g1 = O.Geometry(*geo), O.Geometry(*geo, halo_copy=True)
     rows = np.arange(g0.N_tot)
