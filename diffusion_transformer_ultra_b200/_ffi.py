@@ -57,7 +57,7 @@ class PlanInfo(ctypes.Structure):
         ("halo_slots_per_window", ctypes.c_int32), ("N_kv", ctypes.c_int64),
         ("off_halo", ctypes.c_int64), ("qk_format", ctypes.c_int32), ("q_exp", ctypes.c_int32),
         ("k_exp", ctypes.c_int32), ("lr_block", ctypes.c_int32), ("kv_rows", ctypes.c_int64),
-        ("n_halo_ops", ctypes.c_int32),
+        ("n_halo_ops", ctypes.c_int32), ("n_long_items", ctypes.c_int32),
     ]
 
     def as_dict(self):

@@ -33,7 +33,7 @@ void free_device(ultragen_plan_t* p) {
   DeviceTables& d = p->dev;
   void* ptrs[] = {d.items, d.entries, d.mask_off, d.mask_pool, d.perm, d.inv_perm,
                   d.slot_pos, d.halo_ptr, d.halo_dst, d.halo_pad, d.halo_ops, d.item_order, d.rope,
-                  d.combine, d.error, d.clock, d.ws};
+                  d.combine, d.error, d.clock, d.sched, d.ws};
   for (void* q : ptrs)
     if (q) cudaFree(q);
   d = DeviceTables();
@@ -82,7 +82,8 @@ int ensure_device(ultragen_plan_t* p) {
       (st = upload(&d.halo_ops, p->halo_ops)) || (st = upload(&d.item_order, p->item_order)) ||
       (st = upload(&d.rope, rope)) ||
       (st = upload(&d.combine, comb)) || (st = upload(&d.error, std::vector<int>(1, 0))) ||
-      (st = upload(&d.clock, std::vector<unsigned long long>(5, 0ull)))) {
+      (st = upload(&d.clock, std::vector<unsigned long long>(5, 0ull))) ||
+      (st = upload(&d.sched, std::vector<int>(2, 0)))) {
     free_device(p);
     return st;
   }
@@ -292,6 +293,7 @@ int launch_attention(const ultragen_plan_t* p, const void* qp, const void* kp, c
   f.ws = ws;
   f.err = p->dev.error;
   f.n_items_head = (int)p->items.size();
+  f.n_long = p->n_long_items;
   f.total_items = (int)items;
   f.N_tot = (int)p->N_tot;
   f.N_kv = (int)p->kv_rows;
@@ -318,6 +320,7 @@ int launch_attention(const ultragen_plan_t* p, const void* qp, const void* kp, c
   f.n_entries = (int)p->entries.size();
   f.n_mask_words = (int)p->mask_pool.size();
   f.clock = p->clock_record ? p->dev.clock : nullptr;
+  f.sched = p->dev.sched;
   const int grid = (int)std::min<int64_t>(items, sm_count());
   // few items per CTA: hand them out item-major, longest first, so that the last round holds
   // the short ones; otherwise head-major keeps one head's shared key tiles (its LR segment)

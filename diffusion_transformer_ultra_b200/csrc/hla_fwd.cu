@@ -73,11 +73,16 @@ struct FwdCfg {
   static constexpr int BAR_OFF = KV_OFF + NS * TILE_BYTES;
   // barrier indices
   // B_KVF / B_KVE + g: stage slot g full / empty (g < NSTG)
+  // B_IF / B_IE + s: item ring slot s full / empty (s < NIR)
+  static constexpr int NIR = 4;                     // item ring slots
   static constexpr int B_QF = 0, B_QE = 1, B_KVF = 2, B_KVE = 2 + NSTG, B_SF = 2 + 2 * NSTG,
-                       B_PF = 4 + 2 * NSTG, B_OF = 6 + 2 * NSTG, B_DRAIN = 8 + 2 * NSTG;
-  static constexpr int NBAR = 9 + 2 * NSTG;
+                       B_PF = 4 + 2 * NSTG, B_OF = 6 + 2 * NSTG, B_DRAIN = 8 + 2 * NSTG,
+                       B_IF = 9 + 2 * NSTG, B_IE = 9 + 2 * NSTG + NIR;
+  static constexpr int NBAR = 9 + 2 * NSTG + 2 * NIR;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
-  static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;   // + slack for 1024-B alignment
+  // misc words: 0 TMEM base, 1 abort flag, 2-3 unused, 4.. the item ring
+  static constexpr int RING_OFF = MISC_OFF + 16;
+  static constexpr int SMEM_BYTES = RING_OFF + 4 * NIR + 1024;   // + slack for 1024-B alignment
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA exceeds 227 KB");
   // the tile slots of stage slot g: V at 2 g, K at 2 g + 1
   static __device__ __forceinline__ uint32_t v_slot(uint32_t g) { return 2 * g; }
@@ -129,6 +134,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
+// Work items reach the roles of a CTA through a ring of NIR slots in shared memory.  The
+// producer thread takes the next item of the launch -- from the work counter (one atomic add
+// per item, so a CTA that finishes early takes more), or from the round-robin sequence
+// blockIdx.x, blockIdx.x + gridDim.x, ... without one -- writes its index, or -1 after the
+// last, into slot k % NIR and arrives on that slot's "full" barrier; the MMA thread and the
+// eight softmax warps read the slot and arrive on its "empty" barrier.
+constexpr int kRingReaders = 1 + 8;     // the MMA thread and one arrive per softmax warp
+
 // The i-th work item of the launch: its 8-int record and its (batch, head) index.
 __device__ __forceinline__ const int32_t* item_at(const FwdParams& p, int it, int& bh) {
   if (p.item_major) {
@@ -136,8 +149,16 @@ __device__ __forceinline__ const int32_t* item_at(const FwdParams& p, int it, in
     bh = it - k * p.units;
     return p.items + __ldg(p.item_order + k) * 8;
   }
-  bh = it / p.n_items_head;
-  return p.items + (it - bh * p.n_items_head) * 8;
+  const int nl = p.n_long * p.units;
+  if (it < nl) {
+    const int k = it / p.units;
+    bh = it - k * p.units;
+    return p.items + k * 8;
+  }
+  it -= nl;
+  const int nr = p.n_items_head - p.n_long;
+  bh = it / nr;
+  return p.items + (p.n_long + it - bh * nr) * 8;
 }
 
 // ------------------------------------------------------------------------ producer warp
@@ -148,7 +169,7 @@ __device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
   using C = FwdCfg<D>;
   constexpr int QK_BYTES = QK8 ? 128 * D : C::TILE_BYTES;   // one Q or K tile
   const uint32_t sQ = sbase + C::Q_OFF, sKV = sbase + C::KV_OFF, bar = sbase + C::BAR_OFF;
-  uint32_t st = 0, qi = 0;                                  // stages and Q loads issued
+  uint32_t st = 0, qi = 0, ik = 0;                          // stages, Q loads, items published
   bool ok = true;
   // one tile: e4m3 Q or K is a single [128 x 128]-byte box, bf16 D / 64 boxes of [128 x 64]
   auto load_tile = [&](const CUtensorMap* tm, bool bytes, uint32_t dst, int y, uint32_t b) {
@@ -195,7 +216,22 @@ __device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
     }
     return true;
   };
-  for (int it = blockIdx.x; it < p.total_items && ok; it += gridDim.x) {
+  while (ok) {
+    // the ik-th item of this CTA: from the counter, or round-robin
+    int it = p.sched != nullptr ? atomicAdd(p.sched, 1) : (int)(blockIdx.x + ik * gridDim.x);
+    if (it >= p.total_items) it = -1;
+    {
+      const uint32_t s = ik % C::NIR;
+      if (!mbar_wait(bar + 8 * (C::B_IE + s), ((ik / C::NIR) & 1) ^ 1, abort_flag, p.err,
+                     DEV_TIMEOUT_PRODUCER, p.timeout_ns)) {
+        ok = false;
+        break;
+      }
+      st_shared_s32(sbase + C::RING_OFF + 4 * s, it);
+      mbar_arrive(bar + 8 * (C::B_IF + s));
+      ++ik;
+    }
+    if (it < 0) break;
     int bh;
     const int32_t* I = item_at(p, it, bh);
     const int qt0 = I[0], qt1 = I[1], e0 = I[2], n = I[3] - I[2];
@@ -251,6 +287,13 @@ __device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
                 DEV_TIMEOUT_DRAIN, kDrainNs);
     if (qi > 0) mbar_wait(bar + 8 * C::B_QF, (qi - 1) & 1, nullptr, p.err, DEV_TIMEOUT_DRAIN, kDrainNs);
   }
+  // The work counter resets itself for the next launch: each CTA's producer counts itself out
+  // once it will take no more items (on the abort path too), and the last one clears both
+  // words, when no producer of this launch can take another item.
+  if (p.sched != nullptr && atomicAdd(p.sched + 1, 1) == (int)gridDim.x - 1) {
+    atomicExch(p.sched, 0);
+    atomicExch(p.sched + 1, 0);
+  }
 }
 
 // ------------------------------------------------------------------------ MMA warp
@@ -298,8 +341,15 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t tbase,
   auto wait = [&](int b, uint32_t par) {
     return mbar_wait(bar + 8 * b, par, abort_flag, p.err, DEV_TIMEOUT_MMA, p.timeout_ns);
   };
+  uint32_t ik = 0;
   bool ok = true;
-  for (int it = blockIdx.x; it < p.total_items && ok; it += gridDim.x) {
+  while (ok) {
+    const uint32_t s = ik % C::NIR;
+    if (!wait(C::B_IF + s, (ik / C::NIR) & 1)) { ok = false; break; }
+    const int it = ld_shared_s32(sbase + C::RING_OFF + 4 * s);
+    mbar_arrive(bar + 8 * (C::B_IE + s));
+    ++ik;
+    if (it < 0) break;
     int bh;
     const int32_t* I = item_at(p, it, bh);
     (void)bh;
@@ -404,9 +454,21 @@ __device__ void softmax_role(const FwdParams& p, uint32_t sbase, uint32_t tbase,
   const uint32_t tS = tbase + lane_off + (uint32_t)(t * 128);
   const uint32_t tO = tbase + lane_off + C::O_COL + (uint32_t)(t * D);
   const float scale = p.scale_log2;
-  uint32_t sc = 0, oc = 0;
+  uint32_t sc = 0, oc = 0, ik = 0;
 
-  for (int it = blockIdx.x; it < p.total_items; it += gridDim.x) {
+  for (;;) {
+    int it;
+    {
+      const uint32_t s = ik % C::NIR;
+      const bool ok = mbar_wait(bar + 8 * (C::B_IF + s), (ik / C::NIR) & 1, abort_flag, p.err,
+                                DEV_TIMEOUT_SOFTMAX, p.timeout_ns);
+      if (!__all_sync(0xffffffffu, ok)) return;
+      it = ld_shared_s32(sbase + C::RING_OFF + 4 * s);
+      __syncwarp();
+      if ((threadIdx.x & 31) == 0) mbar_arrive(bar + 8 * (C::B_IE + s));
+      ++ik;
+    }
+    if (it < 0) break;
     int bh;
     const int32_t* I = item_at(p, it, bh);
     const int qt = t ? I[1] : I[0];
@@ -607,9 +669,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(bar + 8 * C::B_QF, 1);
     mbar_init(bar + 8 * C::B_QE, 1);
-    for (int s = 0; s < C::NS; ++s) {
+    for (int s = 0; s < C::NSTG; ++s) {
       mbar_init(bar + 8 * (C::B_KVF + s), 1);
       mbar_init(bar + 8 * (C::B_KVE + s), 1);
+    }
+    for (int s = 0; s < C::NIR; ++s) {
+      mbar_init(bar + 8 * (C::B_IF + s), 1);
+      mbar_init(bar + 8 * (C::B_IE + s), kRingReaders);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar + 8 * (C::B_SF + t), 1);

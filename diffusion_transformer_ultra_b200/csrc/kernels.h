@@ -80,8 +80,11 @@ struct FwdParams {
   float* ws;                       // split partials [B*heads][n_ws_head][2][128][D+1]
   int* err;                        // device error word
   int n_items_head;
-  // work order: 0 head-major (item i of the layer is item i % n_items_head of (batch, head)
-  // i / n_items_head); 1 item-major over item_order, longest first (item i is item
+  int n_long = 0;                  // the first n_long items of each head are long groups
+  // work order: 0 head-major -- the long items of every (batch, head) first (item i < n_long *
+  // units is item i / units of (batch, head) i % units), then the rest head by head (item
+  // n_long * units + i is item n_long + i % (n_items_head - n_long) of (batch, head)
+  // i / (n_items_head - n_long)); 1 item-major over item_order, longest first (item i is item
   // item_order[i / units] of (batch, head) i % units), used when a layer has few items per CTA
   int item_major = 0;
   int units = 1;                   // batch * heads of the launch
@@ -105,6 +108,9 @@ struct FwdParams {
   int N_raster = 0, heads = 1;
   int n_entries = 0;               // table sizes for the index checks of debug builds
   int n_mask_words = 0;
+  // work counter (2 words, zero between launches; null: round-robin items): word 0 hands out
+  // item indices, word 1 counts the CTAs that are done taking them
+  int* sched = nullptr;
   // launch clock record: CTA 0 adds 1, its cycles and its nanoseconds to words 0-2, keeping
   // its start in words 3-4 (null: not recorded)
   unsigned long long* clock = nullptr;

@@ -455,12 +455,19 @@ void build_schedule(ultragen_plan_t* p) {
     chunk = p->split_req;
     threshold = chunk;
   } else if (p->split_req < 0) {
-    int longest = 0;
+    int longest = 0, longest_all = 0;
+    int64_t steps = 0;
     for (const Group& g : groups) {
       const int64_t s0 = (int64_t)g.qt0 * kTile;
       if (s0 >= p->off_hr && g.n > longest) longest = g.n;   // HR and LR groups
+      longest_all = std::max(longest_all, g.n);
+      steps += g.n;
     }
-    if (longest > 0) {
+    // The attention hands items out from a work counter, longest first, so a group needs no
+    // split unless it alone outlasts a streaming multiprocessor's share of the layer (one
+    // batch element of all heads on kPlanSMs): then a split only adds partials and a merge.
+    const bool fits = (double)longest_all * kPlanSMs <= (double)steps * p->heads;
+    if (longest > 0 && !fits) {
       chunk = std::max(longest, 8);
       threshold = 1.5 * chunk;
     }
@@ -483,6 +490,7 @@ void build_schedule(ultragen_plan_t* p) {
     it.v[7] = 0;
     return it;
   };
+  std::vector<ug::Item> split_items;
   for (const Group& g : groups) {
     if (chunk > 0 && g.n > threshold && g.n > chunk) {
       const int nsplit = cdiv(g.n, chunk);
@@ -492,13 +500,31 @@ void build_schedule(ultragen_plan_t* p) {
       for (int s = 0; s < nsplit; ++s) {
         const int e0 = g.e0 + s * cs;
         const int e1 = g.e0 + std::min(g.n, (s + 1) * cs);
-        p->items.push_back(make(g, e0, e1, p->n_split_items++));
+        split_items.push_back(make(g, e0, e1, p->n_split_items++));
       }
     } else {
       rest.push_back(make(g, g.e0, g.e0 + g.n, -1));
     }
   }
-  p->items.insert(p->items.end(), rest.begin(), rest.end());
+  // Per-head item order: long groups first (longer than the longest HR / LR group, e.g.
+  // unsplit text groups), longest first -- the head-major work order hands these out for all
+  // heads at the start of the launch instead of as each head begins -- then the split items,
+  // then the rest in query-tile order.
+  int hr_longest = 0;
+  for (const Group& g : groups)
+    if ((int64_t)g.qt0 * kTile >= p->off_hr) hr_longest = std::max(hr_longest, g.n);
+  std::stable_partition(rest.begin(), rest.end(),
+                        [&](const ug::Item& it) { return it.v[3] - it.v[2] > hr_longest; });
+  const auto long_end = std::find_if(rest.begin(), rest.end(), [&](const ug::Item& it) {
+    return it.v[3] - it.v[2] <= hr_longest;
+  });
+  std::stable_sort(rest.begin(), long_end, [](const ug::Item& a, const ug::Item& b) {
+    return a.v[3] - a.v[2] > b.v[3] - b.v[2];
+  });
+  p->n_long_items = (int)(long_end - rest.begin());
+  p->items.insert(p->items.end(), rest.begin(), long_end);
+  p->items.insert(p->items.end(), split_items.begin(), split_items.end());
+  p->items.insert(p->items.end(), long_end, rest.end());
   // longest items first, for the item-major order small layers use (ties keep the list order)
   p->item_order.resize(p->items.size());
   for (size_t i = 0; i < p->items.size(); ++i) p->item_order[i] = (int32_t)i;
@@ -701,6 +727,7 @@ int ultragen_plan_info(const ultragen_plan_t* p, ultragen_plan_info_t* o) {
   o->halo_copy = p->halo_copy;
   o->kv_rows = p->kv_rows;
   o->n_halo_ops = (int32_t)p->halo_ops.size();
+  o->n_long_items = p->n_long_items;
   o->halo_slots_per_window = (int32_t)p->G;
   o->N_kv = p->N_kv;
   o->off_halo = p->off_halo;

@@ -10,6 +10,7 @@
 namespace ug {
 
 constexpr int kTile = 128;          // query and key tile edge (rows / columns)
+constexpr int kPlanSMs = 148;       // streaming multiprocessors the split policy plans for
 
 // One piece of a window's halo block (R18): rows [di, di + nr) x cols [dj, dj + nc) relative
 // to the window's top-left token, stored in raster order from slot `off` of the block.
@@ -141,6 +142,7 @@ struct DeviceTables {
   int32_t* combine = nullptr;      // CombineGroup[]
   int* error = nullptr;            // device error word
   unsigned long long* clock = nullptr;   // launch clock record: launches, cycles, ns; 2 scratch
+  int* sched = nullptr;            // the attention's work counter (2 words, zero between launches)
   float* ws = nullptr;             // split partials
   size_t ws_bytes = 0;
 };
@@ -211,6 +213,7 @@ struct ultragen_plan {
   std::vector<ug::Item> items;               // per (batch, head)
   std::vector<ug::CombineGroup> combine;     // split groups
   int n_split_items = 0;
+  int n_long_items = 0;            // items[0, n_long_items): long groups, longest first
 
   // device
   ug::DeviceTables dev;

@@ -94,6 +94,7 @@ typedef struct {
   int64_t kv_rows;            /* rows per (batch, head) of the K/V buffers: N_kv, or N_tot
                                  when the attention gathers the halo blocks (halo_copy 2) */
   int32_t n_halo_ops;         /* words of ultragen_plan_export_halo_ops (0 without gathering) */
+  int32_t n_long_items;       /* work items of a head that are long groups, handed out first */
 } ultragen_plan_info_t;
 
 /* Human-readable name of a status code.  Never NULL. */
@@ -124,8 +125,11 @@ int ultragen_plan(int H, int W, int l, int b, int rho, int text_len, int heads,
 int ultragen_plan_set_rope(ultragen_plan_t* plan, int ax0, int ax1, int ax2, double theta);
 
 /* Split long query groups' key lists into chunks of `chunk` key tiles, merged by a
- * log-sum-exp combine.  chunk = -1: automatic (the default; chunk = the longest HR/LR
- * group, applied to groups at least 1.5x longer); chunk = 0: never split. */
+ * log-sum-exp combine.  chunk = 0: never split.  chunk = -1: automatic (the default): no
+ * split when the longest group fits one streaming multiprocessor's share of a layer of one
+ * batch element (longest * 148 <= key-tile steps of all heads), since the attention hands
+ * out work items longest first from a counter; otherwise chunk = the longest HR/LR group,
+ * applied to groups at least 1.5x longer. */
 int ultragen_plan_set_split(ultragen_plan_t* plan, int chunk);
 
 /* Scope of the LR tokens an HR query sees.  radius = -1 (default): all LR tokens, the

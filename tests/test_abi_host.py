@@ -344,12 +344,20 @@ def test_plan_4k_8k_sampled_and_pair_counts(ffi):
 
 
 def test_split_policy(ffi):
-    p = ffi.Plan(256, 256, 16, 4, 4, 512, 24, 128)
+    # 24 heads: the longest group (a text pair over all 548 key tiles) is below one SM's share
+    # of the layer (24 heads x the key-tile steps of a head / 148), so nothing is split and the
+    # two text groups of a head are its long items, handed out first
+    p24 = ffi.Plan(256, 256, 16, 4, 4, 512, 24, 128)
+    assert p24.info["split_chunk"] == 0 and p24.info["n_split_groups"] == 0
+    assert p24.info["n_long_items"] == 2
+    # one head: the text groups outlast that share and are split
+    p = ffi.Plan(256, 256, 16, 4, 4, 512, 1, 128)
     i = p.info
     # automatic chunk: the longest HR / LR query-tile list, applied to the text groups only
     _, row_ptr, _ = p.export()
     longest = int(np.diff(row_ptr)[i["off_hr"] // 128:].max())
     assert i["split_chunk"] == max(longest, 8) and i["n_split_groups"] == 2
+    assert i["n_long_items"] == 0
     p.set_split(0)
     assert p.info["n_split_groups"] == 0 and p.info["workspace_bytes_per_head"] == 0
     p.set_split(7)

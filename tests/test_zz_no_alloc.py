@@ -47,7 +47,8 @@ def test_noalloc_matches_hla_forward_bitwise_on_two_calls_in_a_row(ug):
     base = ug.WORKLOADS["1k"]
     for call in range(2):
         wl = dataclasses.replace(base, cfg=base.cfg + 100 * (call + 1), batch=2)
-        plan = ug.plan_for(wl)                 # default split: text groups write partials
+        plan = ug.plan_for(wl)
+        plan.set_split(11)                     # text groups split: their partials use the scratch
         need = plan.info["workspace_bytes_per_head"] * wl.heads * wl.batch
         assert plan.info["n_split_items"] > 0 and 0 < need <= (64 << 20)
         q, k, v = (t.cuda() for t in ug.make_qkv(wl))
@@ -61,6 +62,7 @@ def test_noalloc_refuses_a_plan_changed_after_upload(ug):
     import torch
     wl = ug.WORKLOADS["1k"]
     plan = ug.plan_for(wl)
+    plan.set_split(11)
     q, k, v = (t.cuda() for t in ug.make_qkv(wl))
     lay = ug.Layer(plan, wl.batch)
     ug.permute_rope(q, k, v, lay.qp, lay.kp, lay.vp, plan)
@@ -82,8 +84,9 @@ def test_noalloc_refuses_what_it_cannot_serve(ug):
     L = ug.lib()
     buf = torch.empty(1024, dtype=torch.bfloat16, device="cuda")
     a = buf.data_ptr()
-    # split partials beyond the fixed scratch: 8K layer, 24 heads, default split
+    # split partials beyond the fixed scratch: 8K layer, 24 heads, text groups split
     big = ug.plan_for(ug.WORKLOADS["8k"])
+    big.set_split(41)
     need = big.info["workspace_bytes_per_head"] * 24
     assert need > (64 << 20)
     assert L.ultragen_hla_forward_noalloc(a, a, a, a, big.handle, 1, None) == 2
