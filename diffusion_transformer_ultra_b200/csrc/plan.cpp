@@ -134,8 +134,12 @@ int build_tables(ultragen_plan_t* p) {
   }
   if (p->halo_req == 0 || p->b == 0) return build_tables_mode(p, 0, lrb);
   if (p->halo_req == 1) return build_tables_mode(p, 1, lrb);
+  // gathered halo tiles read a neighbour's piece as a box of its l x l slots, which needs
+  // every window whole (a partial edge window packs its tokens at the front)
+  const bool gatherable = ug::halo_gather_supported(p->l, p->b, p->qk_format) &&
+                          p->H % p->l == 0 && p->W % p->l == 0;
   if (p->halo_req == 2) {
-    if (!ug::halo_gather_supported(p->l, p->b, p->qk_format)) return ULTRAGEN_ERR_UNSUPPORTED;
+    if (!gatherable) return ULTRAGEN_ERR_UNSUPPORTED;
     return build_tables_mode(p, 2, lrb);
   }
   int st = build_tables_mode(p, 0, lrb);
@@ -159,7 +163,7 @@ int build_tables(ultragen_plan_t* p) {
   }
   // gathered halo tiles cost the permute nothing: take them whenever they save entries; copied
   // blocks only when the saved entries outweigh the copies
-  const bool gather = ug::halo_gather_supported(p->l, p->b, p->qk_format);
+  const bool gather = gatherable;
   const double copy_tiles = (double)p->nWh * p->nWw * (G / kTile);
   if (gather ? saved > 0 : (double)saved > 3.3 * copy_tiles)
     return build_tables_mode(p, gather ? 2 : 1, lrb);
@@ -214,7 +218,9 @@ int build_tables_mode(ultragen_plan_t* p, int halo, int lr_block) {
   for (int i = 0; i < p->H; ++i) {
     for (int j = 0; j < p->W; ++j) {
       const int64_t win = (int64_t)(i / p->l) * p->nWw + (j / p->l);
-      const int64_t s = p->off_hr + win * l2 + (int64_t)(i % p->l) * p->l + (j % p->l);
+      // raster order inside the window's part in the image (rows of cn tokens)
+      const int cn = std::min(p->l, p->W - (j / p->l) * p->l);
+      const int64_t s = p->off_hr + win * l2 + (int64_t)(i % p->l) * cn + (j % p->l);
       const int64_t r = p->T + (int64_t)i * p->W + j;
       p->perm[s] = (int32_t)r;
       p->inv_perm[r] = (int32_t)s;

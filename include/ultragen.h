@@ -22,12 +22,15 @@
  *
  * Sequence layout (the "permuted" layout; where the pages leave it open, the plainest reading):
  *   slots [0, T) text | pad to a multiple of 128 | HR tokens window-first (windows row-major,
- *   l*l slots each, raster order inside; partial edge windows padded) | pad to 128 |
+ *   l*l slots each, raster order inside; a partial edge window holds its tokens first, in
+ *   raster order of its part inside the image, then pad slots) | pad to 128 |
  *   LR tokens raster, or in 8 x 16 blocks of the LR grid (ultragen_plan_set_lr_order) |
  *   pad to 128.   N_tot = number of slots, a multiple of 128.
- *   K/V layout: the same N_tot slots, then, when the plan uses compact halo blocks
+ *   K/V slots: the same N_tot slots, then, when the plan uses compact halo blocks
  *   (ultragen_plan_set_halo), one block of G slots per window holding that window's halo
- *   tokens; N_kv = N_tot + nWh * nWw * G (N_kv = N_tot without blocks).  Q and O use N_tot.
+ *   tokens; N_kv = N_tot + nWh * nWw * G (N_kv = N_tot without blocks).  The K/V buffers hold
+ *   kv_rows rows per (batch, head): N_kv when the permute copies the blocks, N_tot when the
+ *   attention gathers them (ultragen_plan_info).  Q and O use N_tot.
  *   Raster layout: tokens ordered text, HR raster (row i, column j), LR raster.
  */
 #ifndef ULTRAGEN_H
@@ -163,9 +166,9 @@ int ultragen_plan_set_lr_order(ultragen_plan_t* plan, int mode);
  *   mode 1: ultragen_permute_rope copies the blocks into the K/V buffers (kv_rows = N_kv).
  *   mode 2: the blocks stay virtual: the attention assembles each halo tile itself with one
  *           tile copy per piece from the neighbours' window-first slots (kv_rows = N_tot, no
- *           copies).  It needs every piece within one tile and pieces, gaps and offsets on
- *           multiples of b*b slots (at least 8), b < l <= 256 (e.g. l = 16 with b = 4 or 8);
- *           ULTRAGEN_ERR_UNSUPPORTED otherwise.
+ *           copies).  It needs whole windows (H and W multiples of l), every piece within
+ *           one tile, and pieces, gaps and offsets on multiples of b*b slots (at least 8),
+ *           b < l <= 256 (e.g. l = 16 with b = 4 or 8); ULTRAGEN_ERR_UNSUPPORTED otherwise.
  *   mode 0: no blocks.  mode -1 (the default): mode 2 when it is possible and saves tile steps,
  *           else mode 1 when the steps saved outweigh the copies (e.g. b = 4 with l = 16), else
  *           none (always none for b = 0, and when the neighbours' tiles are all fully visible,

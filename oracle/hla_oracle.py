@@ -43,9 +43,11 @@ Readings taken where the pages are silent or garbled:
       consecutively; pair k of an axis of width d rotates by pos * theta**(-2k/d);
       theta = 1e4; axis 0 position is always 0; text tokens sit at (0, 0, 0).
   R8  Sequence layout [text | pad | HR window-first | pad | LR | pad], every segment
-      starting on a multiple of 128; partial edge windows keep l*l slots (pad slots).
+      starting on a multiple of 128; partial edge windows keep l*l slots: their tokens first,
+      in raster order of the window's part inside the image, then pad slots.
   R9  H counts rows (axis 1 <- row i), W counts columns (axis 2 <- column j).
-  R13 Windows in row-major order; raster order inside a window.
+  R13 Windows in row-major order; raster order inside a window (of its part inside the
+      image, for a partial edge window: rows of min(l, W - wc*l) tokens).
   R15 Pad slots are not tokens: never visible as keys; pad query rows output 0; tile lists
       are derived from the mask rows of real tokens only.
   R18 Optional compact halo blocks (halo_copy): the K/V layout appends, per window w, a block
@@ -225,7 +227,8 @@ def slot_of_tokens(g: Geometry) -> np.ndarray:
     """Permuted slot of every raster token (window-first order, [UG-note] 关键设计 1; R8, R13).
 
     HR token (i, j) lies in window (i // l, j // l); windows are numbered row-major and
-    tokens inside a window are numbered in raster order.
+    tokens inside a window are numbered in raster order of the window's part inside the
+    image, whose rows hold min(l, W - wc * l) tokens (R8, R13).
     """
     seg, ca, cb = raster_tokens(g)
     slot = np.empty(g.N_raster, np.int64)
@@ -234,7 +237,8 @@ def slot_of_tokens(g: Geometry) -> np.ndarray:
     hr = seg == HR
     i, j = ca[hr], cb[hr]
     window = (i // g.l) * g.nWw + (j // g.l)
-    slot[hr] = g.off_hr + window * g.l * g.l + (i % g.l) * g.l + (j % g.l)
+    cols = np.minimum(g.l, g.W - (j // g.l) * g.l)       # the window's columns in the image
+    slot[hr] = g.off_hr + window * g.l * g.l + (i % g.l) * cols + (j % g.l)
     lr = seg == LR
     m, n = ca[lr], cb[lr]
     if g.lr_block:

@@ -209,13 +209,13 @@ def test_plan_bit_exact_full(ffi, name, halo):
     assert p.info["useful_pairs"] == O.visible_pair_count(g)
 
 
-# shapes whose halo tiles the attention can gather (b * b a multiple of 8, pieces within one
-# tile), with partial windows at the right and bottom edges
+# shapes whose halo tiles the attention can gather (whole windows, b * b a multiple of 8,
+# pieces within one tile); their border windows take zero boxes for the pieces outside
 GATHER_GEOMS = {
     "1k": GEOMS["1k"],
-    "l16_b8": (48, 40, 16, 8, 4, 20),
-    "l32_b4": (70, 52, 32, 4, 4, 33),
-    "l8_b4": (20, 36, 8, 4, 2, 5),
+    "l16_b8": (48, 64, 16, 8, 4, 20),
+    "l32_b4": (64, 96, 32, 4, 4, 33),
+    "l8_b4": (24, 40, 8, 4, 2, 5),
 }
 
 
@@ -316,6 +316,13 @@ def test_halo_mode_argument_checks_and_auto_choice(ffi):
     assert ffi.lib().ultragen_plan_set_halo(s.handle, 2) == 2
     s.set_halo(1)
     assert s.info["halo_copy"] == 1
+    # partial edge windows (W = 72) pack their tokens at the front: no gather; copied blocks
+    # still work
+    e = ffi.Plan(64, 72, 16, 4, 4, 512, 2, 64)
+    assert e.info["halo_copy"] != 2
+    assert ffi.lib().ultragen_plan_set_halo(e.handle, 2) == 2
+    e.set_halo(1)
+    assert e.info["halo_copy"] == 1
     # b = l: every neighbour tile is fully visible, so the automatic choice keeps them
     q = ffi.Plan(256, 135, 16, 16, 4, 256, 2, 64)
     assert q.info["halo_copy"] == 0

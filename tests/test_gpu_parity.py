@@ -71,11 +71,12 @@ CUSTOM = {
                         batch=2, axes=(16, 24, 24)),
     "rho_exceeds": dict(name="rho_exceeds", cfg=18, H=4, W=4, l=2, b=2, rho=8, T=1, heads=1, D=128, batch=1),
     "thin": dict(name="thin", cfg=19, H=3, W=130, l=4, b=1, rho=2, T=129, heads=2, D=128, batch=1),
-    # halo tiles the attention gathers itself (b * b a multiple of 8), partial edge windows
-    "l16_b8": dict(name="l16_b8", cfg=20, H=48, W=40, l=16, b=8, rho=4, T=20, heads=2, D=128, batch=2),
-    "l32_b4": dict(name="l32_b4", cfg=21, H=70, W=52, l=32, b=4, rho=4, T=33, heads=2, D=64, batch=1,
+    # halo tiles the attention gathers itself (whole windows, b * b a multiple of 8); border
+    # windows take zero boxes for their pieces outside the image
+    "l16_b8": dict(name="l16_b8", cfg=20, H=48, W=64, l=16, b=8, rho=4, T=20, heads=2, D=128, batch=2),
+    "l32_b4": dict(name="l32_b4", cfg=21, H=64, W=96, l=32, b=4, rho=4, T=33, heads=2, D=64, batch=1,
                    axes=(16, 24, 24)),
-    "l8_b4": dict(name="l8_b4", cfg=22, H=20, W=36, l=8, b=4, rho=2, T=5, heads=3, D=128, batch=1),
+    "l8_b4": dict(name="l8_b4", cfg=22, H=24, W=40, l=8, b=4, rho=2, T=5, heads=3, D=128, batch=1),
 }
 
 
@@ -177,7 +178,7 @@ def test_unpermute_inverts_permute_bitwise(ug, name):
     # and forced off where the automatic choice takes them
     ("win32_rho2", None, 0),
     # halo tiles gathered by the attention from the window segment (the automatic choice for
-    # l = 16, b = 4), with split groups and partial edge windows; copied and no blocks beside
+    # l = 16, b = 4), with split groups and border windows; copied and no blocks beside
     ("1k", 5, 2), ("l16_b8", None, 2), ("l16_b8", 3, 2), ("l32_b4", None, 2), ("l8_b4", None, 2),
     ("l16_b8", None, 1), ("1k", None, 0)])
 def test_attention_full_parity(ug, name, split, halo):

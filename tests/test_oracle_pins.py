@@ -37,19 +37,19 @@ def bf_tokens(H, W, rho, T):
 
 
 def bf_slots(H, W, l, rho, T, lr_block=False):
-    """Walk the permuted sequence slot by slot: text, pad to 128, windows row-major with
-    raster order inside, pad to 128, LR raster (or, with lr_block, LR blocks of 8 rows x 16
-    columns row-major, raster order inside, out-of-grid cells as pads), pad to 128.  Returns
-    list of token keys (None for pad)."""
+    """Walk the permuted sequence slot by slot: text, pad to 128, windows row-major, each
+    holding l*l slots: the window's tokens inside the image in raster order, then pads; pad to
+    128, LR raster (or, with lr_block, LR blocks of 8 rows x 16 columns row-major, raster order
+    inside, out-of-grid cells as pads), pad to 128.  Returns list of token keys (None for
+    pad)."""
     seq = [("text", t, 0) for t in range(T)]
     while len(seq) % 128:
         seq.append(None)
     for wr in range(math.ceil(H / l)):
         for wc in range(math.ceil(W / l)):
-            for di in range(l):
-                for dj in range(l):
-                    i, j = wr * l + di, wc * l + dj
-                    seq.append(("hr", i, j) if (i < H and j < W) else None)
+            inside = [("hr", wr * l + di, wc * l + dj) for di in range(l) for dj in range(l)
+                      if wr * l + di < H and wc * l + dj < W]
+            seq.extend(inside + [None] * (l * l - len(inside)))
     while len(seq) % 128:
         seq.append(None)
     if rho and lr_block:
