@@ -17,8 +17,12 @@
  *     asynchronous on that stream; errors raised by a kernel while it runs (a wait that
  *     timed out) are read back by ultragen_sync_status().
  *   - A plan is not thread-safe: do not use one plan from two host threads or on two
- *     streams at once.  The first device call on a plan uploads its tables with a
- *     synchronous copy; make that call before any stream capture.
+ *     streams at once (its device tables, split workspace and work counter are shared by its
+ *     calls).  The first device call on a plan uploads its tables with a synchronous copy;
+ *     make that call before any stream capture.
+ *   - A plan's device tables live on one device at a time: a device call on another current
+ *     device frees them and uploads them there.  A process that drives several GPUs at once
+ *     keeps one plan per device.
  *
  * Sequence layout (the "permuted" layout; where the pages leave it open, the plainest reading):
  *   slots [0, T) text | pad to a multiple of 128 | HR tokens window-first (windows row-major,
