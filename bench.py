@@ -197,6 +197,11 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm), "source": self.source}
 
 
+# throttle reasons that void a timed region (sw_power_cap is kept: a 1 kW part hits it under
+# dense tensor work)
+SLOWDOWN_REASONS = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
+
+
 def max_over_ranks(x: float, world: int, device) -> float:
     """Largest value of x over all ranks (the job is as slow as its slowest rank)."""
     if world <= 1:
@@ -585,26 +590,36 @@ def measure_layer(ug, args, wl, world, local, rank, heads_range=None, with_e2e=F
     if plan.sync_status() != 0:
         raise RuntimeError("device error during warm-up")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler(local)
-    # the attention kernel's own clock record (SM cycles over nanoseconds of its first CTA),
-    # for the timed launches only
-    plan.set_clock_record(True)
-    plan.read_clock()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    sampler.start()
-    launches = 0
-    start.record(stream)
-    for i in range(args.steps):
-        launches += step(evs[i])
-    end.record(stream)
-    torch.cuda.synchronize()
-    clocks = sampler.stop()
-    kclock = plan.read_clock()
-    plan.set_clock_record(False)
+    def timed_steps():
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        sampler = ClockSampler(local)
+        # the attention kernel's own clock record (SM cycles over nanoseconds of its first CTA),
+        # for the timed launches only
+        plan.set_clock_record(True)
+        plan.read_clock()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        sampler.start()
+        launches = 0
+        start.record(stream)
+        for i in range(args.steps):
+            launches += step(evs[i])
+        end.record(stream)
+        torch.cuda.synchronize()
+        clocks = sampler.stop()
+        kclock = plan.read_clock()
+        plan.set_clock_record(False)
+        return evs, start, end, clocks, kclock, launches
+
+    evs, start, end, clocks, kclock, launches = timed_steps()
+    # a hardware or thermal slowdown during the timed steps voids them: time them once more
+    # (every rank together, so that all take the same collective steps)
+    slowed = sorted(set(clocks.get("reasons", [])) & SLOWDOWN_REASONS)
+    if max_over_ranks(1.0 if slowed else 0.0, world, "cuda") > 0:
+        evs, start, end, clocks, kclock, launches = timed_steps()
+        clocks["remeasured_after"] = slowed or ["another rank's slowdown"]
     clocks["kernel_sm_mhz"] = kclock["sm_mhz"]
     clocks["kernel_clock_note"] = ("hla_forward's own record: SM cycles (clock64) over nanoseconds "
                                    "(globaltimer) of its first CTA, summed over the %d timed launches"
