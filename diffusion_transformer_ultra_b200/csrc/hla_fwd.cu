@@ -586,8 +586,7 @@ __device__ void softmax_role(const FwdParams& p, uint32_t sbase, uint32_t tbase,
         lsum += part;
       }
       __syncwarp();
-      tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(&s[0]));
-      tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(&s[32]));
+      tmem_st64(tS, s);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
