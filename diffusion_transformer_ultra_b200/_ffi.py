@@ -37,7 +37,7 @@ SYMBOLS = (
     "ultragen_host_runner_destroy", "ultragen_plan_set_halo", "ultragen_plan_export_kv",
     "ultragen_plan_set_qk_format", "ultragen_plan_set_lr_order",
     "ultragen_plan_set_clock_record", "ultragen_plan_read_clock",
-    "ultragen_plan_export_halo_ops",
+    "ultragen_plan_export_halo_ops", "ultragen_plan_export_items",
 )
 
 
@@ -94,6 +94,7 @@ def lib() -> ctypes.CDLL:
     L.ultragen_plan_set_halo.argtypes = [vp, cint]
     L.ultragen_plan_export_kv.argtypes = [vp, vp]
     L.ultragen_plan_export_halo_ops.argtypes = [vp, vp]
+    L.ultragen_plan_export_items.argtypes = [vp, vp]
     L.ultragen_plan_set_qk_format.argtypes = [vp, cint, cint, cint]
     L.ultragen_plan_set_lr_order.argtypes = [vp, cint]
     L.ultragen_plan_set_clock_record.argtypes = [vp, cint]
@@ -188,6 +189,13 @@ class Plan:
         kv = np.empty(self.info["N_kv"], np.int32)
         _check("ultragen_plan_export_kv", lib().ultragen_plan_export_kv(self._h, kv.ctypes.data))
         return kv
+
+    def export_items(self):
+        """The work items of one (batch, head): [n_items, 8] int32 (qt0, qt1, e0, e1, split
+        slot, row classes, first window, 0)."""
+        items = np.zeros((max(1, self.info["n_items"]), 8), np.int32)
+        _check("ultragen_plan_export_items", lib().ultragen_plan_export_items(self._h, items.ctypes.data))
+        return items[:self.info["n_items"]]
 
     def export_halo_ops(self):
         ops = np.zeros(max(1, self.info["n_halo_ops"]), np.int32)

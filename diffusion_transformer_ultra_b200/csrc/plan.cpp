@@ -759,6 +759,13 @@ int ultragen_plan_export_kv(const ultragen_plan_t* p, int32_t* kv_perm) {
   return ULTRAGEN_OK;
 }
 
+int ultragen_plan_export_items(const ultragen_plan_t* p, int32_t* out) {
+  if (!p || !out) return ULTRAGEN_ERR_INVALID_ARG;
+  for (size_t i = 0; i < p->items.size(); ++i)
+    std::memcpy(out + i * ug::kItemInts, p->items[i].v, sizeof(p->items[i].v));
+  return ULTRAGEN_OK;
+}
+
 int ultragen_plan_export_halo_ops(const ultragen_plan_t* p, int32_t* out) {
   if (!p || !out) return ULTRAGEN_ERR_INVALID_ARG;
   if (!p->halo_ops.empty())

@@ -223,6 +223,15 @@ int ultragen_plan_export_kv(const ultragen_plan_t* plan, int32_t* kv_perm);
  * 128 rows exactly once.  n_halo_ops is 0 without gathered tiles (nothing is written). */
 int ultragen_plan_export_halo_ops(const ultragen_plan_t* plan, int32_t* out);
 
+/* Host copy of the attention's work items of one (batch, head), in the order the head-major
+ * work order takes them: out [n_items][8] int32 with, per item, its query tiles qt0 and qt1
+ * (-1: a single tile), the range [e0, e1) of entries of qt0's tile list it covers (qt1's list
+ * is identical), its split-partial slot (-1: unsplit, written straight to the output), the
+ * number of row classes of qt0 and the first window of qt0 (-1 outside the window segment), and
+ * 0.  The first n_long_items items are the long groups, longest first; the split items follow;
+ * then the rest in query-tile order.  No counterpart in the pages (a schedule). */
+int ultragen_plan_export_items(const ultragen_plan_t* plan, int32_t* out);
+
 /* Per-row visibility of query tile `qtile`: out[e][r][w] (uint32) for each of the tile's
  * entries e, rows r in [0,128), words w in [0,4); bit c%32 of word c/32 = key column c of
  * the entry's key tile visible to row r.  Rows of pad slots are 0.  `out` holds

@@ -350,6 +350,78 @@ def test_plan_4k_8k_sampled_and_pair_counts(ffi):
     assert sum(closed_form_pairs(512, 512, 16, 4, 4, 512).values()) == 4_988_354_560
 
 
+def check_schedule(p):
+    """The work items cover every query tile's key list exactly once: a paired item covers two
+    adjacent query tiles with identical lists and the same masks on every real row, a split
+    group's items partition its
+    list in order with distinct partial slots, and the long groups come first, longest first,
+    then the split items, then the rest."""
+    info = p.info
+    perm, row_ptr, entries = p.export()
+    items = p.export_items()
+    assert len(items) == info["n_items"] and (items[:, 7] == 0).all()
+    ranges = {}
+    second = set()
+    for qt0, qt1, e0, e1, ws, _, _, _ in items.tolist():
+        assert row_ptr[qt0] <= e0 <= e1 <= row_ptr[qt0 + 1]
+        ranges.setdefault(qt0, []).append((e0, e1, ws))
+        if qt1 >= 0:
+            assert qt1 == qt0 + 1
+            n = row_ptr[qt0 + 1] - row_ptr[qt0]
+            assert row_ptr[qt1 + 1] - row_ptr[qt1] == n
+            np.testing.assert_array_equal(entries[row_ptr[qt0]:row_ptr[qt0 + 1]],
+                                          entries[row_ptr[qt1]:row_ptr[qt1 + 1]])
+            # the same masks on every real row of both tiles (pad rows export as 0)
+            m0, m1 = p.rowmasks(qt0, n), p.rowmasks(qt1, n)
+            r0 = perm[qt0 * 128:(qt0 + 1) * 128] >= 0
+            r1 = perm[qt1 * 128:(qt1 + 1) * 128] >= 0
+            ref = m0[:, np.argmax(r0)]
+            assert (m0[:, r0] == ref[:, None]).all() and (m1[:, r1] == ref[:, None]).all()
+            second.add(qt1)
+    # every query tile is the first tile of exactly one group or the second tile of a pair
+    assert set(ranges) | second == set(range(info["n_qtiles"]))
+    assert not set(ranges) & second
+    slots = []
+    for qt0, rs in ranges.items():
+        rs.sort()
+        assert rs[0][0] == row_ptr[qt0] and rs[-1][1] == row_ptr[qt0 + 1]
+        assert all(a[1] == b[0] for a, b in zip(rs, rs[1:]))
+        if len(rs) > 1:
+            assert all(ws >= 0 for _, _, ws in rs)
+            slots += [ws for _, _, ws in rs]
+        else:
+            assert rs[0][2] == -1
+    assert sorted(slots) == list(range(info["n_split_items"]))
+    # order: long groups (longest first), split items, the rest
+    n = items[:, 3] - items[:, 2]
+    nl = info["n_long_items"]
+    assert (items[:nl, 4] == -1).all() and (np.diff(n[:nl]) <= 0).all()
+    rest = items[nl:]
+    split_end = int((rest[:, 4] >= 0).sum())
+    assert (rest[:split_end, 4] >= 0).all() and (rest[split_end:, 4] == -1).all()
+    if nl and split_end < len(rest):
+        assert n[:nl].min() > n[nl + split_end:].max()
+
+
+@pytest.mark.parametrize("name", ["tiny", "1k", "odd", "small_l", "no_lr_text", "win32_rho2",
+                                  "single", "win_exceeds", "thin"])
+@pytest.mark.parametrize("split", [None, 0, 3])
+def test_schedule_covers_every_query_tile_once(ffi, name, split):
+    p = ffi.Plan(*GEOMS[name], 2, 64)
+    if split is not None:
+        p.set_split(split)
+    check_schedule(p)
+
+
+@pytest.mark.parametrize("heads", [1, 24])
+def test_schedule_at_4k(ffi, heads):
+    """4K with one head splits its text groups; with 24 it splits nothing and hands the two text
+    groups out first."""
+    p = ffi.Plan(256, 256, 16, 4, 4, 512, heads, 128)
+    check_schedule(p)
+    assert (p.info["n_split_items"] > 0) == (heads == 1)
+
+
 def test_split_policy(ffi):
     # 24 heads: the longest group (a text pair over all 548 key tiles) is below one SM's share
     # of the layer (24 heads x the key-tile steps of a head / 148), so nothing is split and the
